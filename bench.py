@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the WavePrune causal-attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic inputs
+already resident in HBM:
+  * prefill, 32K context (B1, H_q 32 / H_kv 8, N 32768, d 128, theta 1e6,
+    half-split): rotate Q and K (wp_rope_apply), then wp_prefill with the
+    grouped cutoffs;
+  * decode (16 sequences, lengths U[16384, 32768], same heads): rotate the new
+    queries at position len-1, then wp_decode (split-KV + LSE combine).
+``value`` is the prefill's useful TFLOP/s (non-skipped group QK MMAs plus PV,
+counted per 128x128 tile) over the whole step time; the decode's GB/s over
+required bytes (K of in-window groups plus all of V) is reported next to it.
+Both are also given as fractions of the measured B200 peaks.
+
+``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of
+query rows per step) on the host cores, as the slow reference arm.
+
+Run: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run every rank runs an independent replica (the work is
+data-parallel over heads and sequences with no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import wp_synthetic as syn  # noqa: E402
+
+METRIC = "prefill useful TFLOP/s & decode GB/s at 32K ctx, % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+BM = BN = 128
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=40)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- setup
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_flops(N, d, Hq, B, wg):
+    """(tile-level, pair-exact) useful FLOPs of one causal prefill.
+
+    Tile level: per 128x128 causal tile, one 2*BM*BN*16 MMA per non-skipped
+    group plus the 2*BM*BN*d PV MMA. Pair exact: per pair j <= i,
+    2*16 per group with i-j <= W_g plus 2*d."""
+    import rope_period_truncated_b200 as wp
+    _, counts = wp.wp_schedule(N, BM, BN, wg, want_map=False)
+    tiles = int(counts[0].sum())
+    qk = sum(int(counts[g, 1] + counts[g, 2]) for g in range(len(wg))) * 2 * BM * BN * 16
+    pv = tiles * 2 * BM * BN * d
+    tile_level = float(qk + pv) * B * Hq
+    delta = np.arange(N, dtype=np.int64)
+    pairs = (N - delta).astype(np.float64)
+    active = (delta[:, None] <= np.asarray(wg, dtype=np.int64)[None, :]).sum(1)
+    pair_exact = float((pairs * (2 * 16 * active + 2 * d)).sum()) * B * Hq
+    dense_tile = float(tiles * (2 * BM * BN * d * 2)) * B * Hq
+    return tile_level, pair_exact, dense_tile
+
+
+def decode_required_bytes(lens, wg, B, Hq, Hkv, d):
+    """K bytes of in-window groups (32 B per group per key) plus all of V,
+    plus the query, output and LSE."""
+    lens = np.asarray(lens, dtype=np.int64)
+    wg = np.asarray(wg, dtype=np.int64)
+    per_seq = (32 * np.minimum(wg[None, :] + 1, lens[:, None])).sum(1) + 2 * d * lens
+    kv = float(per_seq.sum()) * Hkv
+    dense_kv = float((4 * d * lens).sum()) * Hkv
+    io = B * Hq * d * 2 * 2 + B * Hq * 4
+    return kv + io, dense_kv + io
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            uuid = None
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+            except Exception:
+                pass
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+            if uuid:
+                cmd += ["-i", uuid]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Path:
+    """Device buffers and launches of one hot-path step."""
+
+    def __init__(self, device):
+        import rope_period_truncated_b200 as wp
+        self.wp = wp
+        self.pw = syn.workload("long_32k")
+        self.dw = syn.workload("decode_32k")
+        pw, dw = self.pw, self.dw
+        q, k, v = syn.prefill_inputs(pw)
+        self.host_prefill = (q, k, v)
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        self.qr, self.kr = torch.empty_like(self.q), torch.empty_like(self.k)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((pw.B, pw.Hq, pw.N), dtype=torch.float32, device=device)
+        _, self.wg = wp.wp_cutoffs(pw.d, pw.theta, pw.layout, scale_all=pw.scale_all)
+        dq, kc, vc, lens = syn.decode_inputs(dw)
+        self.host_decode = (dq, lens)
+        self.dq = dq.to(device).reshape(dw.B, 1, dw.Hq, dw.d)
+        self.dqr = torch.empty_like(self.dq)
+        self.kc, self.vc = kc.to(device), vc.to(device)
+        self.lens_host = lens
+        self.lens = lens.to(device)
+        self.pos = (lens - 1).to(torch.int32).reshape(dw.B, 1).to(device)
+        self.do = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device=device)
+        self.dlse = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=device)
+        self.ws = torch.empty(wp.wp_decode_workspace_bytes(dw.B, dw.Hq, dw.d, dw.Lmax), dtype=torch.uint8,
+                              device=device)
+        _, self.dwg = wp.wp_cutoffs(dw.d, dw.theta, dw.layout)
+        self.launches_per_step = 6  # rope Q, rope K, prefill, rope q(decode), decode split, combine
+
+    def prefill(self, cut="wave"):
+        wp, pw = self.wp, self.pw
+        wp.wp_rope_apply(self.q, pw.theta, pw.layout, scale_all=pw.scale_all, out=self.qr)
+        wp.wp_rope_apply(self.k, pw.theta, pw.layout, scale_all=pw.scale_all, out=self.kr)
+        return self.prefill_only(cut)
+
+    def prefill_only(self, cut="wave"):
+        return self.wp.wp_prefill(self.qr, self.kr, self.v, self.wg if cut == "wave" else None,
+                                  self.wp.MODE_GROUPED, self.pw.layout, out=self.o, lse=self.lse)
+
+    def decode(self, cut="wave"):
+        wp, dw = self.wp, self.dw
+        wp.wp_rope_apply(self.dq, dw.theta, dw.layout, pos=self.pos, out=self.dqr)
+        return self.decode_only(cut)
+
+    def decode_only(self, cut="wave"):
+        dw = self.dw
+        return self.wp.wp_decode(self.dqr.reshape(dw.B, dw.Hq, dw.d), self.kc, self.vc, self.lens,
+                                 self.dwg if cut == "wave" else None, out=self.do, lse=self.dlse,
+                                 workspace=self.ws)
+
+
+def time_kernel(fn, iters, warmup):
+    """Median per-launch time (ms) of fn() with CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for a, b in evs:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs)
+
+
+def cpu_baseline(path: Path, target_s: float):
+    """The fp64 oracle on sampled query rows of the 32K prefill, on this
+    host's cores; returns pair-exact useful TFLOP/s of the sample."""
+    import oracle
+    pw = path.pw
+    q, k, v = path.host_prefill
+    threads = os.cpu_count() or 1
+    kr = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(
+        oracle.rope(k.double().numpy(), pw.theta, pw.layout, scale_all=pw.scale_all)))
+    vr = v.double().numpy()
+    wg = np.asarray(path.wg, dtype=np.int64)
+
+    def sample(nrows, seed):
+        g = torch.Generator().manual_seed(seed)
+        rh = torch.randint(0, pw.Hq, (nrows,), generator=g)
+        ri = torch.randint(0, pw.N, (nrows,), generator=g)
+        rb = torch.zeros(nrows, dtype=torch.int64)
+        rows = q[rb, ri, rh].unsqueeze(0).unsqueeze(2)
+        qrot = oracle.rope(rows.double().numpy(), pw.theta, pw.layout, pos=ri.numpy().reshape(1, -1),
+                           scale_all=pw.scale_all)
+        qrot = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qrot))[0, :, 0]
+        keys = ri.numpy().astype(np.int64) + 1
+        flops = 0.0
+        for n in keys:
+            delta = np.arange(n)
+            flops += float(((delta[:, None] <= wg[None, :]).sum() * 2 * 16) + n * 2 * pw.d)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qrot, (rb.numpy(), rh.numpy(), ri.numpy()), kr, vr, pw.Hq, path.wg,
+                              oracle.MODE_GROUPED, pw.layout, nthreads=threads)
+        return flops, time.perf_counter() - t0
+
+    f0, t0 = sample(32, 1)
+    nrows = int(min(8192, max(32, 32 * target_s / max(t0, 1e-3))))
+    f1, t1 = sample(nrows, 2)
+    return {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nrows} random query rows (all heads) of the 32K prefill, fp64, {t1:.1f} s"}
+
+
+def run_ours(args, rank, world, local):
+    import rope_period_truncated_b200 as wp
+    from rope_period_truncated_b200 import build as wpbuild
+    wpbuild.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    path = Path(dev)
+    peaks, peak_kind = load_peaks()
+    pw, dw = path.pw, path.dw
+    tile_flops, pair_flops, dense_tile_flops = prefill_flops(pw.N, pw.d, pw.Hq, pw.B, path.wg)
+    dec_bytes, dense_dec_bytes = decode_required_bytes(path.lens_host.numpy(), path.dwg, dw.B, dw.Hq, dw.Hkv, dw.d)
+
+    def step(evp=None, evd=None):
+        if evp is None:
+            path.prefill()
+        else:
+            wp.wp_rope_apply(path.q, pw.theta, pw.layout, scale_all=pw.scale_all, out=path.qr)
+            wp.wp_rope_apply(path.k, pw.theta, pw.layout, scale_all=pw.scale_all, out=path.kr)
+            evp[0].record()
+            path.prefill_only()
+            evp[1].record()
+        if evd is None:
+            path.decode()
+        else:
+            wp.wp_rope_apply(path.dq, dw.theta, dw.layout, pos=path.pos, out=path.dqr)
+            evd[0].record()
+            path.decode_only()
+            evd[1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if wp.wp_device_status() != 0:
+        raise RuntimeError("device status word set during warm-up")
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    K = args.steps
+    evp = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    evd = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start.record()
+    for s in range(K):
+        step(evp[s], evd[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = statistics.mean(a.elapsed_time(b) for a, b in evp)
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evd)
+    if wp.wp_device_status() != 0:
+        raise RuntimeError("device status word set during the timed steps")
+    if world > 1:
+        t = torch.tensor([total_ms, prefill_ms, decode_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms, prefill_ms, decode_ms = t.tolist()
+    ms_per_step = total_ms / K
+    value = world * tile_flops / (ms_per_step * 1e-3) / 1e12
+
+    # dense comparison: the same kernels with every cutoff infinite
+    dense = None
+    if not args.no_dense:
+        dpf = time_kernel(lambda: path.prefill_only("dense"), 5, 2)
+        ddc = time_kernel(lambda: path.decode_only("dense"), 20, 5)
+        wpf = time_kernel(lambda: path.prefill_only("wave"), 5, 2)
+        wdc = time_kernel(lambda: path.decode_only("wave"), 20, 5)
+        dense = {"prefill_ms": round(dpf, 4), "decode_ms": round(ddc, 5),
+                 "prefill_speedup": round(dpf / wpf, 4), "decode_speedup": round(ddc / wdc, 4),
+                 "prefill_dense_tflops": round(dense_tile_flops / (dpf * 1e-3) / 1e12, 2),
+                 "decode_dense_gbs": round(dense_dec_bytes / (ddc * 1e-3) / 1e9, 1)}
+
+    # end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (t.pin_memory() for t in path.host_prefill)
+        dqh = path.host_decode[0].reshape(dw.B, 1, dw.Hq, dw.d).pin_memory()
+        lensh = path.lens_host.pin_memory()
+        posh = (path.lens_host - 1).to(torch.int32).reshape(dw.B, 1).pin_memory()
+        oh = torch.empty(path.o.shape, dtype=torch.bfloat16).pin_memory()
+        lseh = torch.empty(path.lse.shape, dtype=torch.float32).pin_memory()
+        doh = torch.empty(path.do.shape, dtype=torch.bfloat16).pin_memory()
+        dlh = torch.empty(path.dlse.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            path.q.copy_(qh, non_blocking=True)
+            path.k.copy_(kh, non_blocking=True)
+            path.v.copy_(vh, non_blocking=True)
+            path.dq.copy_(dqh, non_blocking=True)
+            path.lens.copy_(lensh, non_blocking=True)
+            path.pos.copy_(posh, non_blocking=True)
+            path.prefill()
+            path.decode()
+            oh.copy_(path.o, non_blocking=True)
+            lseh.copy_(path.lse, non_blocking=True)
+            doh.copy_(path.do, non_blocking=True)
+            dlh.copy_(path.dlse, non_blocking=True)
+
+        ke = max(3, min(K, 10))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(ke):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / ke
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = t.item()
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, dqh, lensh, posh))
+        d2h = sum(t.numel() * t.element_size() for t in (oh, lseh, doh, dlh))
+        e2e = {"value": round(world * tile_flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "note": "KV cache of the decode stays resident in HBM (serving state); all per-step "
+                       "inputs and outputs cross PCIe"}
+
+    peak_t = peaks["bf16_tflops"]
+    achieved = tile_flops / (prefill_ms * 1e-3) / 1e12
+    dec_gbs = dec_bytes / (decode_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": "prefill long_32k (B1 Hq32/Hkv8 N32768 d128 theta1e6 half-split, grouped cutoffs) + "
+                        "decode_32k (16 seqs Hq32/Hkv8 d128 L~U[16384,32768]); step = rope Q,K + prefill + "
+                        "rope q + split-KV decode",
+            "l2": "inputs larger than L2 each step (384 MiB prefill Q/K/V, 2 GiB KV cache); no flush",
+            "parallelism": f"replicas x{world} (independent heads/sequences, no collective)",
+            "group_cutoffs": [int(x) for x in path.wg],
+        },
+        "roofline": {
+            "kernel": "wp_prefill (grouped, tcgen05)",
+            "bound": "tensor",
+            "achieved": round(achieved, 2),
+            "peak": peak_t,
+            "unit": "TFLOP/s",
+            "frac": round(achieved / peak_t, 4),
+            "peak_kind": f"{peak_kind} bf16 dense burst",
+            "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+            "traffic": None,
+            "kernel_ms": round(prefill_ms, 4),
+            "flops_per_launch": tile_flops,
+            "pair_exact_flops_per_launch": pair_flops,
+            "pair_exact_tflops": round(pair_flops / (prefill_ms * 1e-3) / 1e12, 2),
+        },
+        "decode": {
+            "kernel": "wp_decode (split + combine)",
+            "bound": "hbm",
+            "value": round(dec_gbs, 1),
+            "unit": "GB/s",
+            "peak": peaks["hbm_gbs"],
+            "frac": round(dec_gbs / peaks["hbm_gbs"], 4),
+            "kernel_ms": round(decode_ms, 5),
+            "required_bytes": dec_bytes,
+        },
+        "dense_comparison": dense,
+        "e2e": e2e,
+        "gpu_launches": path.launches_per_step * K,
+        "clocks": clk,
+        "paper_context": {"source": "A100 FlashWavePrune vs FlashAttention-2, d128, theta 1e6 (context only)",
+                          "prefill_speedup_32k": 1.15, "decode_speedup_32k": 1.24},
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(path, args.cpu_seconds)
+    return out
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The fp64 oracle as the reference arm: each step is a bounded sample of
+    query rows of the 32K prefill, timed on the host cores."""
+    import oracle
+    oracle.build()
+    pw = syn.workload("long_32k")
+    q, k, v = syn.prefill_inputs(pw)
+    _, wg = oracle.cutoffs(pw.d, pw.theta, pw.layout, scale_all=pw.scale_all)
+    kr = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(
+        oracle.rope(k.double().numpy(), pw.theta, pw.layout, scale_all=pw.scale_all)))
+    vr = v.double().numpy()
+    threads = os.cpu_count() or 1
+    rows_per_step = 64
+    wgl = np.asarray(wg, dtype=np.int64)
+
+    def one(seed):
+        g = torch.Generator().manual_seed(seed)
+        rh = torch.randint(0, pw.Hq, (rows_per_step,), generator=g)
+        ri = torch.randint(0, pw.N, (rows_per_step,), generator=g)
+        rb = torch.zeros(rows_per_step, dtype=torch.int64)
+        rows = q[rb, ri, rh].unsqueeze(0).unsqueeze(2)
+        qrot = oracle.rope(rows.double().numpy(), pw.theta, pw.layout, pos=ri.numpy().reshape(1, -1))
+        qrot = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qrot))[0, :, 0]
+        flops = 0.0
+        for n in ri.numpy().astype(np.int64) + 1:
+            delta = np.arange(n)
+            flops += float(((delta[:, None] <= wgl[None, :]).sum() * 2 * 16) + n * 2 * pw.d)
+        t0 = time.perf_counter()
+        oracle.attention_rows(qrot, (rb.numpy(), rh.numpy(), ri.numpy()), kr, vr, pw.Hq, wg,
+                              oracle.MODE_GROUPED, pw.layout, nthreads=threads)
+        return flops, time.perf_counter() - t0
+
+    for s in range(args.warmup):
+        one(100 + s)
+    tot_f = tot_t = 0.0
+    for s in range(args.steps):
+        f, t = one(1000 + s)
+        tot_f += f
+        tot_t += t
+    value = tot_f / tot_t / 1e12
+    sample = f"{rows_per_step} random query rows of the 32K prefill per step, fp64 oracle, {threads} threads"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill long_32k sampled rows (B1 Hq32/Hkv8 N32768 d128 theta1e6 half-split)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=torch.device("cuda", local))
+    try:
+        out = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

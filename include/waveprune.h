@@ -1,0 +1,191 @@
+/*
+ * waveprune.h — C ABI of libwaveprune.so: WavePrune causal attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * WavePrune keeps each RoPE channel's contribution to a query-key logit only
+ * while the query-key distance is within one period of that channel, and adds
+ * 0 (not -inf) otherwise. Pages cited below, by title:
+ *   [RN] "WavePrune：RoPE 通常只需一个旋转周期" — reading notes of
+ *        arXiv:2610.06963 "WavePrune: One period is often enough for RoPE".
+ *   [KC] "WavePrune：RoPE只用一个旋转周期，长文本性能反而更好".
+ *   [TW] "Guancheng Du @ducatiqwq" — the author's thread.
+ *
+ * Conventions for every call:
+ *   - Return value is a wp_status. Argument checks run on the host before any
+ *     launch; a failing check launches nothing. Launch failures give
+ *     WP_ERR_CUDA. Nothing in the library exits or aborts the process.
+ *   - Device pointers must be 16-byte aligned and tensors contiguous in the
+ *     stated layout. The caller owns every buffer and the stream; the library
+ *     allocates no device memory. Device calls are asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - A kernel that waits longer than the wait limit on one of its internal
+ *     barriers stops, records WP_ERR_TIMEOUT in a device status word and
+ *     returns; wp_device_status() reads and clears that word.
+ *   - bf16 is IEEE bfloat16 (raw 16-bit patterns); outputs round to nearest
+ *     even.
+ */
+#ifndef WAVEPRUNE_H
+#define WAVEPRUNE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WP_OK = 0,
+    WP_ERR_ARG = 1,          /* invalid argument (NULL, size, alignment, value) */
+    WP_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d_h not 64/128) */
+    WP_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+    WP_ERR_TIMEOUT = 4       /* a kernel gave up waiting on an internal barrier */
+} wp_status;
+
+/* RoPE rotation layouts. Interleaved [KC, RoPE matrix]: channel c rotates the
+ * dim pair (2c, 2c+1). Half-split: channel c rotates (c, c + d_h/2), the
+ * rotate_half convention of Llama/Qwen checkpoints. */
+enum { WP_ROPE_INTERLEAVED = 0, WP_ROPE_HALF_SPLIT = 1 };
+
+/* Logit modes. Channel mode is the exact per-channel rule [RN §2.1, Eq. (6)];
+ * grouped mode gives each 16-dim group the largest cutoff of the channels
+ * owning its dims [RN §2.3, Eq. (8); TW (6/7)]. */
+enum { WP_MODE_GROUPED = 0, WP_MODE_CHANNEL = 1 };
+
+/* A cutoff that never masks. */
+#define WP_CUTOFF_INF INT32_MAX
+
+/* Tile classes written by wp_schedule. */
+enum { WP_TILE_SKIP = 0, WP_TILE_FULL = 1, WP_TILE_BOUNDARY = 2, WP_TILE_NONE = 3 };
+
+/*
+ * wp_cutoffs — integer cutoff tables, host only, fp64.
+ * [RN §1.1, Eq. (2)-(5)]: f_c = theta^(-2c/d_h), c = 0..d_h/2-1, times any
+ * frequency scale (the cutoffs follow the scaled frequencies, [RN §1.1]).
+ * [RN §2.1, after Eq. (6)]: w_c = alpha*pi/f_c (alpha = 2: one period) and a
+ * channel is kept iff distance <= floor(w_c). [RN §2.3, Eq. (8)]: the cutoff of
+ * group g (dims [16g, 16g+16)) is the max over the channels owning its dims.
+ *   d_h          head dim, a multiple of 16 (>= 16).
+ *   theta        RoPE base, > 1.
+ *   freq_scale   host [d_h/2] per-channel multipliers of f_c, or NULL (= 1).
+ *   scale_all    uniform multiplier of f_c (e.g. 0.25 = position interpolation
+ *                by 4), finite and > 0.
+ *   alpha        period multiple, > 0 (2.0 = the pages' default).
+ *   layout       WP_ROPE_INTERLEAVED or WP_ROPE_HALF_SPLIT.
+ *   chan_cut     host out [d_h/2] (may be NULL); group_cut host out [d_h/16]
+ *                (may be NULL). Values saturate at WP_CUTOFF_INF.
+ * Touches no GPU. Errors: WP_ERR_ARG.
+ */
+int wp_cutoffs(int d_h, double theta, const double *freq_scale, double scale_all, double alpha, int layout,
+               int32_t *chan_cut, int32_t *group_cut);
+
+/*
+ * wp_rope_apply — rotate bf16 Q or K by position * f_c [KC, RoPE matrix;
+ * RN §1.1: the channel at position i rotates by i*f_c].
+ *   x, y        device bf16 [B, N, H, d_h]; y may equal x (in place), other
+ *               overlap is not allowed.
+ *   pos         device int32 [B, N] positions, or NULL: position = pos0 + t.
+ *   theta, freq_scale (host, [d_h/2] or NULL), scale_all, layout: as in
+ *               wp_cutoffs; frequencies are formed in fp64 on the host.
+ * The angle is formed and reduced modulo 2*pi in fp64, the rotation is fp32,
+ * the result rounds to bf16. d_h in {64, 128}. Errors: WP_ERR_ARG,
+ * WP_ERR_UNSUPPORTED, WP_ERR_CUDA.
+ */
+int wp_rope_apply(const void *x, void *y, int B, int N, int H, int d_h, const int32_t *pos, int pos0, double theta,
+                  const double *freq_scale, double scale_all, int layout, void *stream);
+
+/*
+ * wp_schedule — tile classes of a causal (query block, key block) grid, host
+ * only [RN §2.3, the three-row table; TW (6/7)]. For a tile holding at least
+ * one pair j <= i, the distances span [dmin, dmax]; a cutoff W marks the tile
+ * WP_TILE_SKIP if dmin > W, WP_TILE_FULL if dmax <= W, WP_TILE_BOUNDARY
+ * otherwise. Tiles with no causal pair are WP_TILE_NONE and not counted.
+ * The prefill kernel classifies its tiles with this same function.
+ *   N, BM, BN   sequence length and block sizes (> 0).
+ *   cut         host [n_cut] cutoffs (>= 0), n_cut in 1..64.
+ *   cls         host out [nqb][nkb][n_cut] uint8 (nqb = ceil(N/BM),
+ *               nkb = ceil(N/BN)), or NULL.
+ *   counts      host out [n_cut][3] int64: skip, full, boundary.
+ * Errors: WP_ERR_ARG.
+ */
+int wp_schedule(int N, int BM, int BN, const int32_t *cut, int n_cut, uint8_t *cls, int64_t *counts);
+
+/*
+ * wp_prefill — causal WavePrune attention over positions 0..N-1, so that the
+ * distance of a pair is i - j [RN §2.1, Eq. (6) and the softmax after it].
+ *   q           device bf16 [B, N, H_q, d_h], rotated.
+ *   k, v        device bf16 [B, N, H_kv, d_h], k rotated. H_q % H_kv == 0;
+ *               query head h reads KV head h / (H_q / H_kv).
+ *   o           device bf16 out [B, N, H_q, d_h].
+ *   lse         device fp32 out [B, H_q, N]: natural-log logsumexp of the
+ *               row's logits (softmax scale included), or NULL.
+ *   mode        WP_MODE_GROUPED: cut = host group_cut [d_h/16] — the fast path
+ *               (TMA loads of only the K columns of non-skipped groups, one
+ *               tcgen05 MMA per 16-dim group into TMEM, boundary groups in a
+ *               separate TMEM accumulator masked per element).
+ *               WP_MODE_CHANNEL: cut = host chan_cut [d_h/2] — exact rule,
+ *               correctness path (CUDA cores), not tuned for speed.
+ *               cut = NULL means every cutoff is WP_CUTOFF_INF (dense).
+ *   layout      rotation layout; used by channel mode to pair dims.
+ *   softmax_scale  > 0, or <= 0 for 1/sqrt(d_h) [RN §2.1, detail 3].
+ * d_h in {64, 128}. Masked channels add 0 to the logit (the pair still takes
+ * part in the softmax) [RN §2.1, detail 1]. Errors: WP_ERR_ARG,
+ * WP_ERR_UNSUPPORTED, WP_ERR_CUDA.
+ */
+int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int N, int H_q, int H_kv,
+               int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream);
+
+/*
+ * wp_decode_workspace_bytes — size of the scratch that wp_decode needs for
+ * the split-KV partial results of a batch (fp32 partial O and LSE per split).
+ */
+size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax);
+
+/*
+ * wp_decode — one new query per sequence against a KV cache, grouped cutoffs.
+ * The query sits at position lens[b]-1 and attends keys 0..lens[b]-1, key j at
+ * distance lens[b]-1-j. [RN §2.3, table row 1]: in decode a skipped group's
+ * K bytes are not read; V is read in full.
+ *   q           device bf16 [B, H_q, d_h], rotated.
+ *   kcache, vcache  device bf16 [B, H_kv, Lmax, d_h] (keys rotated).
+ *   lens        device int32 [B], each in 1..Lmax (a length outside that
+ *               range makes the kernel write NaN rows for that sequence).
+ *   group_cut   host [d_h/16] (NULL: dense).
+ *   o           device bf16 out [B, H_q, d_h]; lse device fp32 out [B, H_q]
+ *               or NULL.
+ *   workspace   device scratch of at least wp_decode_workspace_bytes(...)
+ *               bytes, 256-byte aligned; contents on entry do not matter.
+ * Split-KV: the cache is streamed in key chunks with 16-byte vector loads;
+ * each chunk's partial (O, LSE) is merged by LSE. d_h in {64, 128}.
+ * Errors: WP_ERR_ARG, WP_ERR_UNSUPPORTED, WP_ERR_CUDA.
+ */
+int wp_decode(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B, int H_q,
+              int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+              void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * wp_device_status — synchronises `stream`, then reads and clears the device
+ * status word of the current device. Returns WP_OK, WP_ERR_TIMEOUT (a kernel
+ * gave up waiting since the last call) or WP_ERR_CUDA.
+ */
+int wp_device_status(void *stream);
+
+/* wp_set_wait_limit — cycles a kernel waits on one internal barrier before it
+ * gives up (default 2e9, about one second). Values <= 0 restore the default.
+ * Returns the previous value. Host only. */
+long long wp_set_wait_limit(long long cycles);
+
+/* wp_wait_probe — launches one CTA that waits on a barrier nothing ever
+ * completes, under the current wait limit; the kernel then records
+ * WP_ERR_TIMEOUT and returns. Used to test the timeout path without faulting
+ * or hanging the GPU. Errors: WP_ERR_CUDA. */
+int wp_wait_probe(void *stream);
+
+/* wp_status_str — static description of a status code. */
+const char *wp_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WAVEPRUNE_H */

@@ -1,0 +1,254 @@
+"""WavePrune causal attention for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of ``libwaveprune.so`` (C ABI in ``include/waveprune.h``).
+Every function here only marshals arguments: tensors must already be
+contiguous, correctly typed and on the GPU; all arithmetic runs in the
+library's CUDA kernels (or, for the cutoff tables and tile schedule, in the
+library's host code). PyTorch supplies device memory and the current stream.
+There is no fallback: if the library is missing, importing a function raises.
+
+WavePrune (arXiv:2610.06963; reading notes "WavePrune：RoPE 通常只需一个旋转
+周期", §2.1 Eq. (6) and §2.3 Eq. (8)) keeps RoPE channel c's contribution to
+the logit of pair (i, j) only while i - j <= floor(2*pi/f_c); a dropped
+channel adds 0 and the pair stays in the softmax.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+__all__ = [
+    "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
+    "WavePruneError", "library_path", "load_library",
+    "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
+    "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
+]
+
+ROPE_INTERLEAVED = 0
+ROPE_HALF_SPLIT = 1
+MODE_GROUPED = 0
+MODE_CHANNEL = 1
+CUTOFF_INF = 2 ** 31 - 1
+
+WP_OK, WP_ERR_ARG, WP_ERR_UNSUPPORTED, WP_ERR_CUDA, WP_ERR_TIMEOUT = range(5)
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libwaveprune.so")
+_lib = None
+
+
+class WavePruneError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        super().__init__(f"{fn}: {wp_status_str(code)} (status {code})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libwaveprune.so (build it first with ``python -m
+    rope_period_truncated_b200.build``). Raises if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libwaveprune.so not built ({_LIB_PATH}); run python -m rope_period_truncated_b200.build")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I, D, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_double, ctypes.c_float
+    lib.wp_cutoffs.restype = I
+    lib.wp_cutoffs.argtypes = [I, D, P, D, D, I, P, P]
+    lib.wp_rope_apply.restype = I
+    lib.wp_rope_apply.argtypes = [P, P, I, I, I, I, P, I, D, P, D, I, P]
+    lib.wp_schedule.restype = I
+    lib.wp_schedule.argtypes = [I, I, I, P, I, P, P]
+    lib.wp_prefill.restype = I
+    lib.wp_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, F, P]
+    lib.wp_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.wp_decode_workspace_bytes.argtypes = [I, I, I, I]
+    lib.wp_decode.restype = I
+    lib.wp_decode.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
+    lib.wp_device_status.restype = I
+    lib.wp_device_status.argtypes = [P]
+    lib.wp_set_wait_limit.restype = ctypes.c_longlong
+    lib.wp_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.wp_wait_probe.restype = I
+    lib.wp_wait_probe.argtypes = [P]
+    lib.wp_status_str.restype = ctypes.c_char_p
+    lib.wp_status_str.argtypes = [I]
+    _lib = lib
+    return lib
+
+
+def wp_status_str(code: int) -> str:
+    return load_library().wp_status_str(int(code)).decode()
+
+
+def _check(fn: str, code: int):
+    if code != WP_OK:
+        raise WavePruneError(fn, code)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _host_i32(a, n: int | None = None):
+    if a is None:
+        return None, None
+    arr = np.ascontiguousarray(np.asarray(a), dtype=np.int32)
+    if n is not None and arr.size != n:
+        raise ValueError(f"expected {n} cutoffs, got {arr.size}")
+    return arr, arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def _host_f64(a):
+    if a is None:
+        return None, None
+    arr = np.ascontiguousarray(np.asarray(a), dtype=np.float64)
+    return arr, arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# --------------------------------------------------------------------- host
+
+def wp_cutoffs(d_h: int, theta: float, layout: int, alpha: float = 2.0, freq_scale=None, scale_all: float = 1.0):
+    """Integer cutoffs (chan_cut [d_h/2], group_cut [d_h/16]) as numpy int32."""
+    fs, fs_p = _host_f64(freq_scale)
+    wc = np.zeros(d_h // 2, dtype=np.int32)
+    wg = np.zeros(max(d_h // 16, 1), dtype=np.int32)
+    _check("wp_cutoffs", load_library().wp_cutoffs(d_h, theta, fs_p, scale_all, alpha, layout,
+                                                    wc.ctypes.data_as(ctypes.c_void_p),
+                                                    wg.ctypes.data_as(ctypes.c_void_p)))
+    return wc, wg
+
+
+def wp_schedule(N: int, BM: int, BN: int, cut, want_map: bool = True):
+    """Tile classes (cls [nqb,nkb,n] uint8 or None, counts [n,3] int64)."""
+    cut_a, cut_p = _host_i32(cut)
+    n = cut_a.size
+    nqb, nkb = -(-N // BM), -(-N // BN)
+    cls = np.empty((nqb, nkb, n), dtype=np.uint8) if want_map else None
+    counts = np.zeros((n, 3), dtype=np.int64)
+    _check("wp_schedule", load_library().wp_schedule(
+        N, BM, BN, cut_p, n, None if cls is None else cls.ctypes.data_as(ctypes.c_void_p),
+        counts.ctypes.data_as(ctypes.c_void_p)))
+    return cls, counts
+
+
+# ------------------------------------------------------------------- device
+
+def wp_rope_apply(x: torch.Tensor, theta: float, layout: int, pos: torch.Tensor | None = None, pos0: int = 0,
+                  freq_scale=None, scale_all: float = 1.0, out: torch.Tensor | None = None, stream=None):
+    """Rotate bf16 x [B,N,H,d] by position*f_c; returns ``out`` (x itself if
+    out is x; a new tensor if out is None)."""
+    _need(x, "x", torch.bfloat16, 4)
+    B, N, H, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", torch.bfloat16, 4)
+    if out.shape != x.shape:
+        raise ValueError("out shape mismatch")
+    if pos is not None:
+        _need(pos, "pos", torch.int32, 2)
+        if tuple(pos.shape) != (B, N):
+            raise ValueError("pos must be [B, N]")
+    fs, fs_p = _host_f64(freq_scale)
+    _check("wp_rope_apply", load_library().wp_rope_apply(
+        _ptr(x), _ptr(out), B, N, H, d, _ptr(pos), int(pos0), float(theta), fs_p, float(scale_all), int(layout),
+        _stream(stream)))
+    return out
+
+
+def wp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cut=None, mode: int = MODE_GROUPED,
+               layout: int = ROPE_HALF_SPLIT, softmax_scale: float = 0.0, out: torch.Tensor | None = None,
+               lse: torch.Tensor | None = None, want_lse: bool = True, stream=None):
+    """Causal WavePrune prefill. q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 (rotated).
+    ``cut``: host group cutoffs [d/16] (grouped) or channel cutoffs [d/2]
+    (channel mode), None = dense. Returns (o [B,N,Hq,d] bf16, lse [B,Hq,N] fp32)."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
+        raise ValueError("k/v shape mismatch")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 4)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    n_expected = d // 16 if mode == MODE_GROUPED else d // 2
+    cut_a, cut_p = _host_i32(cut, n_expected)
+    _check("wp_prefill", load_library().wp_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, Hq, Hkv, d, int(mode), cut_p, int(layout),
+        float(softmax_scale), _stream(stream)))
+    return out, lse
+
+
+def wp_decode_workspace_bytes(B: int, Hq: int, d_h: int, Lmax: int) -> int:
+    return int(load_library().wp_decode_workspace_bytes(B, Hq, d_h, Lmax))
+
+
+def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens: torch.Tensor, group_cut=None,
+              softmax_scale: float = 0.0, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, want_lse: bool = True, stream=None):
+    """Split-KV decode. q [B,Hq,d] (rotated), caches [B,Hkv,Lmax,d] bf16, lens
+    int32 [B] (device). Returns (o [B,Hq,d] bf16, lse [B,Hq] fp32)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(lens, "lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = kcache.shape
+    if tuple(kcache.shape) != (B, Hkv, Lmax, d) or tuple(vcache.shape) != tuple(kcache.shape):
+        raise ValueError("cache shape mismatch")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = wp_decode_workspace_bytes(B, Hq, d, Lmax)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small")
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    _check("wp_decode", load_library().wp_decode(
+        _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
+        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def wp_device_status(stream=None) -> int:
+    """Synchronise the stream, read and clear the device status word."""
+    return int(load_library().wp_device_status(_stream(stream)))
+
+
+def wp_set_wait_limit(cycles: int) -> int:
+    return int(load_library().wp_set_wait_limit(int(cycles)))
+
+
+def wp_wait_probe(stream=None):
+    _check("wp_wait_probe", load_library().wp_wait_probe(_stream(stream)))

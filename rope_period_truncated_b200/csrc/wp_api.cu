@@ -1,0 +1,312 @@
+// C ABI of libwaveprune.so: argument checks, cutoff tables, tile schedule,
+// tensor maps and kernel launches. Declarations and contracts: waveprune.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "waveprune.h"
+#include "wp_decode.h"
+#include "wp_device.cuh"
+#include "wp_prefill.h"
+#include "wp_rope.h"
+#include "wp_tile.h"
+
+namespace wp {
+
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr long long DEFAULT_WAIT_LIMIT = 2000000000LL;  // SM cycles, about one second
+long long g_wait_limit = DEFAULT_WAIT_LIMIT;
+
+constexpr double kPi = 3.14159265358979323846;
+constexpr double kLog2e = 1.4426950408889634074;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dim_supported(int d_h) { return d_h == 64 || d_h == 128; }
+
+// f_c = theta^(-2c/d_h) * freq_scale[c] * scale_all (WavePrune reading notes
+// "WavePrune：RoPE 通常只需一个旋转周期", §1.1: the cutoffs follow the scaled
+// frequencies).
+double channel_freq(int c, int d_h, double theta, const double *freq_scale, double scale_all) {
+  double f = std::pow(theta, -2.0 * static_cast<double>(c) / static_cast<double>(d_h));
+  if (freq_scale != nullptr) f *= freq_scale[c];
+  return f * scale_all;
+}
+
+bool freq_args_ok(int d_h, double theta, const double *freq_scale, double scale_all) {
+  if (!(theta > 1.0) || !std::isfinite(theta)) return false;
+  if (!(scale_all > 0.0) || !std::isfinite(scale_all)) return false;
+  if (freq_scale != nullptr)
+    for (int c = 0; c < d_h / 2; ++c)
+      if (!(freq_scale[c] > 0.0) || !std::isfinite(freq_scale[c])) return false;
+  return true;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D bf16 view (d, H, N, B) of a [B, N, H, d] tensor; box (box_d, 1, 128, 1).
+bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int d, int box_d, CUtensorMapSwizzle sw) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
+                           static_cast<cuuint64_t>(N) * H * d * 2};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? WP_OK : WP_ERR_CUDA; }
+
+__global__ void wait_probe_kernel(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, limit, nullptr);  // nothing arrives: gives up after `limit`
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace wp
+
+using namespace wp;
+
+extern "C" {
+
+int wp_cutoffs(int d_h, double theta, const double *freq_scale, double scale_all, double alpha, int layout,
+               int32_t *chan_cut, int32_t *group_cut) {
+  if (d_h < 16 || d_h % 16 != 0 || d_h > 1024) return WP_ERR_ARG;
+  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
+  if (!freq_args_ok(d_h, theta, freq_scale, scale_all) || !(alpha > 0.0)) return WP_ERR_ARG;
+  const int C = d_h / 2;
+  int32_t wc[512];
+  // WavePrune reading notes, §2.1 (after Eq. (6)): w_c = alpha*pi/f_c, and a
+  // channel is kept iff distance <= floor(w_c).
+  for (int c = 0; c < C; ++c) {
+    const double w = alpha * kPi / channel_freq(c, d_h, theta, freq_scale, scale_all);
+    const double fl = std::floor(w);
+    wc[c] = fl < 2147483647.0 ? static_cast<int32_t>(fl) : WP_CUTOFF_INF;
+  }
+  if (chan_cut != nullptr) std::memcpy(chan_cut, wc, sizeof(int32_t) * C);
+  // §2.3 Eq. (8): the group cutoff is the largest cutoff of the channels that
+  // own its 16 dims (interleaved: dim k -> channel k/2; half-split: k mod C).
+  if (group_cut != nullptr)
+    for (int g = 0; g < d_h / 16; ++g) {
+      int32_t m = 0;
+      for (int k = 16 * g; k < 16 * g + 16; ++k) {
+        const int c = layout == WP_ROPE_INTERLEAVED ? k / 2 : k % C;
+        if (wc[c] > m) m = wc[c];
+      }
+      group_cut[g] = m;
+    }
+  return WP_OK;
+}
+
+int wp_schedule(int N, int BM, int BN, const int32_t *cut, int n_cut, uint8_t *cls, int64_t *counts) {
+  if (N <= 0 || BM <= 0 || BN <= 0 || cut == nullptr || counts == nullptr || n_cut < 1 || n_cut > 64)
+    return WP_ERR_ARG;
+  for (int g = 0; g < n_cut; ++g)
+    if (cut[g] < 0) return WP_ERR_ARG;
+  const int64_t nqb = (static_cast<int64_t>(N) + BM - 1) / BM, nkb = (static_cast<int64_t>(N) + BN - 1) / BN;
+  for (int g = 0; g < 3 * n_cut; ++g) counts[g] = 0;
+  for (int64_t qb = 0; qb < nqb; ++qb)
+    for (int64_t kb = 0; kb < nkb; ++kb) {
+      int64_t dmin = 0, dmax = -1;
+      const bool causal = tile_distance_range(N, BM, BN, qb, kb, &dmin, &dmax);
+      for (int g = 0; g < n_cut; ++g) {
+        const int c = causal ? classify_cutoff(dmin, dmax, cut[g]) : TILE_NONE;
+        if (cls != nullptr) cls[(qb * nkb + kb) * n_cut + g] = static_cast<uint8_t>(c);
+        if (c != TILE_NONE) counts[3 * g + c] += 1;
+      }
+    }
+  return WP_OK;
+}
+
+int wp_rope_apply(const void *x, void *y, int B, int N, int H, int d_h, const int32_t *pos, int pos0, double theta,
+                  const double *freq_scale, double scale_all, int layout, void *stream) {
+  if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return WP_ERR_ARG;
+  if (B <= 0 || N <= 0 || H <= 0) return WP_ERR_ARG;
+  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  if (!freq_args_ok(d_h, theta, freq_scale, scale_all)) return WP_ERR_ARG;
+  if (x != y) {  // only exact in-place aliasing is allowed
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x), b0 = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t n = static_cast<uintptr_t>(B) * N * H * d_h * 2;
+    if (a0 < b0 + n && b0 < a0 + n) return WP_ERR_ARG;
+  }
+  RopeArgs a;
+  a.x = static_cast<const __nv_bfloat16 *>(x);
+  a.y = static_cast<__nv_bfloat16 *>(y);
+  a.pos = pos;
+  a.tokens = static_cast<int64_t>(B) * N;
+  a.N = N;
+  a.H = H;
+  a.pos0 = pos0;
+  for (int c = 0; c < 64; ++c) a.freq[c] = c < d_h / 2 ? channel_freq(c, d_h, theta, freq_scale, scale_all) : 0.0;
+  return from_cuda(launch_rope(a, d_h, layout, static_cast<cudaStream_t>(stream)));
+}
+
+int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int N, int H_q, int H_kv,
+               int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return WP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return WP_ERR_ARG;
+  if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return WP_ERR_ARG;
+  if (B > 65535 || H_q > 65535) return WP_ERR_UNSUPPORTED;
+  if (mode != WP_MODE_GROUPED && mode != WP_MODE_CHANNEL) return WP_ERR_ARG;
+  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  if (!std::isfinite(softmax_scale)) return WP_ERR_ARG;
+  const float scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(d_h)));
+  const float scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (mode == WP_MODE_CHANNEL) {
+    ChannelPrefillArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.k = static_cast<const __nv_bfloat16 *>(k);
+    a.v = static_cast<const __nv_bfloat16 *>(v);
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.lse = lse;
+    a.B = B;
+    a.N = N;
+    a.Hq = H_q;
+    a.Hkv = H_kv;
+    a.layout = layout;
+    for (int c = 0; c < 64; ++c) {
+      a.cut[c] = (cut == nullptr || c >= d_h / 2) ? WP_CUTOFF_INF : cut[c];
+      if (a.cut[c] < 0) return WP_ERR_ARG;
+    }
+    a.scale_log2 = scale_log2;
+    return from_cuda(launch_prefill_channel(d_h, a, s));
+  }
+
+  PrefillArgs a;
+  a.o = static_cast<__nv_bfloat16 *>(o);
+  a.lse = lse;
+  a.B = B;
+  a.N = N;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  for (int g = 0; g < 8; ++g) {
+    a.cut[g] = (cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : cut[g];
+    if (a.cut[g] < 0) return WP_ERR_ARG;
+  }
+  a.scale_log2 = scale_log2;
+  a.wait_limit = g_wait_limit;
+  if ((N + 127) / 128 > 65535) return WP_ERR_UNSUPPORTED;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, B, N, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map(&tk, k, B, N, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map(&tv, v, B, N, H_kv, d_h, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return WP_ERR_CUDA;
+  return from_cuda(launch_prefill_grouped(d_h, tq, tk, tv, a, s));
+}
+
+size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {
+  if (B <= 0 || H_q <= 0 || d_h <= 0 || Lmax <= 0) return 0;
+  const int nsplit = (Lmax + DECODE_CHUNK - 1) / DECODE_CHUNK;
+  return decode_workspace_bytes(B, H_q, nsplit, d_h);
+}
+
+int wp_decode(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B, int H_q,
+              int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+              void *workspace, size_t ws_bytes, void *stream) {
+  if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr ||
+      workspace == nullptr)
+    return WP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || (reinterpret_cast<uintptr_t>(lens) & 3u) != 0 ||
+      (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
+    return WP_ERR_ARG;
+  if (B <= 0 || Lmax <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  const int R = H_q / H_kv;
+  if (R != 1 && R != 2 && R != 4 && R != 8) return WP_ERR_UNSUPPORTED;
+  if (B > 65535 || H_kv > 65535) return WP_ERR_UNSUPPORTED;
+  if (!std::isfinite(softmax_scale)) return WP_ERR_ARG;
+  const int nsplit = (Lmax + DECODE_CHUNK - 1) / DECODE_CHUNK;
+  if (ws_bytes < decode_workspace_bytes(B, H_q, nsplit, d_h)) return WP_ERR_ARG;
+  const float scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(d_h)));
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q);
+  a.kc = static_cast<const __nv_bfloat16 *>(kcache);
+  a.vc = static_cast<const __nv_bfloat16 *>(vcache);
+  a.lens = lens;
+  a.o = static_cast<__nv_bfloat16 *>(o);
+  a.lse = lse;
+  a.o_part = static_cast<float *>(workspace);
+  a.lse_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) +
+                                         decode_partial_o_bytes(B, H_q, nsplit, d_h));
+  a.B = B;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  a.Lmax = Lmax;
+  a.nsplit = nsplit;
+  a.chunk = DECODE_CHUNK;
+  for (int g = 0; g < 8; ++g) {
+    a.cut[g] = (group_cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : group_cut[g];
+    if (a.cut[g] < 0) return WP_ERR_ARG;
+  }
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
+  return from_cuda(launch_decode(a, d_h, static_cast<cudaStream_t>(stream)));
+}
+
+int wp_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return WP_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_status, sizeof(int)) != cudaSuccess) return WP_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return WP_ERR_CUDA;
+  return h == 0 ? WP_OK : h;
+}
+
+long long wp_set_wait_limit(long long cycles) {
+  const long long prev = g_wait_limit;
+  g_wait_limit = cycles > 0 ? cycles : DEFAULT_WAIT_LIMIT;
+  return prev;
+}
+
+int wp_wait_probe(void *stream) {
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_wait_limit);
+  return from_cuda(cudaGetLastError());
+}
+
+const char *wp_status_str(int status) {
+  switch (status) {
+    case WP_OK: return "ok";
+    case WP_ERR_ARG: return "invalid argument";
+    case WP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case WP_ERR_CUDA: return "CUDA error";
+    case WP_ERR_TIMEOUT: return "kernel gave up waiting on an internal barrier";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

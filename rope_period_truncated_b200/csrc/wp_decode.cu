@@ -1,0 +1,317 @@
+// WavePrune split-KV decode (HBM-bound) and the LSE combine.
+//
+// What it computes: the prefill definition's row len-1 (WavePrune reading
+// notes "WavePrune：RoPE 通常只需一个旋转周期", §2.1 Eq. (6) with the grouped
+// cutoffs of §2.3 Eq. (8)): for the query at position len-1 and key j at
+// distance dist = len-1-j,
+//   s_j = scale * sum_{g : dist <= W_g} q[16g:16g+16] . k_j[16g:16g+16],
+// then softmax over j = 0..len-1 and O = sum_j p_j v_j. §2.3's table: in
+// decode a skipped group's K need not be read at all — only V is read in full.
+//
+// Split kernel: one CTA per (split, KV head, sequence); the CTA's 4 warps each
+// stream 16-key blocks of the split's key chunk through a private 3-stage
+// shared-memory ring filled with 16-byte cp.async loads (coalesced along the
+// head dim). A 16-byte K piece whose group is out of window for that key is
+// not read from HBM: the copy's source size is 0, which zero-fills shared
+// memory, so the group adds exactly 0 to the logit. The GQA query heads of the
+// KV head (H_q/H_kv <= 8) form the rows of warp-level bf16 mma.sync products
+// (scores Q.K^T and P.V, fp32 accumulation); the online softmax keeps the row
+// max and row sum with warp shuffles. The 4 warps merge their states in
+// shared memory and write one partial (O normalised, LSE base 2) per split.
+// Combine kernel: per (sequence, query head) merge the splits by LSE.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "wp_decode.h"
+#include "wp_device.cuh"
+
+namespace wp {
+
+namespace {
+
+constexpr int DEC_WARPS = 4;
+constexpr int DEC_THREADS = DEC_WARPS * 32;
+constexpr int KEYS = 16;   // keys per warp block
+constexpr int STAGES = 3;  // cp.async ring depth per warp
+
+template <int D>
+struct DecLayout {
+  static constexpr int PIECES = D / 8;                   // 16-byte pieces per row
+  static constexpr uint32_t ROWB = D * 2;                // bytes per row
+  static constexpr uint32_t TILE = KEYS * ROWB;          // one 16-key K (or V) block
+  static constexpr uint32_t STAGE = 2 * TILE;            // K then V
+  static constexpr uint32_t WARP_BYTES = STAGES * STAGE;
+  static constexpr uint32_t RING_BYTES = DEC_WARPS * WARP_BYTES;
+  // after the loop the ring is reused for the cross-warp merge
+  static constexpr uint32_t MERGE_BYTES = DEC_WARPS * 8 * (D + 2) * 4;
+  static constexpr uint32_t BYTES = RING_BYTES > MERGE_BYTES ? RING_BYTES : MERGE_BYTES;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte offset of 16-byte piece p of row r inside a block: pieces are XOR
+// swizzled by the row so 8 rows read at one column hit 8 distinct banks.
+template <int D>
+__device__ __forceinline__ uint32_t piece_off(int r, int p) {
+  return static_cast<uint32_t>(r) * DecLayout<D>::ROWB + static_cast<uint32_t>((p ^ (r & 7)) * 16);
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeArgs a) {
+  using L = DecLayout<D>;
+  constexpr int PIECES = L::PIECES;
+  constexpr int KSTEPS = D / 16;
+  constexpr int NT = D / 8;  // output n-tiles of 8 dims
+  extern __shared__ __align__(128) uint8_t dsmem[];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int len = a.lens[b];
+  if (len < 1 || len > a.Lmax) return;  // the combine writes NaN for this sequence
+  const int start = split * a.chunk;
+  const int end = min(start + a.chunk, len);
+  const int hq0 = hk * R;
+  const int64_t part = (static_cast<int64_t>(b) * a.Hq + hq0) * a.nsplit + split;  // head hq0's slot
+  if (start >= len) {
+    if (threadIdx.x < R) a.lse_part[part + static_cast<int64_t>(threadIdx.x) * a.nsplit] = -INFINITY;
+    return;
+  }
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t qpos = len - 1;
+
+  // Q as the A operand (rows = query heads; rows >= R and 8..15 are zero).
+  uint32_t qa[KSTEPS][2];
+  {
+    const __nv_bfloat16 *qrow = a.q + (static_cast<int64_t>(b) * a.Hq + hq0 + (g < R ? g : 0)) * D;
+#pragma unroll
+    for (int c = 0; c < KSTEPS; ++c) {
+      uint32_t lo = 0, hi = 0;
+      if (g < R) {
+        lo = *reinterpret_cast<const uint32_t *>(qrow + 16 * c + 2 * t);
+        hi = *reinterpret_cast<const uint32_t *>(qrow + 16 * c + 8 + 2 * t);
+      }
+      qa[c][0] = lo;
+      qa[c][1] = hi;
+    }
+  }
+
+  const __nv_bfloat16 *kbase = a.kc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;
+  const __nv_bfloat16 *vbase = a.vc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;
+  const uint32_t ring = smem_u32(dsmem) + warp * L::WARP_BYTES;
+
+  // Issue the loads of one 16-key block into stage `st`.
+  auto load_block = [&](int kb0, int st) {
+    const uint32_t kdst = ring + st * L::STAGE, vdst = kdst + L::TILE;
+#pragma unroll
+    for (int it = 0; it < KEYS * PIECES / 32; ++it) {
+      const int idx = it * 32 + lane;
+      const int r = idx / PIECES, p = idx % PIECES;
+      const int key = kb0 + r;
+      const bool valid = key < end;
+      const int64_t dist = qpos - key;
+      const bool kin = valid && dist <= static_cast<int64_t>(a.cut[p >> 1]);
+      const int64_t row = valid ? key : kb0;  // any in-range address when nothing is read
+      cp_async16(kdst + piece_off<D>(r, p), kbase + row * D + 8 * p, kin ? 16u : 0u);
+      cp_async16(vdst + piece_off<D>(r, p), vbase + row * D + 8 * p, valid ? 16u : 0u);
+    }
+  };
+
+  float m_run = -INFINITY, l_run = 0.f;  // for query head g (rows g < R)
+  float o[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+  // This warp's blocks: start + 16*(warp + 4n).
+  const int first = start + KEYS * warp;
+  const int stride = KEYS * DEC_WARPS;
+  const int nblk = first < end ? (end - first + stride - 1) / stride : 0;
+#pragma unroll
+  for (int s = 0; s < STAGES - 1; ++s) {
+    if (s < nblk) load_block(first + s * stride, s);
+    cp_async_commit();
+  }
+  for (int n = 0; n < nblk; ++n) {
+    if (n + STAGES - 1 < nblk) load_block(first + (n + STAGES - 1) * stride, (n + STAGES - 1) % STAGES);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
+    __syncwarp();
+    const int st = n % STAGES;
+    const uint32_t ks = ring + st * L::STAGE, vs = ks + L::TILE;
+    const int kb0 = first + n * stride;
+
+    // scores S[head][key] for keys 0-7 (s0) and 8-15 (s1)
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < KSTEPS; ++c) {
+      const int mi = lane >> 3, rr = (mi >> 1) * 8 + (lane & 7), pp = 2 * c + (mi & 1);
+      uint32_t b00, b01, b10, b11;
+      ldsm_x4(ks + piece_off<D>(rr, pp), b00, b01, b10, b11);
+      mma_16816(s0, qa[c][0], 0u, qa[c][1], 0u, b00, b01);
+      mma_16816(s1, qa[c][0], 0u, qa[c][1], 0u, b10, b11);
+    }
+    // lane holds head g, keys 2t, 2t+1 (s0[0..1]) and 8+2t, 9+2t (s1[0..1])
+    float sc[4] = {s0[0], s0[1], s1[0], s1[1]};
+    const int kk[4] = {2 * t, 2 * t + 1, 8 + 2 * t, 9 + 2 * t};
+    float mx = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sc[e] = (kb0 + kk[e] < end) ? sc[e] * a.scale_log2 : -INFINITY;
+      mx = fmaxf(mx, sc[e]);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = fast_exp2(m_run - m_new);
+    float p[4], ps = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      p[e] = fast_exp2(sc[e] - m_new);
+      ps += p[e];
+    }
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+    l_run = l_run * alpha + ps;
+    m_run = m_new;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      o[j][0] *= alpha;
+      o[j][1] *= alpha;
+    }
+    const uint32_t pa0 = pack_bf16x2(p[0], p[1]), pa2 = pack_bf16x2(p[2], p[3]);
+#pragma unroll
+    for (int c = 0; c < KSTEPS; ++c) {
+      const int mi = lane >> 3, rr = (mi & 1) * 8 + (lane & 7), pp = 2 * c + (mi >> 1);
+      uint32_t b0a, b1a, b0b, b1b;
+      ldsm_x4_t(vs + piece_off<D>(rr, pp), b0a, b1a, b0b, b1b);
+      mma_16816(o[2 * c], pa0, 0u, pa2, 0u, b0a, b1a);
+      mma_16816(o[2 * c + 1], pa0, 0u, pa2, 0u, b0b, b1b);
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // Merge the 4 warps: warp w's state for head g goes to shared memory.
+  float *merge = reinterpret_cast<float *>(dsmem);
+  float *mw = merge + warp * 8 * (D + 2);  // [8 heads][D + 2]: O..., m, l
+  if (g < R) {
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      mw[g * (D + 2) + 8 * j + 2 * t] = o[j][0];
+      mw[g * (D + 2) + 8 * j + 2 * t + 1] = o[j][1];
+    }
+    if (t == 0) {
+      mw[g * (D + 2) + D] = m_run;
+      mw[g * (D + 2) + D + 1] = l_run;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < R * D; e += DEC_THREADS) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < DEC_WARPS; ++w) M = fmaxf(M, merge[w * 8 * (D + 2) + h * (D + 2) + D]);
+    float Lsum = 0.f, acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < DEC_WARPS; ++w) {
+      const float *mh = merge + w * 8 * (D + 2) + h * (D + 2);
+      const float f = mh[D] == -INFINITY ? 0.f : fast_exp2(mh[D] - M);
+      Lsum += mh[D + 1] * f;
+      acc += mh[d] * f;
+    }
+    const int64_t slot = part + static_cast<int64_t>(h) * a.nsplit;
+    a.o_part[slot * D + d] = acc / Lsum;
+    if (d == 0) a.lse_part[slot] = M + __log2f(Lsum);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
+  const int bh = blockIdx.x;
+  const int b = bh / a.Hq;
+  const int d = threadIdx.x;
+  const int len = a.lens[b];
+  __nv_bfloat16 *orow = a.o + static_cast<int64_t>(bh) * D;
+  if (len < 1 || len > a.Lmax) {
+    orow[d] = __float2bfloat16_rn(__int_as_float(0x7fc00000));
+    if (d == 0 && a.lse != nullptr) a.lse[bh] = __int_as_float(0x7fc00000);
+    return;
+  }
+  const int ns = (len + a.chunk - 1) / a.chunk;  // splits that hold keys
+  const float *lp = a.lse_part + static_cast<int64_t>(bh) * a.nsplit;
+  const float *op = a.o_part + static_cast<int64_t>(bh) * a.nsplit * D;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, lp[s]);
+  float Lsum = 0.f, acc = 0.f;
+  for (int s = 0; s < ns; ++s) {
+    const float w = fast_exp2(lp[s] - M);
+    Lsum += w;
+    acc += w * op[static_cast<int64_t>(s) * D + d];
+  }
+  orow[d] = __float2bfloat16_rn(acc / Lsum);
+  if (d == 0 && a.lse != nullptr) a.lse[bh] = (M + log2f(Lsum)) * 0.69314718055994531f;
+}
+
+template <int D, int R>
+cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+  const uint32_t smem = DecLayout<D>::BYTES;
+  cudaError_t e =
+      cudaFuncSetAttribute(decode_split_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.nsplit, a.Hkv, a.B);
+  decode_split_kernel<D, R><<<grid, DEC_THREADS, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_split_r(const DecodeArgs &a, int R, cudaStream_t stream) {
+  switch (R) {
+    case 1: return launch_split<D, 1>(a, stream);
+    case 2: return launch_split<D, 2>(a, stream);
+    case 4: return launch_split<D, 4>(a, stream);
+    default: return launch_split<D, 8>(a, stream);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream) {
+  const int R = a.Hq / a.Hkv;
+  cudaError_t e = d_h == 128 ? launch_split_r<128>(a, R, stream) : launch_split_r<64>(a, R, stream);
+  if (e != cudaSuccess) return e;
+  if (d_h == 128)
+    decode_combine_kernel<128><<<a.B * a.Hq, 128, 0, stream>>>(a);
+  else
+    decode_combine_kernel<64><<<a.B * a.Hq, 64, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace wp

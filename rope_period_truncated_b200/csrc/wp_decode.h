@@ -1,0 +1,38 @@
+// Internal launch interface of the decode kernels (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace wp {
+
+// Keys per split of the split-KV decode.
+constexpr int DECODE_CHUNK = 1024;
+
+struct DecodeArgs {
+  const __nv_bfloat16 *q;            // [B, Hq, D]
+  const __nv_bfloat16 *kc, *vc;      // [B, Hkv, Lmax, D]
+  const int32_t *lens;               // [B]
+  __nv_bfloat16 *o;                  // [B, Hq, D]
+  float *lse;                        // [B, Hq] or null
+  float *o_part;                     // [B, Hq, nsplit, D]
+  float *lse_part;                   // [B, Hq, nsplit], base-2
+  int B, Hq, Hkv, Lmax, nsplit, chunk;
+  int32_t cut[8];                    // group cutoffs
+  float scale_log2;
+};
+
+// Scratch layout: o_part first, then lse_part at a 256-byte boundary.
+inline size_t decode_partial_o_bytes(int B, int Hq, int nsplit, int D) {
+  return (static_cast<size_t>(B) * Hq * nsplit * D * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+inline size_t decode_workspace_bytes(int B, int Hq, int nsplit, int D) {
+  return decode_partial_o_bytes(B, Hq, nsplit, D) +
+         ((static_cast<size_t>(B) * Hq * nsplit * sizeof(float) + 255) & ~static_cast<size_t>(255));
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream);
+
+}  // namespace wp

@@ -1,0 +1,102 @@
+// WavePrune exact per-channel causal prefill (correctness path, CUDA cores).
+//
+// WavePrune reading notes "WavePrune：RoPE 通常只需一个旋转周期", §2.1 Eq. (6):
+//   L_ij = scale * sum_c 1[i - j <= W_c] * (q_a k_a + q_b k_b),  j <= i,
+// where (a, b) are the two dims of RoPE channel c; then the causal softmax
+// and O = A V. A dropped channel adds 0, the pair stays in the softmax.
+//
+// One warp per query row: lanes take 32 keys at a time, each lane forms its
+// key's logit channel by channel; the warp keeps an online softmax (row max
+// and row sum by warp shuffles) and accumulates O with lanes over head dims.
+// Not tuned for speed: the grouped tensor-core kernel is the fast path.
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "wp_device.cuh"
+#include "wp_prefill.h"
+
+namespace wp {
+
+namespace {
+
+constexpr int ROWS_PER_CTA = 4;
+
+template <int D>
+__global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(const ChannelPrefillArgs a) {
+  constexpr int C = D / 2;
+  constexpr int PER_LANE = D / 32;
+  __shared__ float q_s[ROWS_PER_CTA][D];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * ROWS_PER_CTA + warp;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (a.Hq / a.Hkv);
+  if (i >= a.N) return;
+  const __nv_bfloat16 *qrow = a.q + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+  for (int t = lane; t < D; t += 32) q_s[warp][t] = __bfloat162float(qrow[t]);
+  __syncwarp();
+  const int64_t kstride = static_cast<int64_t>(a.Hkv) * D;
+  const __nv_bfloat16 *kbase = a.k + (static_cast<int64_t>(b) * a.N * a.Hkv + hk) * D;
+  const __nv_bfloat16 *vbase = a.v + (static_cast<int64_t>(b) * a.N * a.Hkv + hk) * D;
+
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[PER_LANE];
+#pragma unroll
+  for (int t = 0; t < PER_LANE; ++t) o[t] = 0.f;
+
+  for (int64_t j0 = 0; j0 <= i; j0 += 32) {
+    const int64_t j = j0 + lane;
+    float s = -INFINITY;
+    if (j <= i) {
+      const __nv_bfloat16 *krow = kbase + j * kstride;
+      const int64_t dist = i - j;
+      float acc = 0.f;
+      for (int c = 0; c < C; ++c) {
+        if (dist > static_cast<int64_t>(a.cut[c])) continue;
+        const int da = a.layout == WP_ROPE_INTERLEAVED ? 2 * c : c;
+        const int db = a.layout == WP_ROPE_INTERLEAVED ? 2 * c + 1 : c + C;
+        acc = fmaf(q_s[warp][da], __bfloat162float(krow[da]), acc);
+        acc = fmaf(q_s[warp][db], __bfloat162float(krow[db]), acc);
+      }
+      s = acc * a.scale_log2;
+    }
+    float mx = s;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = exp2f(m_run - m_new);
+    const float p = exp2f(s - m_new);
+    float ps = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+    l_run = l_run * alpha + ps;
+    m_run = m_new;
+#pragma unroll
+    for (int t = 0; t < PER_LANE; ++t) o[t] *= alpha;
+    const int nvalid = static_cast<int>(i - j0 + 1 < 32 ? i - j0 + 1 : 32);
+    for (int kk = 0; kk < nvalid; ++kk) {
+      const float pk = __shfl_sync(0xffffffffu, p, kk);
+      const __nv_bfloat16 *vrow = vbase + (j0 + kk) * kstride;
+#pragma unroll
+      for (int t = 0; t < PER_LANE; ++t) o[t] = fmaf(pk, __bfloat162float(vrow[lane + 32 * t]), o[t]);
+    }
+  }
+  __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+  const float inv_l = 1.f / l_run;
+#pragma unroll
+  for (int t = 0; t < PER_LANE; ++t) orow[lane + 32 * t] = __float2bfloat16_rn(o[t] * inv_l);
+  if (lane == 0 && a.lse != nullptr)
+    a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_channel(int d_h, const ChannelPrefillArgs &a, cudaStream_t stream) {
+  dim3 grid((a.N + ROWS_PER_CTA - 1) / ROWS_PER_CTA, a.Hq, a.B);
+  if (d_h == 128)
+    prefill_channel_kernel<128><<<grid, ROWS_PER_CTA * 32, 0, stream>>>(a);
+  else
+    prefill_channel_kernel<64><<<grid, ROWS_PER_CTA * 32, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace wp

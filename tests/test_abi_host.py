@@ -1,0 +1,165 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol
+the header declares, the host-only calls (cutoff tables, tile schedule) are
+bit-exact against the fp64 oracle, and argument checks reject bad calls
+before anything is launched."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import rope_period_truncated_b200 as wp
+from rope_period_truncated_b200 import build as wpbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    wpbuild.build()
+    return wp.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    header = open(os.path.join(ROOT, "include", "waveprune.h")).read()
+    declared = set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(wp_\w+)\s*\(", header, re.M))
+    assert {"wp_cutoffs", "wp_rope_apply", "wp_schedule", "wp_prefill", "wp_decode"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+CUTOFF_CASES = [
+    (64, 1e4, wp.ROPE_INTERLEAVED, 1.0, 2.0),
+    (64, 1e4, wp.ROPE_HALF_SPLIT, 1.0, 2.0),
+    (128, 1e6, wp.ROPE_HALF_SPLIT, 1.0, 2.0),
+    (128, 1e6, wp.ROPE_INTERLEAVED, 1.0, 2.0),
+    (128, 1e6, wp.ROPE_HALF_SPLIT, 0.25, 2.0),
+    (128, 5e5, wp.ROPE_HALF_SPLIT, 1.0, 1.5),
+    (64, 1e4, wp.ROPE_INTERLEAVED, 1.0, 1e300),
+]
+
+
+@pytest.mark.parametrize("d,theta,layout,scale_all,alpha", CUTOFF_CASES)
+def test_cutoffs_bit_exact(lib, d, theta, layout, scale_all, alpha):
+    a_c, a_g = wp.wp_cutoffs(d, theta, layout, alpha=alpha, scale_all=scale_all)
+    b_c, b_g = oracle.cutoffs(d, theta, layout, alpha=alpha, scale_all=scale_all)
+    assert np.array_equal(a_c, b_c) and np.array_equal(a_g, b_g)
+
+
+def test_cutoffs_per_channel_scale(lib):
+    rng = np.random.default_rng(0)
+    fs = rng.uniform(0.2, 1.0, 64)
+    a = wp.wp_cutoffs(128, 1e6, wp.ROPE_HALF_SPLIT, freq_scale=fs)
+    b = oracle.cutoffs(128, 1e6, oracle.HALF_SPLIT, freq_scale=fs)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_cutoffs_reject_bad_arguments(lib):
+    out = np.zeros(64, dtype=np.int32)
+    p = out.ctypes.data_as(ctypes.c_void_p)
+    assert lib.wp_cutoffs(100, 1e4, None, 1.0, 2.0, 0, p, p) == wp.WP_ERR_ARG    # d_h not a multiple of 16
+    assert lib.wp_cutoffs(64, 1.0, None, 1.0, 2.0, 0, p, p) == wp.WP_ERR_ARG     # theta <= 1
+    assert lib.wp_cutoffs(64, 1e4, None, 0.0, 2.0, 0, p, p) == wp.WP_ERR_ARG     # scale <= 0
+    assert lib.wp_cutoffs(64, 1e4, None, float("nan"), 2.0, 0, p, p) == wp.WP_ERR_ARG
+    assert lib.wp_cutoffs(64, 1e4, None, 1.0, 0.0, 0, p, p) == wp.WP_ERR_ARG     # alpha <= 0
+    assert lib.wp_cutoffs(64, 1e4, None, 1.0, 2.0, 7, p, p) == wp.WP_ERR_ARG     # layout
+
+
+SCHEDULE_CASES = [(256, 128, 128), (300, 128, 128), (4096, 128, 128), (1000, 64, 128), (777, 128, 64), (1, 128, 128),
+                  (129, 128, 128)]
+
+
+@pytest.mark.parametrize("N,BM,BN", SCHEDULE_CASES)
+def test_schedule_bit_exact_vs_brute_force(lib, N, BM, BN):
+    cuts = [0, 5, 28, 127, 128, 160, 255, 256, 900, 5063, 2 ** 31 - 1]
+    a_cls, a_cnt = wp.wp_schedule(N, BM, BN, cuts)
+    b_cls, b_cnt = oracle.tile_classes(N, BM, BN, cuts)
+    assert np.array_equal(a_cls, b_cls)
+    assert np.array_equal(a_cnt, b_cnt)
+
+
+@pytest.mark.parametrize("name,N", [("long_32k", 32768), ("qwen3_8b_4k", 4096)])
+def test_schedule_workload_counts(lib, name, N):
+    """Bit-exact per-group counts for the benchmark workloads' own cutoffs."""
+    _, wg = oracle.cutoffs(128, 1e6, oracle.HALF_SPLIT)
+    _, a_cnt = wp.wp_schedule(N, 128, 128, wg, want_map=False)
+    _, b_cnt = oracle.tile_classes(N, 128, 128, wg, want_map=False)
+    assert np.array_equal(a_cnt, b_cnt)
+
+
+def test_schedule_rejects_bad_arguments(lib):
+    cut = np.zeros(4, dtype=np.int32)
+    cnt = np.zeros(12, dtype=np.int64)
+    cp, np_ = cut.ctypes.data_as(ctypes.c_void_p), cnt.ctypes.data_as(ctypes.c_void_p)
+    assert lib.wp_schedule(0, 128, 128, cp, 4, None, np_) == wp.WP_ERR_ARG
+    assert lib.wp_schedule(10, 0, 128, cp, 4, None, np_) == wp.WP_ERR_ARG
+    assert lib.wp_schedule(10, 128, 128, None, 4, None, np_) == wp.WP_ERR_ARG
+    neg = np.array([-1], dtype=np.int32)
+    assert lib.wp_schedule(10, 128, 128, neg.ctypes.data_as(ctypes.c_void_p), 1, None, np_) == wp.WP_ERR_ARG
+
+
+# Device calls: every case below breaks a rule that is checked on the host
+# before any CUDA call, so nothing is launched (safe with or without a GPU).
+FAKE = 1 << 20  # a 16-byte aligned fake address, never dereferenced
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    cut = (ctypes.c_int32 * 8)(*([100] * 8))
+    f = lib.wp_prefill
+    ok = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, N=64, Hq=4, Hkv=2, d=128, mode=0, layout=1)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["N"], a["Hq"], a["Hkv"], a["d"], a["mode"],
+                 cut, a["layout"], ctypes.c_float(0.0), None)
+
+    assert call(q=None) == wp.WP_ERR_ARG
+    assert call(o=FAKE + 8) == wp.WP_ERR_ARG          # misaligned
+    assert call(Hq=3) == wp.WP_ERR_ARG                # Hq % Hkv
+    assert call(N=0) == wp.WP_ERR_ARG
+    assert call(d=96) == wp.WP_ERR_UNSUPPORTED
+    assert call(d=100) == wp.WP_ERR_ARG
+    assert call(mode=5) == wp.WP_ERR_ARG
+    assert call(layout=3) == wp.WP_ERR_ARG
+    negcut = (ctypes.c_int32 * 8)(*([-1] * 8))
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 64, 4, 2, 128, 0, negcut, 1, ctypes.c_float(0.0), None) == wp.WP_ERR_ARG
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 64, 4, 2, 128, 0, cut, 1, ctypes.c_float(float("inf")),
+             None) == wp.WP_ERR_ARG
+
+
+def test_decode_rejects_bad_arguments(lib):
+    f = lib.wp_decode
+    ws = lib.wp_decode_workspace_bytes(2, 8, 128, 4096)
+    assert ws > 0
+    args = [FAKE, FAKE, FAKE, FAKE, 4096, 2, 8, 2, 128, None, ctypes.c_float(0.0), FAKE, None, FAKE, ws, None]
+
+    def call(i, val):
+        a = list(args)
+        a[i] = val
+        return f(*a)
+
+    assert call(0, None) == wp.WP_ERR_ARG               # q NULL
+    assert call(13, FAKE + 16) == wp.WP_ERR_ARG         # workspace not 256-aligned
+    assert call(14, ws - 1) == wp.WP_ERR_ARG            # workspace too small
+    assert call(6, 6) == wp.WP_ERR_UNSUPPORTED          # 3 query heads per KV head
+    assert call(8, 72) == wp.WP_ERR_ARG                 # d_h not a multiple of 16
+    assert call(8, 80) == wp.WP_ERR_UNSUPPORTED         # d_h not 64 or 128
+    assert call(4, 0) == wp.WP_ERR_ARG                  # Lmax
+
+
+def test_rope_rejects_bad_arguments(lib):
+    f = lib.wp_rope_apply
+    assert f(None, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG
+    assert f(FAKE, FAKE + 64, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG  # partial overlap
+    assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 0.5, None, 1.0, 0, None) == wp.WP_ERR_ARG       # theta
+    assert f(FAKE, FAKE, 1, 4, 2, 48, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_UNSUPPORTED
+    assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 2, None) == wp.WP_ERR_ARG       # layout
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert wp.wp_status_str(code)
+    assert "unknown" in wp.wp_status_str(99)

@@ -1,0 +1,96 @@
+"""GPU parity of wp_decode (split-KV, grouped cutoffs) against the fp64
+oracle, plus decode-vs-prefill consistency on the GPU."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_period_truncated_b200 as wp
+import wp_synthetic as syn
+from parity import assert_attention_close, widen
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_decode(q, kc, vc, lens, cut):
+    o, lse = wp.wp_decode(q.cuda(), kc.cuda(), vc.cuda(), lens.cuda(), cut)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 4), (8, 4), (16, 2)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_small(Hq, Hkv, d):
+    g = torch.Generator().manual_seed(21 + Hq + d)
+    B, Lmax = 4, 3000
+    lens = torch.tensor([1, 2999, 1500, 1025], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    _, wg = oracle.cutoffs(d, 1e4, oracle.HALF_SPLIT)
+    wg = np.minimum(wg, [5, 40, 300, 1100, 2000, 10 ** 6, 7, 1024][: d // 16]).astype(np.int32)
+    o, lse = _gpu_decode(q, kc, vc, lens, wg)
+    ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o, lse, ro, rl, f"decode Hq={Hq} Hkv={Hkv} d={d}")
+
+
+def test_decode_dense_and_zero_cutoffs():
+    g = torch.Generator().manual_seed(3)
+    B, Hq, Hkv, d, Lmax = 2, 8, 2, 128, 2100
+    lens = torch.tensor([2100, 777], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    for cut in [None, np.zeros(8, dtype=np.int32)]:
+        o, lse = _gpu_decode(q, kc, vc, lens, cut)
+        ocut = cut if cut is not None else np.full(8, 2 ** 31 - 1)
+        ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), ocut)
+        assert_attention_close(o, lse, ro, rl, f"decode cut={'dense' if cut is None else 'zero'}")
+
+
+def test_decode_workload_full():
+    """16 sequences, H32/8, d128, lengths U[16384, 32768], theta 1e6 half-split:
+    the query is rotated on the GPU at position len-1, every row checked."""
+    w = syn.workload("decode_32k")
+    q, kc, vc, lens = syn.decode_inputs(w)
+    _, wg = oracle.cutoffs(w.d, w.theta, w.layout)
+    pos = (lens - 1).to(torch.int32).reshape(w.B, 1)
+    qr = wp.wp_rope_apply(q.cuda().reshape(w.B, 1, w.Hq, w.d), w.theta, w.layout, pos=pos.cuda())
+    o, lse = wp.wp_decode(qr.reshape(w.B, w.Hq, w.d), kc.cuda(), vc.cuda(), lens.cuda(), wg)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    qo = oracle.rope(widen(q).reshape(w.B, 1, w.Hq, w.d), w.theta, w.layout, pos=pos.numpy())
+    qo = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qo)).reshape(w.B, w.Hq, w.d)
+    ro, rl = oracle.decode(qo, widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o, lse, ro, rl, "decode_32k")
+
+
+def test_decode_matches_prefill_last_row():
+    """Decode at length L equals row L-1 of the GPU prefill over the same keys."""
+    g = torch.Generator().manual_seed(9)
+    Hq, Hkv, d, L = 8, 2, 128, 1000
+    q = torch.randn(1, L, Hq, d, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(1, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(1, L, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    _, wg = oracle.cutoffs(d, 1e6, oracle.HALF_SPLIT)
+    po, pl = wp.wp_prefill(q, k, v, wg)
+    kc = k.permute(0, 2, 1, 3).contiguous()
+    vc = v.permute(0, 2, 1, 3).contiguous()
+    do, dl = wp.wp_decode(q[:, L - 1].contiguous(), kc, vc, torch.tensor([L], dtype=torch.int32, device="cuda"), wg)
+    torch.cuda.synchronize()
+    assert (do.float() - po[:, L - 1].float()).abs().max().item() < 2e-2
+    assert (dl - pl[:, :, L - 1]).abs().max().item() < 1e-3 * max(1.0, pl[:, :, L - 1].abs().max().item())
+
+
+def test_decode_bad_length_gives_nan_rows():
+    """A length outside 1..Lmax yields NaN rows for that sequence only."""
+    B, Hq, Hkv, d, Lmax = 2, 4, 1, 64, 256
+    q = torch.ones(B, Hq, d, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    vc = torch.ones(B, Hkv, Lmax, d, dtype=torch.bfloat16, device="cuda")
+    lens = torch.tensor([0, 100], dtype=torch.int32, device="cuda")
+    o, lse = wp.wp_decode(q, kc, vc, lens, None)
+    torch.cuda.synchronize()
+    assert torch.isnan(o[0].float()).all() and torch.isnan(lse[0]).all()
+    assert torch.allclose(o[1].float(), torch.ones_like(o[1].float()))

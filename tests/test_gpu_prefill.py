@@ -1,0 +1,137 @@
+"""GPU parity of wp_prefill (grouped tcgen05 path and exact channel path)
+against the fp64 oracle, on the same seeded inputs.
+
+Small cases run the oracle on every row (several 128-row tiles plus ragged
+tails, multiple boundary cutoffs per tile, all-masked and dense tables); the
+full-size workloads are checked on sampled rows, through the same launch
+(rope of Q and K, then prefill) that the bench times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_period_truncated_b200 as wp
+import wp_synthetic as syn
+from parity import assert_attention_close, widen
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_rotated(x_bf16, theta, layout, scale_all=1.0):
+    """The oracle's own rotation of the bf16 input, rounded to bf16, widened."""
+    r = oracle.rope(widen(x_bf16), theta, layout, scale_all=scale_all)
+    return oracle.bf16_bits_to_f64(oracle.round_bf16_bits(r))
+
+
+def _gpu_path(q, k, v, theta, layout, cut, mode, scale_all=1.0, rope=True):
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    if rope:
+        qg = wp.wp_rope_apply(qg, theta, layout, scale_all=scale_all)
+        kg = wp.wp_rope_apply(kg, theta, layout, scale_all=scale_all)
+    o, lse = wp.wp_prefill(qg, kg, vg, cut, mode, layout)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_tiny_workload(mode):
+    """Tiny workload: B1 H2/2 N256 d64 theta 1e4, interleaved; both modes."""
+    w = syn.workload("tiny")
+    q, k, v = syn.prefill_inputs(w)
+    wc, wg = oracle.cutoffs(w.d, w.theta, w.layout)
+    cut = wg if mode == wp.MODE_GROUPED else wc
+    o, lse = _gpu_path(q, k, v, w.theta, w.layout, cut, mode)
+    qr, kr = _oracle_rotated(q, w.theta, w.layout), _oracle_rotated(k, w.theta, w.layout)
+    ro, rl = oracle.attention(qr, kr, widen(v), cut, mode, w.layout)
+    assert_attention_close(o, lse, ro, rl, f"tiny mode={mode}")
+
+
+def _cut_table(kind, d, theta, layout, mode):
+    G, C = d // 16, d // 2
+    n = G if mode == wp.MODE_GROUPED else C
+    if kind == "wave":
+        wc, wg = oracle.cutoffs(d, theta, layout)
+        return wg if mode == wp.MODE_GROUPED else wc
+    if kind == "dense":
+        return None
+    if kind == "zero":
+        return np.zeros(n, dtype=np.int32)
+    if kind == "mixed":  # several distinct cutoffs inside one 128x128 tile
+        base = np.array([0, 3, 130, 129, 50, 200, 255, 1000], dtype=np.int32)
+        return np.resize(base, n)
+    raise ValueError(kind)
+
+
+SMALL = [
+    # N, d, Hq, Hkv, theta, layout, kind
+    (1, 128, 2, 1, 1e6, wp.ROPE_HALF_SPLIT, "wave"),
+    (127, 64, 2, 2, 1e4, wp.ROPE_INTERLEAVED, "wave"),
+    (129, 128, 4, 2, 1e4, wp.ROPE_HALF_SPLIT, "wave"),
+    (300, 128, 4, 1, 1e6, wp.ROPE_INTERLEAVED, "wave"),   # 28 and 160 boundary in one tile
+    (513, 128, 8, 2, 1e4, wp.ROPE_HALF_SPLIT, "wave"),
+    (640, 128, 4, 4, 1e6, wp.ROPE_HALF_SPLIT, "mixed"),
+    (384, 64, 4, 2, 1e4, wp.ROPE_INTERLEAVED, "mixed"),
+    (300, 128, 2, 2, 1e6, wp.ROPE_HALF_SPLIT, "zero"),
+    (300, 128, 2, 2, 1e6, wp.ROPE_HALF_SPLIT, "dense"),
+]
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,theta,layout,kind", SMALL)
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_small_full_rows(N, d, Hq, Hkv, theta, layout, kind, mode):
+    g = torch.Generator().manual_seed(100 + N + d)
+    q = torch.randn(2, N, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(2, N, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(2, N, Hkv, d, generator=g).to(torch.bfloat16)
+    cut = _cut_table(kind, d, theta, layout, mode)
+    # prefill alone on the drawn values (treated as already rotated)
+    o, lse = _gpu_path(q, k, v, theta, layout, cut, mode, rope=False)
+    ocut = cut if cut is not None else np.full(d // 16 if mode == wp.MODE_GROUPED else d // 2, 2 ** 31 - 1)
+    ro, rl = oracle.attention(widen(q), widen(k), widen(v), ocut, mode, layout)
+    assert_attention_close(o, lse, ro, rl, f"N={N} d={d} {kind} mode={mode}")
+
+
+def _sampled_check(name, per_head):
+    w = syn.workload(name)
+    q, k, v = syn.prefill_inputs(w)
+    _, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
+    o, lse = _gpu_path(q, k, v, w.theta, w.layout, wg, wp.MODE_GROUPED, scale_all=w.scale_all)
+    rb, rh, ri = syn.sample_rows(w, per_head)
+    # oracle: its own rotation of every key and of the sampled query rows
+    kr = _oracle_rotated(k, w.theta, w.layout, w.scale_all)
+    qrows = q[rb, ri, rh].unsqueeze(0).unsqueeze(2)            # [1, R, 1, d]
+    qrot = oracle.rope(widen(qrows), w.theta, w.layout, pos=ri.numpy().reshape(1, -1), scale_all=w.scale_all)
+    qrot = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qrot))[0, :, 0]
+    ro, rl = oracle.attention_rows(qrot, (rb.numpy(), rh.numpy(), ri.numpy()), kr, widen(v), w.Hq, wg,
+                                   oracle.MODE_GROUPED, w.layout)
+    og = o[rb.cuda(), ri.cuda(), rh.cuda()]
+    lg = lse[rb.cuda(), rh.cuda(), ri.cuda()]
+    return assert_attention_close(og, lg, ro, rl, name)
+
+
+def test_qwen3_shaped_sampled_rows():
+    """B2 H32/8 N4096 d128 theta 1e6 half-split, per-dim Q/K scales."""
+    _sampled_check("qwen3_8b_4k", 64)
+
+
+def test_long_32k_sampled_rows():
+    """B1 H32/8 N32768: 256 sampled rows per head."""
+    _sampled_check("long_32k", 256)
+
+
+def test_scaled_128k_sampled_rows():
+    """B1 H32/8 N131072, every f_c divided by 4: 128 sampled rows per head."""
+    _sampled_check("scaled_128k", 128)
+
+
+def test_dense_is_cutoff_infinity():
+    """cut=None (dense comparison path) equals an all-WP_CUTOFF_INF table bit for bit."""
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(1, 700, 4, 128, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(1, 700, 2, 128, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(1, 700, 2, 128, generator=g).to(torch.bfloat16).cuda()
+    o1, l1 = wp.wp_prefill(q, k, v, None)
+    o2, l2 = wp.wp_prefill(q, k, v, np.full(8, 2 ** 31 - 1, dtype=np.int32))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
