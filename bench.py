@@ -56,6 +56,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                   help="restrict the step (profiling a single kernel)")
+    p.add_argument("--prefill-n", type=int, default=0,
+                   help="override the prefill sequence length (smaller profiling case; not a bench line)")
     return p.parse_args()
 
 
@@ -111,30 +115,29 @@ def decode_required_bytes(lens, wg, B, Hq, Hkv, d):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """nvidia-smi clock/throttle samples of this process's GPU, taken while the
+    timed region runs."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.proc = None
         self.path = None
-        self.dev = device_index
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device_index).uuid).lower()
+        except Exception:
+            pass
 
     def start(self):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            uuid = None
-            try:
-                uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
-            except Exception:
-                pass
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
-            if uuid:
-                cmd += ["-i", uuid]
-            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
@@ -146,6 +149,7 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
+        self.out.close()
         rows = []
         with open(self.path) as f:
             for line in f:
@@ -153,8 +157,20 @@ class ClockSampler:
                 if len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.path)
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mine = [r for r in rows if self.uuid and self.uuid in r[0].lower()]
+        if mine:
+            rows = mine
+        elif len({r[0] for r in rows}) > 1:
+            first = rows[0][0]
+            rows = [r for r in rows if r[0] == first]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[1]) for r in rows) if v is not None]
+        mx = [v for v in (num(r[2]) for r in rows) if v is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
@@ -166,10 +182,13 @@ class ClockSampler:
 class Path:
     """Device buffers and launches of one hot-path step."""
 
-    def __init__(self, device):
+    def __init__(self, device, prefill_n=0):
+        import dataclasses
         import rope_period_truncated_b200 as wp
         self.wp = wp
         self.pw = syn.workload("long_32k")
+        if prefill_n:
+            self.pw = dataclasses.replace(self.pw, N=prefill_n)
         self.dw = syn.workload("decode_32k")
         pw, dw = self.pw, self.dw
         q, k, v = syn.prefill_inputs(pw)
@@ -274,14 +293,18 @@ def run_ours(args, rank, world, local):
     wpbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    path = Path(dev)
+    path = Path(dev, args.prefill_n)
     peaks, peak_kind = load_peaks()
+    do_prefill = args.only in ("all", "prefill")
+    do_decode = args.only in ("all", "decode")
     pw, dw = path.pw, path.dw
     tile_flops, pair_flops, dense_tile_flops = prefill_flops(pw.N, pw.d, pw.Hq, pw.B, path.wg)
     dec_bytes, dense_dec_bytes = decode_required_bytes(path.lens_host.numpy(), path.dwg, dw.B, dw.Hq, dw.Hkv, dw.d)
 
     def step(evp=None, evd=None):
-        if evp is None:
+        if not do_prefill:
+            pass
+        elif evp is None:
             path.prefill()
         else:
             wp.wp_rope_apply(path.q, pw.theta, pw.layout, scale_all=pw.scale_all, out=path.qr)
@@ -289,7 +312,9 @@ def run_ours(args, rank, world, local):
             evp[0].record()
             path.prefill_only()
             evp[1].record()
-        if evd is None:
+        if not do_decode:
+            pass
+        elif evd is None:
             path.decode()
         else:
             wp.wp_rope_apply(path.dq, dw.theta, dw.layout, pos=path.pos, out=path.dqr)
@@ -323,8 +348,8 @@ def run_ours(args, rank, world, local):
         torch.distributed.barrier()
     clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
-    prefill_ms = statistics.mean(a.elapsed_time(b) for a, b in evp)
-    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evd)
+    prefill_ms = statistics.mean(a.elapsed_time(b) for a, b in evp) if do_prefill else float("nan")
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evd) if do_decode else float("nan")
     if wp.wp_device_status() != 0:
         raise RuntimeError("device status word set during the timed steps")
     if world > 1:
@@ -336,7 +361,7 @@ def run_ours(args, rank, world, local):
 
     # dense comparison: the same kernels with every cutoff infinite
     dense = None
-    if not args.no_dense:
+    if not args.no_dense and args.only == "all":
         dpf = time_kernel(lambda: path.prefill_only("dense"), 5, 2)
         ddc = time_kernel(lambda: path.decode_only("dense"), 20, 5)
         wpf = time_kernel(lambda: path.prefill_only("wave"), 5, 2)
@@ -348,7 +373,7 @@ def run_ours(args, rank, world, local):
 
     # end to end through the public API with pinned host buffers
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.only == "all":
         qh, kh, vh = (t.pin_memory() for t in path.host_prefill)
         dqh = path.host_decode[0].reshape(dw.B, 1, dw.Hq, dw.d).pin_memory()
         lensh = path.lens_host.pin_memory()
@@ -445,12 +470,14 @@ def run_ours(args, rank, world, local):
         },
         "dense_comparison": dense,
         "e2e": e2e,
-        "gpu_launches": path.launches_per_step * K,
+        "gpu_launches": {"all": 6, "prefill": 3, "decode": 3}[args.only] * K,
         "clocks": clk,
         "paper_context": {"source": "A100 FlashWavePrune vs FlashAttention-2, d128, theta 1e6 (context only)",
                           "prefill_speedup_32k": 1.15, "decode_speedup_32k": 1.24},
     }
-    if rank == 0 and not args.no_cpu_baseline and world == 1:
+    if args.only != "all" or args.prefill_n:
+        out["note"] = "restricted profiling case, not a bench line"
+    if rank == 0 and not args.no_cpu_baseline and world == 1 and args.only == "all":
         out["cpu_baseline"] = cpu_baseline(path, args.cpu_seconds)
     return out
 

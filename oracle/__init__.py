@@ -48,8 +48,12 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB_PATH)
+        # WP_ORACLE_LIB points the pins at a deliberately broken copy of the
+        # oracle (tests/test_oracle_mutations.py), never at anything else.
+        path = os.environ.get("WP_ORACLE_LIB")
+        if not path:
+            path = build()
+        lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         lib.wpo_freq.restype = f64

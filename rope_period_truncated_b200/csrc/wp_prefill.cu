@@ -68,6 +68,16 @@ struct Barriers {
       *drain;
 };
 
+// Row-max growth (base-2 units) below which O is not rescaled.
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+// All lanes poll the barrier, then the warp agrees: the result is uniform and
+// the warp is converged for the .sync.aligned TMEM instructions that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long lim, volatile int *abort_flag) {
+  const bool ok = mbar_wait(bar, parity, lim, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Per key tile: groups computed without mask, groups masked per element.
 struct TileGroups {
   uint32_t full, bnd;
@@ -309,17 +319,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------- softmax warps
+    // Every tcgen05.ld/st/wait below is .sync.aligned: the whole warp must
+    // issue it together. So every wait is made warp-uniform (warp_wait), the
+    // O-rescale decision is a warp vote, and only the global stores of the
+    // padding rows of a ragged last tile are predicated.
     const int r = threadIdx.x;  // row of the query tile == TMEM lane
     const int64_t i = static_cast<int64_t>(qb) * BM + r;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    const float c2 = a.scale_log2;  // logits to base-2 exponent units
+    float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units) and sum
     int bnd_used = 0;
     bool ok = true;
     for (int t = 0; t < nkb; ++t) {
       const int kb = qb - t;
       const int sb = t & 1;
       const TileGroups tg = tile_groups(a, G, qb, kb);
-      if (!mbar_wait(&B.s_ready[sb], (t >> 1) & 1, lim, abort_flag)) {
+      if (!warp_wait(&B.s_ready[sb], (t >> 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
@@ -345,7 +360,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int32_t W;
       uint32_t cls;
       while (next_boundary_class(a, tg.bnd, prev, &W, &cls)) {
-        if (!mbar_wait(B.bnd_ready, bnd_used & 1, lim, abort_flag)) {
+        if (!warp_wait(B.bnd_ready, bnd_used & 1, lim, abort_flag)) {
           ok = false;
           break;
         }
@@ -376,16 +391,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        s[c] *= a.scale_log2;
-        mx = fmaxf(mx, s[c]);
-      }
-      const float m_new = fmaxf(m_run, mx);
-      if (t > 0 && m_new > m_run) {
+      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * c2;  // scale > 0, so the max commutes with it
+      if (t == 0) {
+        m_run = m_tile;  // the diagonal tile always holds key j = i
+      } else if (__any_sync(0xffffffffu, m_tile > m_run + RESCALE_THRESHOLD)) {
+        // Rescale only when some row's max grew by more than 2^8: otherwise
+        // the stale max stays exact (p <= 2^8 fits bf16 P and fp32 sums).
+        const float m_new = fmaxf(m_run, m_tile);
         const float alpha = fast_exp2(m_run - m_new);
-        l_run *= alpha;
         // O holds the sum through key tile t-1: wait for that PV, rescale.
-        if (!mbar_wait(B.o_ready, (t - 1) & 1, lim, abort_flag)) {
+        if (!warp_wait(B.o_ready, (t - 1) & 1, lim, abort_flag)) {
           ok = false;
           break;
         }
@@ -400,50 +416,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_st32(lane_addr + COL_O + 32 * c4, u);
         }
         tmem_wait_st();
+        l_run *= alpha;
+        m_run = m_new;
       }
-      m_run = m_new;
       float rowsum = 0.f;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
-          const float p0 = fast_exp2(s[64 * c2 + 2 * k] - m_run);
-          const float p1 = fast_exp2(s[64 * c2 + 2 * k + 1] - m_run);
+          const float p0 = fast_exp2(fmaf(s[64 * h2 + 2 * k], c2, -m_run));
+          const float p1 = fast_exp2(fmaf(s[64 * h2 + 2 * k + 1], c2, -m_run));
           rowsum += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(s_addr + 32 * c2, pk);
+        tmem_st32(s_addr + 32 * h2, pk);
       }
       l_run += rowsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&B.p_ready[sb]);
     }
-    if (ok && nkb > 0 && mbar_wait(B.o_ready, (nkb - 1) & 1, lim, abort_flag)) {
+    if (ok && nkb > 0 && warp_wait(B.o_ready, (nkb - 1) & 1, lim, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      if (i < a.N) {
-        __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
 #pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
-          uint32_t u[32];
-          tmem_ld32(lane_addr + COL_O + 32 * c4, u);
-          tmem_wait_ld(u);
-          uint4 pk[4];
-          uint32_t *pw = reinterpret_cast<uint32_t *>(pk);
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t u[32];
+        tmem_ld32(lane_addr + COL_O + 32 * c4, u);
+        tmem_wait_ld(u);
+        uint4 pk[4];
+        uint32_t *pw = reinterpret_cast<uint32_t *>(pk);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pw[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * inv_l, __uint_as_float(u[2 * k + 1]) * inv_l);
+        for (int k = 0; k < 16; ++k)
+          pw[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * inv_l, __uint_as_float(u[2 * k + 1]) * inv_l);
+        if (i < a.N) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c4);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = pk[k];
         }
-        if (a.lse != nullptr)
-          a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
       }
+      if (i < a.N && a.lse != nullptr)
+        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     } else {
-      // Tell the other roles to stop waiting for this row's progress.
+      // Tell the other roles to stop waiting for this warp's progress.
       *abort_flag = 1;
     }
   }
@@ -451,6 +468,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
+    __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }

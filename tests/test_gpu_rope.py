@@ -12,11 +12,35 @@ from parity import bf16_bits, ulp_distance, widen
 pytestmark = pytest.mark.gpu
 
 
+def _pair_magnitude(x, layout):
+    """|x_a| + |x_b| of the channel pair every element belongs to."""
+    C = x.shape[-1] // 2
+    m = np.empty_like(x)
+    if layout == wp.ROPE_INTERLEAVED:
+        pm = np.abs(x[..., 0::2]) + np.abs(x[..., 1::2])
+        m[..., 0::2], m[..., 1::2] = pm, pm
+    else:
+        pm = np.abs(x[..., :C]) + np.abs(x[..., C:])
+        m[..., :C], m[..., C:] = pm, pm
+    return m
+
+
 def _check(y_gpu, x_cpu, theta, layout, pos=None, pos0=0, scale_all=1.0, freq_scale=None):
-    ref = oracle.rope(widen(x_cpu), theta, layout, pos=pos, pos0=pos0, scale_all=scale_all, freq_scale=freq_scale)
+    """The kernel rotates in fp32, so its result is the bf16 rounding of a
+    value within a few fp32 ulps of the pair's magnitude of the exact
+    rotation. Away from cancellation that is at most 1 bf16 ulp; where
+    x_a cos - x_b sin nearly cancels, the absolute fp32 bound applies."""
+    x = widen(x_cpu)
+    ref = oracle.rope(x, theta, layout, pos=pos, pos0=pos0, scale_all=scale_all, freq_scale=freq_scale)
     ref_bits = oracle.round_bf16_bits(ref)
     ulps = ulp_distance(bf16_bits(y_gpu), ref_bits)
-    assert ulps.max() <= 1, f"max ulp distance {ulps.max()}"
+    mag = _pair_magnitude(x, layout)
+    y = widen(y_gpu)
+    ulp_ref = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    err = np.abs(y - ref)
+    assert np.all(err <= ulp_ref + 2.0 ** -20 * mag), f"max excess {np.max(err - ulp_ref - 2.0 ** -20 * mag):.3e}"
+    clean = np.abs(ref) >= 2.0 ** -8 * mag  # no heavy cancellation
+    assert ulps[clean].max() <= 1, f"max ulp distance {ulps[clean].max()} away from cancellation"
     assert (ulps > 0).mean() < 0.02, f"{(ulps > 0).mean():.3%} elements differ"
 
 
