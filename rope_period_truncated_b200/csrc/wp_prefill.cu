@@ -7,23 +7,32 @@
 // logit (detail 1 of §2.1), the pair stays in the softmax.
 //
 // How (one CTA per 128-row query tile of one query head, key tiles of 128
-// visited from the diagonal backwards):
-//   warp 4  TMA producer: Q once (one 16-dim box per group); per key tile only
+// visited from the diagonal backwards; §2.3's skip / full / boundary class of
+// every (tile, group) comes from a per-CTA table built once in shared memory):
+//   warp 8  TMA producer: Q once (one 16-dim box per group); per key tile only
 //           the K column slices of non-skipped groups (16-dim boxes, 32-byte
 //           swizzle) and all of V (64-dim boxes, 128-byte swizzle).
-//   warp 5  MMA issuer: per key tile one tcgen05.mma (M=128, N=128, K=16) per
+//   warp 9  MMA issuer: per key tile one tcgen05.mma (M=128, N=128, K=16) per
 //           non-skipped group; full groups accumulate into S_full (TMEM),
 //           boundary groups into the separate S_bnd accumulator, one distinct
 //           cutoff at a time in ascending order. Then P (bf16, written back
 //           into TMEM by the softmax warps) times V into the O accumulator.
-//   warps 0-3  one thread per query row: read S_full, add each boundary
-//           accumulator under its per-element mask, causal mask on the
-//           diagonal tile, online softmax (base-2, scale folded in), write P
-//           to TMEM, rescale O when the row max grows; epilogue O/l -> bf16,
-//           LSE = ln(sum exp).
+//   warps 0-7  two threads per query row (one per 64-key half of the tile):
+//           read S_full, add each boundary accumulator under its per-element
+//           mask, causal mask on the diagonal tile, agree on the row max with
+//           the partner warp, online softmax in base 2 with the scale folded
+//           into one FMA, write P to TMEM, rescale O only when a row max grows
+//           by more than 2^8; epilogue O/l -> bf16, LSE = ln(sum exp).
 // TMEM columns: [0, D) O, [128, 256) S_full buffer 0, [256, 384) buffer 1,
 // [384, 512) S_bnd. S_full is double-buffered so the QK MMAs of the next key
 // tile overlap the softmax of the current one.
+//
+// The softmax is the non-tensor bottleneck (16384 exponentials per tile
+// against the MUFU unit's 16 per SM per clock), so 3 of every 8 pairs take
+// 2^x on the FMA pipe instead: Cody-Waite reduction x = j + f, |f| <= 1/2,
+// and a degree-3 minimax polynomial for 2^f (coefficients from a Remez fit,
+// max relative error 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in
+// the exponent field.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -40,13 +49,20 @@ constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int KST = 3;  // K stages
 constexpr int VST = 2;  // V stages
-constexpr int NTHREADS = 192;
+constexpr int NTHREADS = 320;        // warps 0-7 softmax, 8 TMA producer, 9 MMA issuer
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int SOFTMAX_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_O = 0;
 constexpr uint32_t COL_S0 = 128;
 constexpr uint32_t COL_SB = 384;
 constexpr uint32_t GROUP_TILE_BYTES = 128 * 32;     // 128 rows x 16 bf16
 constexpr uint32_t V_CHUNK_BYTES = 128 * 128;       // 128 keys x 64 bf16
+constexpr uint32_t FULL = 0xffffffffu;
+
+// Row-max growth (base-2 units) below which O is not rescaled.
+constexpr float RESCALE_THRESHOLD = 8.0f;
 
 template <int D>
 struct Layout {
@@ -57,42 +73,31 @@ struct Layout {
   static constexpr uint32_t V_OFF = K_OFF + KST * K_STAGE;
   static constexpr uint32_t V_STAGE = (D / 64) * V_CHUNK_BYTES;
   static constexpr uint32_t BAR_OFF = V_OFF + VST * V_STAGE;
-  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 1;
+  // + 4 warp pairs x (2 per-tile exchange barriers + 1 final exchange barrier)
+  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 1 + 12;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t BYTES = MISC_OFF + 16;
-  static constexpr uint32_t ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+  static constexpr uint32_t XCH_OFF = MISC_OFF + 16;  // row-max exchange [2 parity][2 half][128 rows] + row sums
+  static constexpr uint32_t TT_OFF = XCH_OFF + (4 * 128 + 2 * 128) * 4;  // tile table: one uint16 per key tile
+  static uint32_t bytes(int nqb) { return TT_OFF + ((2u * nqb + 15u) & ~15u) + 1024u; }  // + alignment slack
 };
 
 struct Barriers {
   uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_ready, *bnd_ready, *bnd_free, *p_ready, *o_ready,
-      *drain;
+      *drain, *pair, *pair_fin;
 };
 
-// Row-max growth (base-2 units) below which O is not rescaled.
-constexpr float RESCALE_THRESHOLD = 8.0f;
-
-// All lanes poll the barrier, then the warp agrees: the result is uniform and
-// the warp is converged for the .sync.aligned TMEM instructions that follow.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long lim, volatile int *abort_flag) {
-  const bool ok = mbar_wait(bar, parity, lim, abort_flag);
-  return __all_sync(0xffffffffu, ok);
-}
-
-// Per key tile: groups computed without mask, groups masked per element.
-struct TileGroups {
-  uint32_t full, bnd;
-};
-
-__device__ __forceinline__ TileGroups tile_groups(const PrefillArgs &a, int G, int64_t qb, int64_t kb) {
+// Class masks of tile (qb, kb): bits 0-7 full groups, bits 8-15 boundary groups.
+__device__ __forceinline__ uint32_t tile_masks(const PrefillArgs &a, int G, int64_t qb, int64_t kb) {
   int64_t dmin = 0, dmax = -1;
-  TileGroups tg{0u, 0u};
-  if (!tile_distance_range(a.N, BM, BN, qb, kb, &dmin, &dmax)) return tg;
-  for (int g = 0; g < G; ++g) {
-    const int c = classify_cutoff(dmin, dmax, a.cut[g]);
-    if (c == TILE_FULL) tg.full |= 1u << g;
-    if (c == TILE_BOUNDARY) tg.bnd |= 1u << g;
+  uint32_t full = 0, bnd = 0;
+  if (tile_distance_range(a.N, BM, BN, qb, kb, &dmin, &dmax)) {
+    for (int g = 0; g < G; ++g) {
+      const int c = classify_cutoff(dmin, dmax, a.cut[g]);
+      if (c == TILE_FULL) full |= 1u << g;
+      if (c == TILE_BOUNDARY) bnd |= 1u << g;
+    }
   }
-  return tg;
+  return full | (bnd << 8);
 }
 
 // Smallest cutoff among the boundary groups in `bnd` that is > prev
@@ -102,8 +107,7 @@ __device__ __forceinline__ bool next_boundary_class(const PrefillArgs &a, uint32
                                                     int32_t *W, uint32_t *mask) {
   int64_t best = INT64_MAX;
   for (uint32_t m = bnd; m; m &= m - 1) {
-    const int g = __ffs(m) - 1;
-    const int64_t w = a.cut[g];
+    const int64_t w = a.cut[__ffs(m) - 1];
     if (w > prev && w < best) best = w;
   }
   if (best == INT64_MAX) return false;
@@ -115,6 +119,70 @@ __device__ __forceinline__ bool next_boundary_class(const PrefillArgs &a, uint32
   *W = static_cast<int32_t>(best);
   *mask = mk;
   return true;
+}
+
+// All lanes poll the barrier, then the warp agrees: the result is uniform and
+// the warp is converged for the .sync.aligned TMEM instructions that follow.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long long lim, volatile int *abort_flag) {
+  const bool ok = mbar_wait(bar, parity, lim, abort_flag);
+  return __all_sync(FULL, ok);
+}
+
+// 64 TMEM columns of this warp's lanes into r, one wait for both loads.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]),
+                 "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]),
+                 "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]),
+                 "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]),
+                 "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63])
+               :
+               : "memory");
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x on the FMA pipe (see the file comment). x below -120 returns ~2^-120,
+// which is 0 for every sum this kernel forms.
+__device__ __forceinline__ float poly_exp2(float x) {
+  constexpr float C0 = 0.99992806f, C1 = 0.69326097f, C2 = 0.24261113f, C3 = 0.05517167f;
+  constexpr float ROUND = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  x = fmaxf(x, -120.f);
+  const float t = x + ROUND;
+  const float j = t - ROUND;
+  const float f = x - j;
+  const float p = fmaf(fmaf(fmaf(C3, f, C2), f, C1), f, C0);
+  const int ji = __float_as_int(t) - __float_as_int(ROUND);
+  return __int_as_float(__float_as_int(p) + (ji << 23));
 }
 
 template <int D>
@@ -141,8 +209,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   B.bnd_free = B.bnd_ready + 1;
   B.o_ready = B.bnd_free + 1;
   B.drain = B.o_ready + 1;
+  B.pair = B.drain + 1;         // [4 pairs][2 parities]
+  B.pair_fin = B.pair + 8;      // [4 pairs]
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
+  uint16_t *ttab = reinterpret_cast<uint16_t *>(smem + L::TT_OFF);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -167,15 +238,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_ready[s], 1);
-      mbar_init(&B.p_ready[s], 128);
+      mbar_init(&B.p_ready[s], SOFTMAX_THREADS);
     }
     mbar_init(B.bnd_ready, 1);
-    mbar_init(B.bnd_free, 128);
+    mbar_init(B.bnd_free, SOFTMAX_THREADS);
     mbar_init(B.o_ready, 1);
     mbar_init(B.drain, 1);
+    for (int k = 0; k < 8; ++k) mbar_init(&B.pair[k], 64);
+    for (int k = 0; k < 4; ++k) mbar_init(&B.pair_fin[k], 64);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  // Tile table: key tile t = key block qb - t.
+  for (int t = threadIdx.x; t <= qb; t += NTHREADS) ttab[t] = static_cast<uint16_t>(tile_masks(a, G, qb, qb - t));
+  if (warp == MMA_WARP) {
     tmem_alloc(tmem_base_slot, TMEM_COLS);
     tmem_relinquish();
   }
@@ -185,280 +260,343 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_base_slot;
   const int nkb = *abort_flag ? 0 : qb + 1;  // key tiles qb, qb-1, ..., 0 (BM == BN)
 
-  if (warp == 4) {
+  if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits); one elected lane
+    // issues each bulk copy.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(B.q_full, G * GROUP_TILE_BYTES);
       for (int g = 0; g < G; ++g)
         tma_load_4d(smem + L::Q_OFF + g * GROUP_TILE_BYTES, &tm_q, B.q_full, 16 * g, h, qb * BM, b);
-      int k_issued = 0, v_issued = 0;
-      bool ok = true;
-      auto load_v = [&](int t) -> bool {
-        const int st = t % VST;
-        if (t >= VST && !mbar_wait(&B.v_empty[st], ((t / VST) - 1) & 1, lim, abort_flag)) return false;
-        const int kb = qb - t;
+    }
+    __syncwarp();
+    int k_issued = 0, v_issued = 0;
+    bool ok = true;
+    auto load_v = [&](int t) -> bool {
+      const int st = t % VST;
+      if (t >= VST && !warp_wait(&B.v_empty[st], ((t / VST) - 1) & 1, lim, abort_flag)) return false;
+      const int kb = qb - t;
+      if (leader) {
         mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * V_CHUNK_BYTES);
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(smem + L::V_OFF + st * L::V_STAGE + c * V_CHUNK_BYTES, &tm_v, &B.v_full[st], 64 * c, hk,
                       kb * BN, b);
-        ++v_issued;
-        return true;
-      };
-      for (int t = 0; ok && t < nkb; ++t) {
-        const int st = t % KST;
-        if (t >= KST && !mbar_wait(&B.k_empty[st], ((t / KST) - 1) & 1, lim, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const int kb = qb - t;
-        const TileGroups tg = tile_groups(a, G, qb, kb);
-        const uint32_t need = tg.full | tg.bnd;
+      }
+      __syncwarp();
+      ++v_issued;
+      return true;
+    };
+    for (int t = 0; ok && t < nkb; ++t) {
+      const int st = t % KST;
+      if (t >= KST && !warp_wait(&B.k_empty[st], ((t / KST) - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const int kb = qb - t;
+      const uint32_t tm = ttab[t];
+      const uint32_t need = (tm | (tm >> 8)) & 0xffu;
+      if (leader) {
         mbar_arrive_expect_tx(&B.k_full[st], __popc(need) * GROUP_TILE_BYTES);
         for (uint32_t m = need; m; m &= m - 1) {
           const int g = __ffs(m) - 1;
           tma_load_4d(smem + L::K_OFF + st * L::K_STAGE + g * GROUP_TILE_BYTES, &tm_k, &B.k_full[st], 16 * g,
                       hk, kb * BN, b);
         }
-        ++k_issued;
-        if (t >= 1) ok = load_v(t - 1);
       }
-      if (ok && nkb >= 1) ok = load_v(nkb - 1);
-      // Never leave a bulk copy in flight into shared memory this CTA is
-      // about to release: wait for Q and the last issued load of every stage.
-      mbar_wait(B.q_full, 0, lim, nullptr);
-      for (int s = 0; s < KST && s < k_issued; ++s) {
-        const int last = s + ((k_issued - 1 - s) / KST) * KST;
-        mbar_wait(&B.k_full[s], (last / KST) & 1, lim, nullptr);
-      }
-      for (int s = 0; s < VST && s < v_issued; ++s) {
-        const int last = s + ((v_issued - 1 - s) / VST) * VST;
-        mbar_wait(&B.v_full[s], (last / VST) & 1, lim, nullptr);
-      }
+      __syncwarp();
+      ++k_issued;
+      if (t >= 1) ok = load_v(t - 1);
     }
-    __syncwarp();
-  } else if (warp == 5) {
+    if (ok && nkb >= 1) ok = load_v(nkb - 1);
+    // Never leave a bulk copy in flight into shared memory this CTA is about
+    // to release: wait for Q and the last issued load of every stage.
+    warp_wait(B.q_full, 0, lim, nullptr);
+    for (int s = 0; s < KST && s < k_issued; ++s) {
+      const int last = s + ((k_issued - 1 - s) / KST) * KST;
+      warp_wait(&B.k_full[s], (last / KST) & 1, lim, nullptr);
+    }
+    for (int s = 0; s < VST && s < v_issued; ++s) {
+      const int last = s + ((v_issued - 1 - s) / VST) * VST;
+      warp_wait(&B.v_full[s], (last / VST) & 1, lim, nullptr);
+    }
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t q_addr = smem_u32(smem + L::Q_OFF);
-      const uint32_t k_addr = smem_u32(smem + L::K_OFF);
-      const uint32_t v_addr = smem_u32(smem + L::V_OFF);
-      int bnd_issued = 0;
-      bool ok = mbar_wait(B.q_full, 0, lim, abort_flag);
+    // The whole warp runs the issue loop: control flow and descriptors are
+    // warp-uniform, and one elected lane issues each tcgen05.mma / commit.
+    const bool leader = elect_one();
+    // Descriptor bases; a byte offset within shared memory is added to the
+    // start-address field (bits 0-13, in 16-byte units).
+    const uint64_t q_desc = smem_desc(smem_u32(smem + L::Q_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t k_desc = smem_desc(smem_u32(smem + L::K_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    // V tile: 128 keys x D, dims contiguous (MN-major), 128-byte swizzle;
+    // 8-key row groups 1024 B apart, 64-dim chunks 16 KB apart.
+    const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), V_CHUNK_BYTES, 1024, SMEM_SWIZZLE_128B);
+    int bnd_issued = 0;
+    bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
 
-      auto issue_qk = [&](int t) -> bool {
-        const int st = t % KST;
-        if (!mbar_wait(&B.k_full[st], (t / KST) & 1, lim, abort_flag)) return false;
-        tc_fence_after();
-        const int kb = qb - t;
-        const TileGroups tg = tile_groups(a, G, qb, kb);
-        const uint32_t s_col = tmem + COL_S0 + 128u * (t & 1);
-        uint32_t acc = 0;
-        for (uint32_t m = tg.full; m; m &= m - 1) {
-          const int g = __ffs(m) - 1;
-          const uint64_t ad = smem_desc(q_addr + g * GROUP_TILE_BYTES, 16, 256, SMEM_SWIZZLE_32B);
-          const uint64_t bd = smem_desc(k_addr + st * L::K_STAGE + g * GROUP_TILE_BYTES, 16, 256, SMEM_SWIZZLE_32B);
-          umma_ss(s_col, ad, bd, IDESC_QK, acc);
-          acc = 1;
-        }
-        umma_commit(&B.s_ready[t & 1]);
+    auto issue_qk = [&](int t) -> bool {
+      const int st = t % KST;
+      if (!warp_wait(&B.k_full[st], (t / KST) & 1, lim, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t tm = ttab[t];
+      const uint32_t s_col = tmem + COL_S0 + 128u * (t & 1);
+      const uint64_t kst_desc = k_desc + ((st * L::K_STAGE) >> 4);
+      uint32_t acc = 0;
+      for (uint32_t m = tm & 0xffu; m; m &= m - 1) {
+        const uint32_t g = __ffs(m) - 1;
+        if (leader)
+          umma_ss(s_col, q_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
+                  acc);
+        acc = 1;
+      }
+      if (leader) umma_commit(&B.s_ready[t & 1]);
+      __syncwarp();
+      const uint32_t bnd = tm >> 8;
+      if (bnd) {
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(a, tg.bnd, prev, &W, &cls)) {
+        while (next_boundary_class(a, bnd, prev, &W, &cls)) {
           if (bnd_issued > 0) {
-            if (!mbar_wait(B.bnd_free, (bnd_issued - 1) & 1, lim, abort_flag)) return false;
+            if (!warp_wait(B.bnd_free, (bnd_issued - 1) & 1, lim, abort_flag)) return false;
             tc_fence_after();
           }
           uint32_t bacc = 0;
           for (uint32_t m = cls; m; m &= m - 1) {
-            const int g = __ffs(m) - 1;
-            const uint64_t ad = smem_desc(q_addr + g * GROUP_TILE_BYTES, 16, 256, SMEM_SWIZZLE_32B);
-            const uint64_t bd =
-                smem_desc(k_addr + st * L::K_STAGE + g * GROUP_TILE_BYTES, 16, 256, SMEM_SWIZZLE_32B);
-            umma_ss(tmem + COL_SB, ad, bd, IDESC_QK, bacc);
+            const uint32_t g = __ffs(m) - 1;
+            if (leader)
+              umma_ss(tmem + COL_SB, q_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4),
+                      IDESC_QK, bacc);
             bacc = 1;
           }
-          umma_commit(B.bnd_ready);
+          if (leader) umma_commit(B.bnd_ready);
+          __syncwarp();
           ++bnd_issued;
           prev = W;
         }
-        umma_commit(&B.k_empty[st]);
-        return true;
-      };
+      }
+      if (leader) umma_commit(&B.k_empty[st]);
+      __syncwarp();
+      return true;
+    };
 
-      if (ok && nkb > 0) ok = issue_qk(0);
-      if (ok && nkb > 1) ok = issue_qk(1);
-      for (int t = 0; ok && t < nkb; ++t) {
-        const int sb = t & 1;
-        const int vst = t % VST;
-        if (!mbar_wait(&B.p_ready[sb], (t >> 1) & 1, lim, abort_flag) ||
-            !mbar_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t p_col = tmem + COL_S0 + 128u * sb;
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile: 128 keys x D, dims contiguous (MN-major), 128-byte swizzle;
-          // 8-key row groups 1024 B apart, 64-dim chunks 16 KB apart.
-          const uint64_t bd = smem_desc(v_addr + vst * L::V_STAGE + kk * 2048, V_CHUNK_BYTES, 1024,
-                                        SMEM_SWIZZLE_128B);
-          umma_ts(tmem + COL_O, p_col + kk * 8, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+    if (ok && nkb > 0) ok = issue_qk(0);
+    if (ok && nkb > 1) ok = issue_qk(1);
+    for (int t = 0; ok && t < nkb; ++t) {
+      const int sb = t & 1;
+      const int vst = t % VST;
+      if (!warp_wait(&B.p_ready[sb], (t >> 1) & 1, lim, abort_flag) ||
+          !warp_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t p_col = tmem + COL_S0 + 128u * sb;
+      const uint64_t vst_desc = v_desc + ((vst * L::V_STAGE) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk)
+        // P of keys 0-63 sits in S columns 0-31, of keys 64-127 in columns 64-95
+        if (leader)
+          umma_ts(tmem + COL_O, p_col + kk * 8 + (kk >= 4 ? 32 : 0), vst_desc + kk * (2048 >> 4), IDESC_PV,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+      if (leader) {
         umma_commit(&B.v_empty[vst]);
         umma_commit(B.o_ready);
-        if (t + 2 < nkb) ok = issue_qk(t + 2);
       }
-      // Every MMA this thread issued must finish before TMEM is released.
-      umma_commit(B.drain);
-      mbar_wait(B.drain, 0, lim, nullptr);
+      __syncwarp();
+      if (t + 2 < nkb) ok = issue_qk(t + 2);
     }
+    // Every MMA this warp issued must finish before TMEM is released.
+    if (leader) umma_commit(B.drain);
     __syncwarp();
+    warp_wait(B.drain, 0, lim, nullptr);
   } else {
     // ------------------------------------------------------- softmax warps
-    // Every tcgen05.ld/st/wait below is .sync.aligned: the whole warp must
-    // issue it together. So every wait is made warp-uniform (warp_wait), the
-    // O-rescale decision is a warp vote, and only the global stores of the
-    // padding rows of a ragged last tile are predicated.
-    const int r = threadIdx.x;  // row of the query tile == TMEM lane
+    // Warp w (0-7) owns rows 32*(w%4)..+31 — its TMEM lane quarter — and key
+    // columns 64*(w/4)..+63 of every tile: two warps share each row, which
+    // doubles the warps per scheduler that hide the softmax's latencies. The
+    // pair agrees on the row max through shared memory and an mbarrier
+    // (bounded wait). Every tcgen05.ld/st/wait below is .sync.aligned, so all
+    // waits are warp-uniform, the O-rescale decision is a warp vote (the same
+    // in both warps of a pair, as they see the same row maxima), and only the
+    // global stores of the padding rows of a ragged last tile are predicated.
+    const int q4 = warp & 3;
+    const int half = warp >> 2;
+    const int r = q4 * 32 + lane;  // row of the query tile == TMEM lane
     const int64_t i = static_cast<int64_t>(qb) * BM + r;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t col0 = 64u * half;  // first key column of this warp
+    float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
     const float c2 = a.scale_log2;  // logits to base-2 exponent units
-    float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units) and sum
+    const uint64_t c2x2 = pack_f2(c2, c2);
+    float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units), this half's sum
     int bnd_used = 0;
     bool ok = true;
     for (int t = 0; t < nkb; ++t) {
       const int kb = qb - t;
       const int sb = t & 1;
-      const TileGroups tg = tile_groups(a, G, qb, kb);
-      if (!warp_wait(&B.s_ready[sb], (t >> 1) & 1, lim, abort_flag)) {
+      const uint32_t tm = ttab[t];
+      ok = warp_wait(&B.s_ready[sb], (t >> 1) & 1, lim, abort_flag);
+      const uint32_t s_addr = lane_addr + COL_S0 + 128u * sb + col0;
+      uint32_t su[64];
+      float mh = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        if (tm & 0xffu) {
+          tmem_ld64(s_addr, su);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) su[c] = 0u;
+        }
+        const uint32_t bnd = tm >> 8;
+        if (bnd) {
+          // Boundary accumulators, one distinct cutoff at a time: keep the
+          // element iff its distance i - j is within the cutoff.
+          int64_t prev = -1;
+          int32_t W;
+          uint32_t cls;
+          while (ok && next_boundary_class(a, bnd, prev, &W, &cls)) {
+            ok = warp_wait(B.bnd_ready, bnd_used & 1, lim, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t ub[64];
+            tmem_ld64(lane_addr + COL_SB + col0, ub);
+            tc_fence_before();
+            mbar_arrive(B.bnd_free);
+            ++bnd_used;
+            prev = W;
+            // keep column col0 + c iff (i - kb*BN - col0) - c <= W
+            const int64_t cmin64 = i - static_cast<int64_t>(kb) * BN - col0 - W;
+            const int cmin = cmin64 < 0 ? 0 : (cmin64 > 64 ? 64 : static_cast<int>(cmin64));
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (c >= cmin) su[c] = __float_as_uint(__uint_as_float(su[c]) + __uint_as_float(ub[c]));
+          }
+        }
+        // Causal mask: only the diagonal tile has keys after the query.
+        if (kb == qb) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (static_cast<int>(col0) + c > r) su[c] = __float_as_uint(-INFINITY);
+        }
+        // Half-row max: 4 independent chains of 3-input max.
+        float mx4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float m = __uint_as_float(su[16 * j]);
+#pragma unroll
+          for (int k = 1; k < 15; k += 2)
+            m = max3(m, __uint_as_float(su[16 * j + k]), __uint_as_float(su[16 * j + k + 1]));
+          mx4[j] = fmaxf(m, __uint_as_float(su[16 * j + 15]));
+        }
+        mh = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      }
+      // Exchange half-row maxima with the partner warp (NaN = "aborted").
+      float *xc = xch + (t & 1) * 256;
+      xc[half * 128 + r] = ok ? mh : __int_as_float(0x7fc00000);
+      mbar_arrive(&B.pair[q4 * 2 + (t & 1)]);
+      const bool pok = warp_wait(&B.pair[q4 * 2 + (t & 1)], (t >> 1) & 1, lim, abort_flag);
+      const float mp = xc[(half ^ 1) * 128 + r];
+      if (!__all_sync(FULL, ok && pok && !isnan(mp))) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const uint32_t s_addr = lane_addr + COL_S0 + 128u * sb;
-      float s[BN];
-      if (tg.full) {
-#pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t u[32];
-          tmem_ld32(s_addr + 32 * c4, u);
-          tmem_wait_ld(u);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) s[32 * c4 + k] = __uint_as_float(u[k]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = 0.f;
-      }
-      // Boundary accumulators, one distinct cutoff at a time: keep the
-      // element iff its distance i - j is within the cutoff.
-      int64_t prev = -1;
-      int32_t W;
-      uint32_t cls;
-      while (next_boundary_class(a, tg.bnd, prev, &W, &cls)) {
-        if (!warp_wait(B.bnd_ready, bnd_used & 1, lim, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int64_t base_dist = i - static_cast<int64_t>(kb) * BN;  // distance to key column 0
-#pragma unroll
-        for (int c4 = 0; c4 < BN / 32; ++c4) {
-          uint32_t u[32];
-          tmem_ld32(lane_addr + COL_SB + 32 * c4, u);
-          tmem_wait_ld(u);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int c = 32 * c4 + k;
-            if (base_dist - c <= static_cast<int64_t>(W)) s[c] += __uint_as_float(u[k]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(B.bnd_free);
-        ++bnd_used;
-        prev = W;
-      }
-      if (!ok) break;
-      // Causal mask: only the diagonal tile has keys after the query.
-      if (kb == qb) {
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c > r) s[c] = -INFINITY;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * c2;  // scale > 0, so the max commutes with it
+      const float m_tile = fmaxf(mh, mp) * c2;  // scale > 0, so the max commutes with it
       if (t == 0) {
         m_run = m_tile;  // the diagonal tile always holds key j = i
-      } else if (__any_sync(0xffffffffu, m_tile > m_run + RESCALE_THRESHOLD)) {
+      } else if (__any_sync(FULL, m_tile > m_run + RESCALE_THRESHOLD)) {
         // Rescale only when some row's max grew by more than 2^8: otherwise
         // the stale max stays exact (p <= 2^8 fits bf16 P and fp32 sums).
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = fast_exp2(m_run - m_new);
-        // O holds the sum through key tile t-1: wait for that PV, rescale.
+        // O holds the sum through key tile t-1: wait for that PV, rescale
+        // this half's D/2 columns of O.
         if (!warp_wait(B.o_ready, (t - 1) & 1, lim, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4) {
+#pragma unroll 1
+        for (int c4 = 0; c4 < D / 64; ++c4) {
           uint32_t u[32];
-          tmem_ld32(lane_addr + COL_O + 32 * c4, u);
+          const uint32_t oc = lane_addr + COL_O + half * (D / 2) + 32 * c4;
+          tmem_ld32(oc, u);
           tmem_wait_ld(u);
 #pragma unroll
           for (int k = 0; k < 32; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * alpha);
-          tmem_st32(lane_addr + COL_O + 32 * c4, u);
+          tmem_st32(oc, u);
         }
         tmem_wait_st();
         l_run *= alpha;
         m_run = m_new;
       }
-      float rowsum = 0.f;
+      // p = 2^(s*c2 - m): one packed FMA per pair; 3 of every 8 pairs take
+      // the polynomial exp2, the rest the MUFU unit. Four packed partial sums.
+      // P (bf16 pairs) goes back into this warp's own S columns.
+      const uint64_t negm = pack_f2(-m_run, -m_run);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[32];
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = fast_exp2(fmaf(s[64 * h2 + 2 * k], c2, -m_run));
-          const float p1 = fast_exp2(fmaf(s[64 * h2 + 2 * k + 1], c2, -m_run));
-          rowsum += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+      for (int k = 0; k < 32; ++k) {
+        const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[2 * k]), __uint_as_float(su[2 * k + 1])), c2x2, negm);
+        float x0, x1;
+        unpack_f2(x2, x0, x1);
+        float p0, p1;
+        if ((k & 7) >= 5) {
+          p0 = poly_exp2(x0);
+          p1 = poly_exp2(x1);
+        } else {
+          p0 = fast_exp2(x0);
+          p1 = fast_exp2(x1);
         }
-        tmem_st32(s_addr + 32 * h2, pk);
+        acc[k & 3] = fadd2(acc[k & 3], pack_f2(p0, p1));
+        pk[k] = pack_bf16x2(p0, p1);
       }
-      l_run += rowsum;
+      tmem_st32(s_addr, pk);
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      unpack_f2(acc[0], s0, s1);
+      unpack_f2(acc[1], s2, s3);
+      unpack_f2(acc[2], s4, s5);
+      unpack_f2(acc[3], s6, s7);
+      l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&B.p_ready[sb]);
     }
-    if (ok && nkb > 0 && warp_wait(B.o_ready, (nkb - 1) & 1, lim, abort_flag)) {
+    // Row sum = both halves' sums: one more exchange, then this half's D/2
+    // output columns.
+    float *ls = xch + 512;
+    ls[half * 128 + r] = ok ? l_run : __int_as_float(0x7fc00000);
+    mbar_arrive(&B.pair_fin[q4]);
+    const bool fok = warp_wait(&B.pair_fin[q4], 0, lim, abort_flag);
+    const float l_row = l_run + ls[(half ^ 1) * 128 + r];
+    if (__all_sync(FULL, ok && fok && !isnan(l_row)) && nkb > 0 &&
+        warp_wait(B.o_ready, (nkb - 1) & 1, lim, abort_flag)) {
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+      const float inv_l = 1.f / l_row;
+      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D + half * (D / 2);
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
+      for (int c4 = 0; c4 < D / 64; ++c4) {
         uint32_t u[32];
-        tmem_ld32(lane_addr + COL_O + 32 * c4, u);
+        tmem_ld32(lane_addr + COL_O + half * (D / 2) + 32 * c4, u);
         tmem_wait_ld(u);
-        uint4 pk[4];
-        uint32_t *pw = reinterpret_cast<uint32_t *>(pk);
+        uint4 pk4[4];
+        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           pw[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * inv_l, __uint_as_float(u[2 * k + 1]) * inv_l);
         if (i < a.N) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c4);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = pk[k];
+          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
         }
       }
-      if (i < a.N && a.lse != nullptr)
-        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (half == 0 && i < a.N && a.lse != nullptr)
+        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_row)) * 0.69314718055994531f;
     } else {
       // Tell the other roles to stop waiting for this warp's progress.
       *abort_flag = 1;
@@ -467,7 +605,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == MMA_WARP) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
@@ -479,11 +617,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 template <int D>
 static cudaError_t launch_grouped(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                   const PrefillArgs &a, cudaStream_t stream) {
-  const uint32_t smem = Layout<D>::ALLOC;
+  const int nqb = (a.N + BM - 1) / BM;
+  const uint32_t smem = Layout<D>::bytes(nqb);
+  if (smem > 232448u) return cudaErrorInvalidValue;  // beyond 227 KB: N too large for the tile table
   cudaError_t e = cudaFuncSetAttribute(prefill_grouped_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int nqb = (a.N + BM - 1) / BM;
   dim3 grid(a.Hq, nqb, a.B);
   prefill_grouped_kernel<D><<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
