@@ -164,6 +164,32 @@ int wp_decode(const void *q, const void *kcache, const void *vcache, const int32
               void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * wp_decode_static — wp_decode without a workspace argument, for callers that
+ * cannot allocate device memory (for example a serving engine whose device
+ * memory is planned up front and handed out by its own pool, or a decode loop
+ * that must never reach cudaMalloc/cudaFree, which can synchronise the
+ * device). It allocates nothing: the split-KV partial results go to a
+ * fixed-size scratch array of WP_DECODE_STATIC_SCRATCH_BYTES (16 MiB) that is
+ * part of this library's device image, so every GPU that loads the library
+ * holds it until the process exits. The pages have no counterpart of this
+ * call; it is an interface for those callers.
+ *   Arguments, layouts and results are those of wp_decode.
+ *   The first call on a device looks up the scratch array's device address
+ *   (once per device, with that device current); make that first call before
+ *   any stream capture.
+ *   Every call on a device shares the one array and leaves its contents
+ *   behind; nothing in it needs to start at zero. Calls whose kernels overlap
+ *   on the GPU (e.g. on two streams without ordering) race on the array.
+ *   Errors: WP_ERR_UNSUPPORTED when wp_decode_workspace_bytes(B, H_q, d_h,
+ *   Lmax) exceeds WP_DECODE_STATIC_SCRATCH_BYTES (nothing is launched);
+ *   otherwise those of wp_decode.
+ */
+#define WP_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+int wp_decode_static(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B,
+                     int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+                     void *stream);
+
+/*
  * wp_device_status — synchronises `stream`, then reads and clears the device
  * status word of the current device. Returns WP_OK, WP_ERR_TIMEOUT (a kernel
  * gave up waiting since the last call) or WP_ERR_CUDA.

@@ -24,6 +24,7 @@ __all__ = [
     "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
     "WavePruneError", "library_path", "load_library",
     "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
+    "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES",
     "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
 ]
 
@@ -32,6 +33,7 @@ ROPE_HALF_SPLIT = 1
 MODE_GROUPED = 0
 MODE_CHANNEL = 1
 CUTOFF_INF = 2 ** 31 - 1
+DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 WP_OK, WP_ERR_ARG, WP_ERR_UNSUPPORTED, WP_ERR_CUDA, WP_ERR_TIMEOUT = range(5)
 
@@ -72,6 +74,8 @@ def load_library():
     lib.wp_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.wp_decode.restype = I
     lib.wp_decode.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
+    lib.wp_decode_static.restype = I
+    lib.wp_decode_static.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P]
     lib.wp_device_status.restype = I
     lib.wp_device_status.argtypes = [P]
     lib.wp_set_wait_limit.restype = ctypes.c_longlong
@@ -238,6 +242,33 @@ def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens:
     _check("wp_decode", load_library().wp_decode(
         _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def wp_decode_static(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens: torch.Tensor,
+                     group_cut=None, softmax_scale: float = 0.0, out: torch.Tensor | None = None,
+                     lse: torch.Tensor | None = None, want_lse: bool = True, stream=None):
+    """wp_decode without a workspace: the library's fixed device scratch holds
+    the split partials, so nothing is allocated for them (for callers that
+    cannot allocate device memory). Same arguments and results as wp_decode;
+    raises WavePruneError (unsupported) when the batch needs more than
+    DECODE_STATIC_SCRATCH_BYTES of scratch."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(vcache, "vcache", torch.bfloat16, 4)
+    _need(lens, "lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    _, Hkv, Lmax, _ = kcache.shape
+    if tuple(kcache.shape) != (B, Hkv, Lmax, d) or tuple(vcache.shape) != tuple(kcache.shape):
+        raise ValueError("cache shape mismatch")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    _check("wp_decode_static", load_library().wp_decode_static(
+        _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
+        _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 
