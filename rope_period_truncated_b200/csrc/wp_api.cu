@@ -220,7 +220,7 @@ int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
   }
   a.scale_log2 = scale_log2;
   a.wait_limit = g_wait_limit;
-  if ((N + 127) / 128 > 65535) return WP_ERR_UNSUPPORTED;
+  if ((N + 127) / 128 > 65535 || static_cast<int64_t>(H_kv) * B > 65535) return WP_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, B, N, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
       !make_map(&tk, k, B, N, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||

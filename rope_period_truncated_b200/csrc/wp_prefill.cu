@@ -217,11 +217,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  const int h = blockIdx.x;
+  // Grid (query head within its KV group, query block, KV head x batch): the
+  // CTAs that run together share one KV head, so its K/V stay in L2; within
+  // a KV head the heaviest query blocks go first.
+  const int hk = static_cast<int>(blockIdx.z) % a.Hkv;
+  const int b = static_cast<int>(blockIdx.z) / a.Hkv;
+  const int h = hk * (a.Hq / a.Hkv) + static_cast<int>(blockIdx.x);
   const int nqb = (a.N + BM - 1) / BM;
-  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);  // heaviest query tiles first
-  const int b = blockIdx.z;
-  const int hk = h / (a.Hq / a.Hkv);
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);
   const long long lim = a.wait_limit;
 
   if (threadIdx.x == 0) {
@@ -623,7 +626,7 @@ static cudaError_t launch_grouped(const CUtensorMap &tq, const CUtensorMap &tk, 
   cudaError_t e = cudaFuncSetAttribute(prefill_grouped_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hq, nqb, a.B);
+  dim3 grid(a.Hq / a.Hkv, nqb, a.Hkv * a.B);
   prefill_grouped_kernel<D><<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
