@@ -72,6 +72,17 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over all ranks (identity when
+    torch.distributed is not initialised or there is one rank)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -352,10 +363,7 @@ def run_ours(args, rank, world, local):
     decode_ms = statistics.mean(a.elapsed_time(b) for a, b in evd) if do_decode else float("nan")
     if wp.wp_device_status() != 0:
         raise RuntimeError("device status word set during the timed steps")
-    if world > 1:
-        t = torch.tensor([total_ms, prefill_ms, decode_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms, prefill_ms, decode_ms = t.tolist()
+    total_ms, prefill_ms, decode_ms = max_over_ranks([total_ms, prefill_ms, decode_ms], dev)
     ms_per_step = total_ms / K
     value = world * tile_flops / (ms_per_step * 1e-3) / 1e12
 
@@ -408,10 +416,7 @@ def run_ours(args, rank, world, local):
         b.record()
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b) / ke
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = t.item()
+        e_ms = max_over_ranks([e_ms], dev)[0]
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, dqh, lensh, posh))
         d2h = sum(t.numel() * t.element_size() for t in (oh, lseh, doh, dlh))
         e2e = {"value": round(world * tile_flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",

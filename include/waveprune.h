@@ -121,8 +121,9 @@ int wp_schedule(int N, int BM, int BN, const int32_t *cut, int n_cut, uint8_t *c
  *               row's logits (softmax scale included), or NULL.
  *   mode        WP_MODE_GROUPED: cut = host group_cut [d_h/16] — the fast path
  *               (TMA loads of only the K columns of non-skipped groups, one
- *               tcgen05 MMA per 16-dim group into TMEM, boundary groups in a
- *               separate TMEM accumulator masked per element).
+ *               tcgen05 MMA per 16-dim group into TMEM; on a tile where a
+ *               group is partly in window its contribution is masked per
+ *               element in the logit tile before the remaining groups add in).
  *               WP_MODE_CHANNEL: cut = host chan_cut [d_h/2] — exact rule,
  *               correctness path (CUDA cores), not tuned for speed.
  *               cut = NULL means every cutoff is WP_CUTOFF_INF (dense).

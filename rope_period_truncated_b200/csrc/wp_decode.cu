@@ -12,8 +12,10 @@
 // stream 16-key blocks of the split's key chunk through a private 3-stage
 // shared-memory ring filled with 16-byte cp.async loads (coalesced along the
 // head dim). A 16-byte K piece whose group is out of window for that key is
-// not read from HBM at all: no copy is issued and its shared-memory slot is
-// zeroed, so the group adds exactly 0 to the logit. The GQA query heads of the
+// copied with source size 0 (no bytes read, slot zero-filled), so the group
+// adds exactly 0 to the logit. In the row layout [Lmax, d] the skipped K
+// bytes only leave HBM untouched where a whole 128-byte line is out of
+// window; finer holes are fetched with their line. The GQA query heads of the
 // KV head (H_q/H_kv <= 8) form the rows of warp-level bf16 mma.sync products
 // (scores Q.K^T and P.V, fp32 accumulation); the online softmax keeps the row
 // max and row sum with warp shuffles. The 4 warps merge their states in
@@ -49,9 +51,6 @@ struct DecLayout {
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void st_shared_zero16(uint32_t dst) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -141,17 +140,12 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
       const bool valid = key < end;
       const int64_t dist = qpos - key;
       const bool kin = valid && dist <= static_cast<int64_t>(a.cut[p >> 1]);
-      // A piece nobody needs is not requested at all (a zero-size copy still
-      // costs its memory request); its shared-memory slot is zeroed instead,
-      // so an out-of-window group adds exactly 0 to the score.
-      if (kin)
-        cp_async16(kdst + piece_off<D>(r, p), kbase + static_cast<int64_t>(key) * D + 8 * p, 16u);
-      else
-        st_shared_zero16(kdst + piece_off<D>(r, p));
-      if (valid)
-        cp_async16(vdst + piece_off<D>(r, p), vbase + static_cast<int64_t>(key) * D + 8 * p, 16u);
-      else
-        st_shared_zero16(vdst + piece_off<D>(r, p));
+      // An out-of-window K piece is copied with source size 0: nothing is
+      // read and its shared-memory slot is zero-filled, so the group adds
+      // exactly 0 to the score.
+      const int64_t row = valid ? key : kb0;  // any in-range address when nothing is read
+      cp_async16(kdst + piece_off<D>(r, p), kbase + row * D + 8 * p, kin ? 16u : 0u);
+      cp_async16(vdst + piece_off<D>(r, p), vbase + row * D + 8 * p, valid ? 16u : 0u);
     }
   };
 

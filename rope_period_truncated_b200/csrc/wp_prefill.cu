@@ -6,33 +6,40 @@
 // then the usual causal softmax and O = A V. A masked group adds 0 to the
 // logit (detail 1 of §2.1), the pair stays in the softmax.
 //
-// How (one CTA per 128-row query tile of one query head, key tiles of 128
-// visited from the diagonal backwards; §2.3's skip / full / boundary class of
-// every (tile, group) comes from a per-CTA table built once in shared memory):
-//   warp 8  TMA producer: Q once (one 16-dim box per group); per key tile only
-//           the K column slices of non-skipped groups (16-dim boxes, 32-byte
-//           swizzle) and all of V (64-dim boxes, 128-byte swizzle).
-//   warp 9  MMA issuer: per key tile one tcgen05.mma (M=128, N=128, K=16) per
-//           non-skipped group; full groups accumulate into S_full (TMEM),
-//           boundary groups into the separate S_bnd accumulator, one distinct
-//           cutoff at a time in ascending order. Then P (bf16, written back
-//           into TMEM by the softmax warps) times V into the O accumulator.
-//   warps 0-7  two threads per query row (one per 64-key half of the tile):
-//           read S_full, add each boundary accumulator under its per-element
-//           mask, causal mask on the diagonal tile, agree on the row max with
-//           the partner warp, online softmax in base 2 with the scale folded
-//           into one FMA, write P to TMEM, rescale O only when a row max grows
-//           by more than 2^8; epilogue O/l -> bf16, LSE = ln(sum exp).
-// TMEM columns: [0, D) O, [128, 256) S_full buffer 0, [256, 384) buffer 1,
-// [384, 512) S_bnd. S_full is double-buffered so the QK MMAs of the next key
-// tile overlap the softmax of the current one.
+// How. One CTA takes one 128-row query tile of two query heads that share a
+// KV head (GQA), so every K/V tile it loads feeds both, and visits the key
+// tiles from the diagonal backwards. §2.3's skip / full / boundary class of
+// every (key tile, group) is the same for both heads and comes from a per-CTA
+// table built once in shared memory.
+//   warp 8  TMA producer: Q of both heads once (one 16-dim box per group); per
+//           key tile only the K column slices of non-skipped groups (16-dim
+//           boxes, 32-byte swizzle) and all of V (64-dim boxes, 128-byte
+//           swizzle).
+//   warp 9  MMA issuer (one elected lane, warp-uniform loop). Per key tile and
+//           head: one tcgen05.mma (M=128, N=128, K=16) per non-skipped group
+//           into that head's S accumulator in TMEM, then P (bf16, written back
+//           into S's columns by the softmax warps) times V into its O
+//           accumulator. The two heads ping-pong: PV(head 0), QK(head 0, next
+//           tile), PV(head 1), QK(head 1, next tile), so one head's softmax
+//           runs while the tensor core works for the other.
+//   warps 0-3 / 4-7  softmax of head 0 / head 1, one thread per query row:
+//           causal mask on the diagonal tile, online softmax in base 2 with
+//           the scale folded into one FMA, P to TMEM, O rescaled only when a
+//           row max grows by more than 2^8; epilogue O/l -> bf16 and
+//           LSE = ln(sum exp).
+// Boundary groups: the groups whose cutoff falls inside the tile's distance
+// range go first, one distinct cutoff at a time in ascending order; after each
+// class the softmax warps mask S in place (keep iff i - j <= W, else 0), and
+// the full groups then accumulate on top unmasked. Masks of ascending cutoffs
+// are nested, so m2*(m1*S1 + S2) = m1*S1 + m2*S2: the exact per-class mask.
+// TMEM columns: head s uses [256s, 256s+128) for S / P and [256s+128, 256s+256)
+// for O. If H_q/H_kv is odd the CTA takes a single head.
 //
-// The softmax is the non-tensor bottleneck (16384 exponentials per tile
-// against the MUFU unit's 16 per SM per clock), so 3 of every 8 pairs take
-// 2^x on the FMA pipe instead: Cody-Waite reduction x = j + f, |f| <= 1/2,
-// and a degree-3 minimax polynomial for 2^f (coefficients from a Remez fit,
-// max relative error 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in
-// the exponent field.
+// The softmax's exponentials (16384 per head and tile) compete with the MUFU
+// unit's 16 per SM per clock, so 3 of every 8 pairs take 2^x on the FMA pipe
+// instead: Cody-Waite reduction x = j + f, |f| <= 1/2, and a degree-3 minimax
+// polynomial for 2^f (coefficients from a Remez fit, max relative error
+// 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in the exponent field.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -47,43 +54,42 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int KST = 3;  // K stages
+constexpr int KST = 2;  // K stages
 constexpr int VST = 2;  // V stages
-constexpr int NTHREADS = 320;        // warps 0-7 softmax, 8 TMA producer, 9 MMA issuer
+constexpr int NTHREADS = 320;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9 MMA issuer
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
-constexpr int SOFTMAX_THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_O = 0;
-constexpr uint32_t COL_S0 = 128;
-constexpr uint32_t COL_SB = 384;
-constexpr uint32_t GROUP_TILE_BYTES = 128 * 32;     // 128 rows x 16 bf16
-constexpr uint32_t V_CHUNK_BYTES = 128 * 128;       // 128 keys x 64 bf16
+constexpr uint32_t GROUP_TILE_BYTES = 128 * 32;  // 128 rows x 16 bf16
+constexpr uint32_t V_CHUNK_BYTES = 128 * 128;    // 128 keys x 64 bf16
 constexpr uint32_t FULL = 0xffffffffu;
 
 // Row-max growth (base-2 units) below which O is not rescaled.
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
+__host__ __device__ constexpr uint32_t col_s(int slot) { return 256u * slot; }
+__host__ __device__ constexpr uint32_t col_o(int slot) { return 256u * slot + 128u; }
+
 template <int D>
 struct Layout {
   static constexpr int G = D / 16;
+  static constexpr uint32_t Q_SLOT = G * GROUP_TILE_BYTES;
   static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t K_OFF = Q_OFF + G * GROUP_TILE_BYTES;
+  static constexpr uint32_t K_OFF = Q_OFF + 2 * Q_SLOT;
   static constexpr uint32_t K_STAGE = G * GROUP_TILE_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + KST * K_STAGE;
   static constexpr uint32_t V_STAGE = (D / 64) * V_CHUNK_BYTES;
   static constexpr uint32_t BAR_OFF = V_OFF + VST * V_STAGE;
-  // + 4 warp pairs x (2 per-tile exchange barriers + 1 final exchange barrier)
-  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 + 2 + 2 + 1 + 1 + 12;
+  // q_full, k_full/empty, v_full/empty, per head s_ready/p_ready/o_ready/bnd_ready/bnd_done, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 * 5 + 1;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t XCH_OFF = MISC_OFF + 16;  // row-max exchange [2 parity][2 half][128 rows] + row sums
-  static constexpr uint32_t TT_OFF = XCH_OFF + (4 * 128 + 2 * 128) * 4;  // tile table: one uint16 per key tile
+  static constexpr uint32_t TT_OFF = MISC_OFF + 16;  // tile table: one uint16 per key tile
   static uint32_t bytes(int nqb) { return TT_OFF + ((2u * nqb + 15u) & ~15u) + 1024u; }  // + alignment slack
 };
 
 struct Barriers {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_ready, *bnd_ready, *bnd_free, *p_ready, *o_ready,
-      *drain, *pair, *pair_fin;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *bnd_ready, *bnd_done,
+      *drain;
 };
 
 // Class masks of tile (qb, kb): bits 0-7 full groups, bits 8-15 boundary groups.
@@ -128,7 +134,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long l
   return __all_sync(FULL, ok);
 }
 
-// 64 TMEM columns of this warp's lanes into r, one wait for both loads.
+// 64 TMEM columns of this warp's lanes into r, with one wait for both loads;
+// the registers pass through the wait so no use moves above it.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
   tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -185,6 +192,93 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __int_as_float(__float_as_int(p) + (ji << 23));
 }
 
+// 64 columns of S (or zeros when no group of the tile was computed).
+__device__ __forceinline__ void load_half(uint32_t taddr, bool any_group, uint32_t (&su)[64]) {
+  if (any_group) {
+    tmem_ld64(taddr, su);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) su[c] = 0u;
+  }
+}
+
+// Causal mask of the diagonal tile: key column c0 + c comes after row r.
+__device__ __forceinline__ void causal_mask(uint32_t (&su)[64], int c0, int r) {
+#pragma unroll
+  for (int c = 0; c < 64; ++c)
+    if (c0 + c > r) su[c] = __float_as_uint(-INFINITY);
+}
+
+// Max of 64 values: 4 independent chains of 3-input max.
+__device__ __forceinline__ float half_max(const uint32_t (&su)[64]) {
+  float mx4[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float m = __uint_as_float(su[16 * j]);
+#pragma unroll
+    for (int k = 1; k < 15; k += 2) m = max3(m, __uint_as_float(su[16 * j + k]), __uint_as_float(su[16 * j + k + 1]));
+    mx4[j] = fmaxf(m, __uint_as_float(su[16 * j + 15]));
+  }
+  return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+}
+
+// p = 2^(s*c2 - m) for 64 columns: one packed FMA per pair; 3 of every 8
+// pairs take the polynomial exp2, the rest the MUFU unit. Adds the p to the
+// four packed partial sums and writes them as bf16 pairs (32 TMEM columns)
+// to p_addr.
+__device__ __forceinline__ void exp_half(const uint32_t (&su)[64], uint64_t c2x2, float m, uint64_t (&acc)[4],
+                                         uint32_t p_addr) {
+  const uint64_t negm = pack_f2(-m, -m);
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[2 * k]), __uint_as_float(su[2 * k + 1])), c2x2, negm);
+    float x0, x1;
+    unpack_f2(x2, x0, x1);
+    float p0, p1;
+    if ((k & 7) >= 5) {
+      p0 = poly_exp2(x0);
+      p1 = poly_exp2(x1);
+    } else {
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    }
+    acc[k & 3] = fadd2(acc[k & 3], pack_f2(p0, p1));
+    pk[k] = pack_bf16x2(p0, p1);
+  }
+  tmem_st32(p_addr, pk);
+}
+
+// Multiply n32 x 32 fp32 TMEM columns of this warp's lanes by alpha.
+__device__ __forceinline__ void scale_cols_f32(uint32_t taddr, int n32, float alpha) {
+#pragma unroll 1
+  for (int c4 = 0; c4 < n32; ++c4) {
+    uint32_t u[32];
+    tmem_ld32(taddr + 32 * c4, u);
+    tmem_wait_ld(u);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * alpha);
+    tmem_st32(taddr + 32 * c4, u);
+  }
+  tmem_wait_st();
+}
+
+// Multiply 32 TMEM columns of bf16 pairs (P) of this warp's lanes by alpha.
+__device__ __forceinline__ void scale_cols_bf16x2(uint32_t taddr, float alpha) {
+  tmem_wait_st();  // the P being rescaled was just written by this thread
+  uint32_t u[32];
+  tmem_ld32(taddr, u);
+  tmem_wait_ld(u);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&u[k]);
+    const float2 f = __bfloat1622float2(v);
+    u[k] = pack_bf16x2(f.x * alpha, f.y * alpha);
+  }
+  tmem_st32(taddr, u);
+  tmem_wait_st();
+}
+
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_grouped_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -203,26 +297,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   B.k_empty = B.k_full + KST;
   B.v_full = B.k_empty + KST;
   B.v_empty = B.v_full + VST;
-  B.s_ready = B.v_empty + VST;
+  B.s_ready = B.v_empty + VST;  // [2 heads]
   B.p_ready = B.s_ready + 2;
-  B.bnd_ready = B.p_ready + 2;
-  B.bnd_free = B.bnd_ready + 1;
-  B.o_ready = B.bnd_free + 1;
-  B.drain = B.o_ready + 1;
-  B.pair = B.drain + 1;         // [4 pairs][2 parities]
-  B.pair_fin = B.pair + 8;      // [4 pairs]
+  B.o_ready = B.p_ready + 2;
+  B.bnd_ready = B.o_ready + 2;
+  B.bnd_done = B.bnd_ready + 2;
+  B.drain = B.bnd_done + 2;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
   uint16_t *ttab = reinterpret_cast<uint16_t *>(smem + L::TT_OFF);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
-  // Grid (query head within its KV group, query block, KV head x batch): the
+  // Grid (head pair within its KV group, query block, KV head x batch): the
   // CTAs that run together share one KV head, so its K/V stay in L2; within
   // a KV head the heaviest query blocks go first.
+  const int rep = a.Hq / a.Hkv;
+  const int nslot = (rep % 2 == 0) ? 2 : 1;
   const int hk = static_cast<int>(blockIdx.z) % a.Hkv;
   const int b = static_cast<int>(blockIdx.z) / a.Hkv;
-  const int h = hk * (a.Hq / a.Hkv) + static_cast<int>(blockIdx.x);
+  const int h0 = hk * rep + static_cast<int>(blockIdx.x) * nslot;  // head of slot s = h0 + s
   const int nqb = (a.N + BM - 1) / BM;
   const int qb = nqb - 1 - static_cast<int>(blockIdx.y);
   const long long lim = a.wait_limit;
@@ -241,14 +335,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_ready[s], 1);
-      mbar_init(&B.p_ready[s], SOFTMAX_THREADS);
+      mbar_init(&B.p_ready[s], 128);
+      mbar_init(&B.o_ready[s], 1);
+      mbar_init(&B.bnd_ready[s], 1);
+      mbar_init(&B.bnd_done[s], 128);
     }
-    mbar_init(B.bnd_ready, 1);
-    mbar_init(B.bnd_free, SOFTMAX_THREADS);
-    mbar_init(B.o_ready, 1);
     mbar_init(B.drain, 1);
-    for (int k = 0; k < 8; ++k) mbar_init(&B.pair[k], 64);
-    for (int k = 0; k < 4; ++k) mbar_init(&B.pair_fin[k], 64);
     fence_barrier_init();
   }
   // Tile table: key tile t = key block qb - t.
@@ -272,9 +364,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(B.q_full, G * GROUP_TILE_BYTES);
-      for (int g = 0; g < G; ++g)
-        tma_load_4d(smem + L::Q_OFF + g * GROUP_TILE_BYTES, &tm_q, B.q_full, 16 * g, h, qb * BM, b);
+      mbar_arrive_expect_tx(B.q_full, nslot * G * GROUP_TILE_BYTES);
+      for (int s = 0; s < nslot; ++s)
+        for (int g = 0; g < G; ++g)
+          tma_load_4d(smem + L::Q_OFF + s * L::Q_SLOT + g * GROUP_TILE_BYTES, &tm_q, B.q_full, 16 * g, h0 + s,
+                      qb * BM, b);
     }
     __syncwarp();
     int k_issued = 0, v_issued = 0;
@@ -338,228 +432,218 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // V tile: 128 keys x D, dims contiguous (MN-major), 128-byte swizzle;
     // 8-key row groups 1024 B apart, 64-dim chunks 16 KB apart.
     const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), V_CHUNK_BYTES, 1024, SMEM_SWIZZLE_128B);
-    int bnd_issued = 0;
+    int bnd_cnt[2] = {0, 0};
     bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
 
-    auto issue_qk = [&](int t) -> bool {
-      const int st = t % KST;
-      if (!warp_wait(&B.k_full[st], (t / KST) & 1, lim, abort_flag)) return false;
-      tc_fence_after();
+    // QK of head slot s for key tile t (its K stage already loaded).
+    auto issue_qk = [&](int s, int t) -> bool {
       const uint32_t tm = ttab[t];
-      const uint32_t s_col = tmem + COL_S0 + 128u * (t & 1);
-      const uint64_t kst_desc = k_desc + ((st * L::K_STAGE) >> 4);
+      const uint32_t s_col = tmem + col_s(s);
+      const uint64_t qs_desc = q_desc + ((s * L::Q_SLOT) >> 4);
+      const uint64_t kst_desc = k_desc + (((t % KST) * L::K_STAGE) >> 4);
       uint32_t acc = 0;
-      for (uint32_t m = tm & 0xffu; m; m &= m - 1) {
-        const uint32_t g = __ffs(m) - 1;
-        if (leader)
-          umma_ss(s_col, q_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
-                  acc);
-        acc = 1;
-      }
-      if (leader) umma_commit(&B.s_ready[t & 1]);
-      __syncwarp();
       const uint32_t bnd = tm >> 8;
       if (bnd) {
+        // boundary classes first, ascending cutoff; each one masked in place
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
         while (next_boundary_class(a, bnd, prev, &W, &cls)) {
-          if (bnd_issued > 0) {
-            if (!warp_wait(B.bnd_free, (bnd_issued - 1) & 1, lim, abort_flag)) return false;
-            tc_fence_after();
-          }
-          uint32_t bacc = 0;
           for (uint32_t m = cls; m; m &= m - 1) {
             const uint32_t g = __ffs(m) - 1;
             if (leader)
-              umma_ss(tmem + COL_SB, q_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4),
-                      IDESC_QK, bacc);
-            bacc = 1;
+              umma_ss(s_col, qs_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
+                      acc);
+            acc = 1;
           }
-          if (leader) umma_commit(B.bnd_ready);
+          if (leader) umma_commit(&B.bnd_ready[s]);
           __syncwarp();
-          ++bnd_issued;
+          if (!warp_wait(&B.bnd_done[s], bnd_cnt[s] & 1, lim, abort_flag)) return false;
+          tc_fence_after();
+          ++bnd_cnt[s];
           prev = W;
         }
       }
-      if (leader) umma_commit(&B.k_empty[st]);
+      for (uint32_t m = tm & 0xffu; m; m &= m - 1) {
+        const uint32_t g = __ffs(m) - 1;
+        if (leader)
+          umma_ss(s_col, qs_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
+                  acc);
+        acc = 1;
+      }
+      if (leader) umma_commit(&B.s_ready[s]);
       __syncwarp();
       return true;
     };
 
-    if (ok && nkb > 0) ok = issue_qk(0);
-    if (ok && nkb > 1) ok = issue_qk(1);
+    if (ok && nkb > 0) {
+      ok = warp_wait(&B.k_full[0], 0, lim, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int s = 0; ok && s < nslot; ++s) ok = issue_qk(s, 0);
+        if (ok && leader) umma_commit(&B.k_empty[0]);
+        __syncwarp();
+      }
+    }
     for (int t = 0; ok && t < nkb; ++t) {
-      const int sb = t & 1;
       const int vst = t % VST;
-      if (!warp_wait(&B.p_ready[sb], (t >> 1) & 1, lim, abort_flag) ||
-          !warp_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
+      if (!warp_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const uint32_t p_col = tmem + COL_S0 + 128u * sb;
       const uint64_t vst_desc = v_desc + ((vst * L::V_STAGE) >> 4);
+      for (int s = 0; ok && s < nslot; ++s) {
+        if (!warp_wait(&B.p_ready[s], t & 1, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t p_col = tmem + col_s(s);
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)
-        // P of keys 0-63 sits in S columns 0-31, of keys 64-127 in columns 64-95
-        if (leader)
-          umma_ts(tmem + COL_O, p_col + kk * 8 + (kk >= 4 ? 32 : 0), vst_desc + kk * (2048 >> 4), IDESC_PV,
-                  (t > 0 || kk > 0) ? 1u : 0u);
-      if (leader) {
-        umma_commit(&B.v_empty[vst]);
-        umma_commit(B.o_ready);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          if (leader)
+            umma_ts(tmem + col_o(s), p_col + kk * 8, vst_desc + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        if (leader) {
+          umma_commit(&B.o_ready[s]);
+          if (s == nslot - 1) umma_commit(&B.v_empty[vst]);
+        }
+        __syncwarp();
+        if (t + 1 < nkb) {
+          if (s == 0) {
+            if (!warp_wait(&B.k_full[(t + 1) % KST], ((t + 1) / KST) & 1, lim, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          ok = issue_qk(s, t + 1);
+          if (ok && s == nslot - 1) {
+            if (leader) umma_commit(&B.k_empty[(t + 1) % KST]);
+            __syncwarp();
+          }
+        }
       }
-      __syncwarp();
-      if (t + 2 < nkb) ok = issue_qk(t + 2);
     }
     // Every MMA this warp issued must finish before TMEM is released.
     if (leader) umma_commit(B.drain);
     __syncwarp();
     warp_wait(B.drain, 0, lim, nullptr);
-  } else {
+  } else if (warp / 4 < nslot) {
     // ------------------------------------------------------- softmax warps
-    // Warp w (0-7) owns rows 32*(w%4)..+31 — its TMEM lane quarter — and key
-    // columns 64*(w/4)..+63 of every tile: two warps share each row, which
-    // doubles the warps per scheduler that hide the softmax's latencies. The
-    // pair agrees on the row max through shared memory and an mbarrier
-    // (bounded wait). Every tcgen05.ld/st/wait below is .sync.aligned, so all
-    // waits are warp-uniform, the O-rescale decision is a warp vote (the same
-    // in both warps of a pair, as they see the same row maxima), and only the
-    // global stores of the padding rows of a ragged last tile are predicated.
-    const int q4 = warp & 3;
-    const int half = warp >> 2;
+    // Every tcgen05.ld/st/wait below is .sync.aligned: the whole warp must
+    // issue it together. So every wait is made warp-uniform (warp_wait), the
+    // O-rescale decision is a warp vote, and only the global stores of the
+    // padding rows of a ragged last tile are predicated.
+    const int slot = warp / 4;
+    const int q4 = warp % 4;
     const int r = q4 * 32 + lane;  // row of the query tile == TMEM lane
+    const int h = h0 + slot;
     const int64_t i = static_cast<int64_t>(qb) * BM + r;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t col0 = 64u * half;  // first key column of this warp
-    float *xch = reinterpret_cast<float *>(smem + L::XCH_OFF);
+    const uint32_t s_addr = lane_addr + col_s(slot);
+    const uint32_t o_addr = lane_addr + col_o(slot);
     const float c2 = a.scale_log2;  // logits to base-2 exponent units
     const uint64_t c2x2 = pack_f2(c2, c2);
-    float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units), this half's sum
-    int bnd_used = 0;
+    float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units) and sum
+    int bnd_cnt = 0;
     bool ok = true;
     for (int t = 0; t < nkb; ++t) {
       const int kb = qb - t;
-      const int sb = t & 1;
       const uint32_t tm = ttab[t];
-      ok = warp_wait(&B.s_ready[sb], (t >> 1) & 1, lim, abort_flag);
-      const uint32_t s_addr = lane_addr + COL_S0 + 128u * sb + col0;
-      uint32_t su[64];
-      float mh = -INFINITY;
-      if (ok) {
-        tc_fence_after();
-        if (tm & 0xffu) {
-          tmem_ld64(s_addr, su);
-        } else {
+      const uint32_t bnd = tm >> 8;
+      const bool any_group = (tm & 0xffffu) != 0;
+      if (bnd) {
+        // Mask S in place after each boundary class: keep column c iff
+        // (i - kb*BN) - c <= W, i.e. c >= cmin; otherwise 0.
+        int64_t prev = -1;
+        int32_t W;
+        uint32_t cls;
+        while (next_boundary_class(a, bnd, prev, &W, &cls)) {
+          ok = warp_wait(&B.bnd_ready[slot], bnd_cnt & 1, lim, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const int64_t cmin64 = i - static_cast<int64_t>(kb) * BN - W;
+          const int cmin = cmin64 < 0 ? 0 : (cmin64 > BN ? BN : static_cast<int>(cmin64));
 #pragma unroll
-          for (int c = 0; c < 64; ++c) su[c] = 0u;
-        }
-        const uint32_t bnd = tm >> 8;
-        if (bnd) {
-          // Boundary accumulators, one distinct cutoff at a time: keep the
-          // element iff its distance i - j is within the cutoff.
-          int64_t prev = -1;
-          int32_t W;
-          uint32_t cls;
-          while (ok && next_boundary_class(a, bnd, prev, &W, &cls)) {
-            ok = warp_wait(B.bnd_ready, bnd_used & 1, lim, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t ub[64];
-            tmem_ld64(lane_addr + COL_SB + col0, ub);
-            tc_fence_before();
-            mbar_arrive(B.bnd_free);
-            ++bnd_used;
-            prev = W;
-            // keep column col0 + c iff (i - kb*BN - col0) - c <= W
-            const int64_t cmin64 = i - static_cast<int64_t>(kb) * BN - col0 - W;
-            const int cmin = cmin64 < 0 ? 0 : (cmin64 > 64 ? 64 : static_cast<int>(cmin64));
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t su[64];
+            tmem_ld64(s_addr + 64 * hf, su);
 #pragma unroll
             for (int c = 0; c < 64; ++c)
-              if (c >= cmin) su[c] = __float_as_uint(__uint_as_float(su[c]) + __uint_as_float(ub[c]));
+              if (64 * hf + c < cmin) su[c] = 0u;
+            tmem_st32(s_addr + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+            tmem_st32(s_addr + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&B.bnd_done[slot]);
+          ++bnd_cnt;
+          prev = W;
         }
-        // Causal mask: only the diagonal tile has keys after the query.
-        if (kb == qb) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (static_cast<int>(col0) + c > r) su[c] = __float_as_uint(-INFINITY);
-        }
-        // Half-row max: 4 independent chains of 3-input max.
-        float mx4[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float m = __uint_as_float(su[16 * j]);
-#pragma unroll
-          for (int k = 1; k < 15; k += 2)
-            m = max3(m, __uint_as_float(su[16 * j + k]), __uint_as_float(su[16 * j + k + 1]));
-          mx4[j] = fmaxf(m, __uint_as_float(su[16 * j + 15]));
-        }
-        mh = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        if (!ok) break;
       }
-      // Exchange half-row maxima with the partner warp (NaN = "aborted").
-      float *xc = xch + (t & 1) * 256;
-      xc[half * 128 + r] = ok ? mh : __int_as_float(0x7fc00000);
-      mbar_arrive(&B.pair[q4 * 2 + (t & 1)]);
-      const bool pok = warp_wait(&B.pair[q4 * 2 + (t & 1)], (t >> 1) & 1, lim, abort_flag);
-      const float mp = xc[(half ^ 1) * 128 + r];
-      if (!__all_sync(FULL, ok && pok && !isnan(mp))) {
+      if (!warp_wait(&B.s_ready[slot], t & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
-      const float m_tile = fmaxf(mh, mp) * c2;  // scale > 0, so the max commutes with it
+      tc_fence_after();
+      const uint64_t zero2 = 0ull;
+      uint64_t acc[4] = {zero2, zero2, zero2, zero2};
       if (t == 0) {
-        m_run = m_tile;  // the diagonal tile always holds key j = i
-      } else if (__any_sync(FULL, m_tile > m_run + RESCALE_THRESHOLD)) {
-        // Rescale only when some row's max grew by more than 2^8: otherwise
-        // the stale max stays exact (p <= 2^8 fits bf16 P and fp32 sums).
-        const float m_new = fmaxf(m_run, m_tile);
-        const float alpha = fast_exp2(m_run - m_new);
-        // O holds the sum through key tile t-1: wait for that PV, rescale
-        // this half's D/2 columns of O.
-        if (!warp_wait(B.o_ready, (t - 1) & 1, lim, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c4 = 0; c4 < D / 64; ++c4) {
-          uint32_t u[32];
-          const uint32_t oc = lane_addr + COL_O + half * (D / 2) + 32 * c4;
-          tmem_ld32(oc, u);
-          tmem_wait_ld(u);
+        // Diagonal tile: causal mask, and the row max from both halves first
+        // (the running max starts here), then a second read for the exps.
+        float mx = -INFINITY;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) u[k] = __float_as_uint(__uint_as_float(u[k]) * alpha);
-          tmem_st32(oc, u);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t su[64];
+          load_half(s_addr + 64 * hf, any_group, su);
+          causal_mask(su, 64 * hf, r);
+          mx = fmaxf(mx, half_max(su));
         }
-        tmem_wait_st();
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      // p = 2^(s*c2 - m): one packed FMA per pair; 3 of every 8 pairs take
-      // the polynomial exp2, the rest the MUFU unit. Four packed partial sums.
-      // P (bf16 pairs) goes back into this warp's own S columns.
-      const uint64_t negm = pack_f2(-m_run, -m_run);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      uint32_t pk[32];
+        m_run = mx * c2;  // scale > 0, so the max commutes with it
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[2 * k]), __uint_as_float(su[2 * k + 1])), c2x2, negm);
-        float x0, x1;
-        unpack_f2(x2, x0, x1);
-        float p0, p1;
-        if ((k & 7) >= 5) {
-          p0 = poly_exp2(x0);
-          p1 = poly_exp2(x1);
-        } else {
-          p0 = fast_exp2(x0);
-          p1 = fast_exp2(x1);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t su[64];
+          load_half(s_addr + 64 * hf, any_group, su);
+          causal_mask(su, 64 * hf, r);
+          exp_half(su, c2x2, m_run, acc, s_addr + 32 * hf);
         }
-        acc[k & 3] = fadd2(acc[k & 3], pack_f2(p0, p1));
-        pk[k] = pack_bf16x2(p0, p1);
+      } else {
+        // One read of S per half: exponentiate against the running max right
+        // away, unless some row's max grew by more than 2^8 (rare): then O, the
+        // row sum and the P already written for the first half are rescaled.
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t su[64];
+          load_half(s_addr + 64 * hf, any_group, su);
+          const float m_half = half_max(su) * c2;
+          if (__any_sync(FULL, m_half > m_run + RESCALE_THRESHOLD)) {
+            const float m_new = fmaxf(m_run, m_half);
+            const float alpha = fast_exp2(m_run - m_new);
+            // O holds the sum through key tile t-1: wait for that PV.
+            if (!warp_wait(&B.o_ready[slot], (t - 1) & 1, lim, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            scale_cols_f32(o_addr, D / 32, alpha);
+            if (hf == 1) scale_cols_bf16x2(s_addr, alpha);  // P of keys 0-63
+            float a0, a1;
+            unpack_f2(acc[0], a0, a1);
+            acc[0] = pack_f2(a0 * alpha, a1 * alpha);
+            unpack_f2(acc[1], a0, a1);
+            acc[1] = pack_f2(a0 * alpha, a1 * alpha);
+            unpack_f2(acc[2], a0, a1);
+            acc[2] = pack_f2(a0 * alpha, a1 * alpha);
+            unpack_f2(acc[3], a0, a1);
+            acc[3] = pack_f2(a0 * alpha, a1 * alpha);
+            l_run *= alpha;
+            m_run = m_new;
+          }
+          exp_half(su, c2x2, m_run, acc, s_addr + 32 * hf);
+        }
+        if (!ok) break;
       }
-      tmem_st32(s_addr, pk);
       float s0, s1, s2, s3, s4, s5, s6, s7;
       unpack_f2(acc[0], s0, s1);
       unpack_f2(acc[1], s2, s3);
@@ -568,24 +652,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&B.p_ready[sb]);
+      mbar_arrive(&B.p_ready[slot]);
     }
-    // Row sum = both halves' sums: one more exchange, then this half's D/2
-    // output columns.
-    float *ls = xch + 512;
-    ls[half * 128 + r] = ok ? l_run : __int_as_float(0x7fc00000);
-    mbar_arrive(&B.pair_fin[q4]);
-    const bool fok = warp_wait(&B.pair_fin[q4], 0, lim, abort_flag);
-    const float l_row = l_run + ls[(half ^ 1) * 128 + r];
-    if (__all_sync(FULL, ok && fok && !isnan(l_row)) && nkb > 0 &&
-        warp_wait(B.o_ready, (nkb - 1) & 1, lim, abort_flag)) {
+    if (ok && nkb > 0 && warp_wait(&B.o_ready[slot], (nkb - 1) & 1, lim, abort_flag)) {
       tc_fence_after();
-      const float inv_l = 1.f / l_row;
-      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D + half * (D / 2);
+      const float inv_l = 1.f / l_run;
+      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 64; ++c4) {
+      for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t u[32];
-        tmem_ld32(lane_addr + COL_O + half * (D / 2) + 32 * c4, u);
+        tmem_ld32(o_addr + 32 * c4, u);
         tmem_wait_ld(u);
         uint4 pk4[4];
         uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
@@ -598,8 +674,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
         }
       }
-      if (half == 0 && i < a.N && a.lse != nullptr)
-        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_row)) * 0.69314718055994531f;
+      if (i < a.N && a.lse != nullptr)
+        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     } else {
       // Tell the other roles to stop waiting for this warp's progress.
       *abort_flag = 1;
@@ -626,7 +702,9 @@ static cudaError_t launch_grouped(const CUtensorMap &tq, const CUtensorMap &tk, 
   cudaError_t e = cudaFuncSetAttribute(prefill_grouped_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hq / a.Hkv, nqb, a.Hkv * a.B);
+  const int rep = a.Hq / a.Hkv;
+  const int nslot = (rep % 2 == 0) ? 2 : 1;
+  dim3 grid(rep / nslot, nqb, a.Hkv * a.B);
   prefill_grouped_kernel<D><<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   return cudaGetLastError();
 }
