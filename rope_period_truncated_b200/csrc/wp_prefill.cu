@@ -36,8 +36,8 @@
 // for O. If H_q/H_kv is odd the CTA takes a single head.
 //
 // The softmax's exponentials (16384 per head and tile) compete with the MUFU
-// unit's 16 per SM per clock, so 3 of every 8 pairs take 2^x on the FMA pipe
-// instead: Cody-Waite reduction x = j + f, |f| <= 1/2, and a degree-3 minimax
+// unit's 16 per SM per clock, so POLY_PAIRS of every 8 pairs take 2^x on the
+// FMA pipe instead, in packed f32x2 arithmetic: Cody-Waite reduction x = j + f, |f| <= 1/2, and a degree-3 minimax
 // polynomial for 2^f (coefficients from a Remez fit, max relative error
 // 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in the exponent field.
 #include <cuda.h>
@@ -66,6 +66,11 @@ constexpr uint32_t FULL = 0xffffffffu;
 
 // Row-max growth (base-2 units) below which O is not rescaled.
 constexpr float RESCALE_THRESHOLD = 8.0f;
+#ifndef WP_POLY_PAIRS
+#define WP_POLY_PAIRS 1
+#endif
+constexpr int POLY_PAIRS = WP_POLY_PAIRS;  // of every 8 exponent pairs, on the FMA pipe
+static_assert(POLY_PAIRS >= 0 && POLY_PAIRS <= 8, "POLY_PAIRS counts pairs out of 8");
 
 __host__ __device__ constexpr uint32_t col_s(int slot) { return 256u * slot; }
 __host__ __device__ constexpr uint32_t col_o(int slot) { return 256u * slot + 128u; }
@@ -178,18 +183,33 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x on the FMA pipe (see the file comment). x below -120 returns ~2^-120,
-// which is 0 for every sum this kernel forms.
-__device__ __forceinline__ float poly_exp2(float x) {
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of exponents on the FMA pipe (see the file comment), in
+// packed f32x2 arithmetic. x below -120 gives ~2^-120, which is 0 for every
+// sum this kernel forms.
+__device__ __forceinline__ void poly_exp2x2(uint64_t x2, float &p0, float &p1) {
   constexpr float C0 = 0.99992806f, C1 = 0.69326097f, C2 = 0.24261113f, C3 = 0.05517167f;
   constexpr float ROUND = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-  x = fmaxf(x, -120.f);
-  const float t = x + ROUND;
-  const float j = t - ROUND;
-  const float f = x - j;
-  const float p = fmaf(fmaf(fmaf(C3, f, C2), f, C1), f, C0);
-  const int ji = __float_as_int(t) - __float_as_int(ROUND);
-  return __int_as_float(__float_as_int(p) + (ji << 23));
+  float x0, x1;
+  unpack_f2(x2, x0, x1);
+  x2 = pack_f2(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
+  const uint64_t t2 = fadd2(x2, pack_f2(ROUND, ROUND));   // low mantissa bits hold j = rint(x)
+  const uint64_t f2 = fsub2(x2, fsub2(t2, pack_f2(ROUND, ROUND)));  // f = x - j in [-1/2, 1/2]
+  uint64_t q2 = ffma2(pack_f2(C3, C3), f2, pack_f2(C2, C2));
+  q2 = ffma2(q2, f2, pack_f2(C1, C1));
+  q2 = ffma2(q2, f2, pack_f2(C0, C0));
+  float t0, t1;
+  unpack_f2(t2, t0, t1);
+  unpack_f2(q2, p0, p1);
+  // 2^j * 2^f: add j to the exponent field. The bits of t are those of ROUND
+  // plus j, and ROUND's own bits vanish from a 23-bit left shift.
+  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // 64 columns of S (or zeros when no group of the tile was computed).
@@ -222,7 +242,7 @@ __device__ __forceinline__ float half_max(const uint32_t (&su)[64]) {
   return fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
 }
 
-// p = 2^(s*c2 - m) for 64 columns: one packed FMA per pair; 3 of every 8
+// p = 2^(s*c2 - m) for 64 columns: one packed FMA per pair; POLY_PAIRS of 8
 // pairs take the polynomial exp2, the rest the MUFU unit. Adds the p to the
 // four packed partial sums and writes them as bf16 pairs (32 TMEM columns)
 // to p_addr.
@@ -236,9 +256,8 @@ __device__ __forceinline__ void exp_half(const uint32_t (&su)[64], uint64_t c2x2
     float x0, x1;
     unpack_f2(x2, x0, x1);
     float p0, p1;
-    if ((k & 7) >= 5) {
-      p0 = poly_exp2(x0);
-      p1 = poly_exp2(x1);
+    if ((k & 7) >= 8 - POLY_PAIRS) {
+      poly_exp2x2(x2, p0, p1);
     } else {
       p0 = fast_exp2(x0);
       p1 = fast_exp2(x1);
@@ -335,10 +354,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&B.s_ready[s], 1);
-      mbar_init(&B.p_ready[s], 128);
+      mbar_init(&B.p_ready[s], 4);  // one arrival per softmax warp
       mbar_init(&B.o_ready[s], 1);
       mbar_init(&B.bnd_ready[s], 1);
-      mbar_init(&B.bnd_done[s], 128);
+      mbar_init(&B.bnd_done[s], 4);
     }
     mbar_init(B.drain, 1);
     fence_barrier_init();
@@ -435,6 +454,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int bnd_cnt[2] = {0, 0};
     bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
 
+    // One MMA per group of `groups` (issued by the elected lane alone, in one
+    // branch), accumulating after the first.
+    auto issue_groups = [&](uint32_t s_col, uint64_t qs_desc, uint64_t kst_desc, uint32_t groups, uint32_t acc) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (groups & (1u << g)) {
+          umma_ss(s_col, qs_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
+                  acc);
+          acc = 1;
+        }
+      }
+    };
     // QK of head slot s for key tile t (its K stage already loaded).
     auto issue_qk = [&](int s, int t) -> bool {
       const uint32_t tm = ttab[t];
@@ -449,14 +480,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int32_t W;
         uint32_t cls;
         while (next_boundary_class(a, bnd, prev, &W, &cls)) {
-          for (uint32_t m = cls; m; m &= m - 1) {
-            const uint32_t g = __ffs(m) - 1;
-            if (leader)
-              umma_ss(s_col, qs_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
-                      acc);
-            acc = 1;
+          if (leader) {
+            issue_groups(s_col, qs_desc, kst_desc, cls, acc);
+            umma_commit(&B.bnd_ready[s]);
           }
-          if (leader) umma_commit(&B.bnd_ready[s]);
+          acc = 1;
           __syncwarp();
           if (!warp_wait(&B.bnd_done[s], bnd_cnt[s] & 1, lim, abort_flag)) return false;
           tc_fence_after();
@@ -464,14 +492,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           prev = W;
         }
       }
-      for (uint32_t m = tm & 0xffu; m; m &= m - 1) {
-        const uint32_t g = __ffs(m) - 1;
-        if (leader)
-          umma_ss(s_col, qs_desc + g * (GROUP_TILE_BYTES >> 4), kst_desc + g * (GROUP_TILE_BYTES >> 4), IDESC_QK,
-                  acc);
-        acc = 1;
+      if (leader) {
+        issue_groups(s_col, qs_desc, kst_desc, tm & 0xffu, acc);
+        umma_commit(&B.s_ready[s]);
       }
-      if (leader) umma_commit(&B.s_ready[s]);
       __syncwarp();
       return true;
     };
@@ -499,11 +523,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_after();
         const uint32_t p_col = tmem + col_s(s);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          if (leader)
-            umma_ts(tmem + col_o(s), p_col + kk * 8, vst_desc + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_ts(tmem + col_o(s), p_col + kk * 8, vst_desc + kk * (2048 >> 4), IDESC_PV,
+                    (t > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&B.o_ready[s]);
           if (s == nslot - 1) umma_commit(&B.v_empty[vst]);
         }
@@ -576,7 +600,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&B.bnd_done[slot]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.bnd_done[slot]);
           ++bnd_cnt;
           prev = W;
         }
@@ -652,7 +677,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&B.p_ready[slot]);
+      __syncwarp();  // the warp's TMEM stores are ordered before lane 0's arrival
+      if (lane == 0) mbar_arrive(&B.p_ready[slot]);
     }
     if (ok && nkb > 0 && warp_wait(&B.o_ready[slot], (nkb - 1) & 1, lim, abort_flag)) {
       tc_fence_after();
