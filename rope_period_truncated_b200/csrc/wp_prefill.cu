@@ -53,12 +53,13 @@ namespace wp {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BN = 128;
+constexpr int BN = 128;   // key tile of the K/V loads
+constexpr int SUB = 64;   // key sub-tile of one S buffer (two per head, double-buffered)
 constexpr int KST = 2;  // K stages
 constexpr int VST = 2;  // V stages
-constexpr int NTHREADS = 320;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9 MMA issuer
+constexpr int NTHREADS = 352;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9/10 MMA issuer of head 0/1
 constexpr int PRODUCER_WARP = 8;
-constexpr int MMA_WARP = 9;
+constexpr int MMA_WARP = 9;  // head s is issued by warp MMA_WARP + s; this one also owns TMEM
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t GROUP_TILE_BYTES = 128 * 32;  // 128 rows x 16 bf16
 constexpr uint32_t V_CHUNK_BYTES = 128 * 128;    // 128 keys x 64 bf16
@@ -85,23 +86,25 @@ struct Layout {
   static constexpr uint32_t V_OFF = K_OFF + KST * K_STAGE;
   static constexpr uint32_t V_STAGE = (D / 64) * V_CHUNK_BYTES;
   static constexpr uint32_t BAR_OFF = V_OFF + VST * V_STAGE;
-  // q_full, k_full/empty, v_full/empty, per head s_ready/p_ready/o_ready/bnd_ready/bnd_done, drain
-  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 * 5 + 1;
+  // q_full, k_full/empty, v_full/empty, per head x half s_ready/p_ready, per head
+  // o_ready/o_final/bnd_ready/bnd_done, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 * 4 + 2 * 4 + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t TT_OFF = MISC_OFF + 16;  // tile table: one uint16 per key tile
-  static uint32_t bytes(int nqb) { return TT_OFF + ((2u * nqb + 15u) & ~15u) + 1024u; }  // + alignment slack
+  static constexpr uint32_t TT_OFF = MISC_OFF + 16;  // sub-tile table: one uint16 per 64-key sub-tile
+  static uint32_t bytes(int nqb) { return TT_OFF + ((4u * nqb + 15u) & ~15u) + 1024u; }  // + alignment slack
 };
 
 struct Barriers {
-  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *bnd_ready, *bnd_done,
-      *drain;
+  uint64_t *q_full, *k_full, *k_empty, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *o_final, *bnd_ready,
+      *bnd_done, *drain;
 };
 
-// Class masks of tile (qb, kb): bits 0-7 full groups, bits 8-15 boundary groups.
-__device__ __forceinline__ uint32_t tile_masks(const PrefillArgs &a, int G, int64_t qb, int64_t kb) {
+// Class masks of the 128-query x 64-key block (qb, kb64): bits 0-7 full
+// groups, bits 8-15 boundary groups.
+__device__ __forceinline__ uint32_t sub_masks(const PrefillArgs &a, int G, int64_t qb, int64_t kb64) {
   int64_t dmin = 0, dmax = -1;
   uint32_t full = 0, bnd = 0;
-  if (tile_distance_range(a.N, BM, BN, qb, kb, &dmin, &dmax)) {
+  if (tile_distance_range(a.N, BM, SUB, qb, kb64, &dmin, &dmax)) {
     for (int g = 0; g < G; ++g) {
       const int c = classify_cutoff(dmin, dmax, a.cut[g]);
       if (c == TILE_FULL) full |= 1u << g;
@@ -282,29 +285,13 @@ __device__ __forceinline__ void scale_cols_f32(uint32_t taddr, int n32, float al
   tmem_wait_st();
 }
 
-// Multiply 32 TMEM columns of bf16 pairs (P) of this warp's lanes by alpha.
-__device__ __forceinline__ void scale_cols_bf16x2(uint32_t taddr, float alpha) {
-  tmem_wait_st();  // the P being rescaled was just written by this thread
-  uint32_t u[32];
-  tmem_ld32(taddr, u);
-  tmem_wait_ld(u);
-#pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&u[k]);
-    const float2 f = __bfloat1622float2(v);
-    u[k] = pack_bf16x2(f.x * alpha, f.y * alpha);
-  }
-  tmem_st32(taddr, u);
-  tmem_wait_st();
-}
-
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_grouped_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
   using L = Layout<D>;
   constexpr int G = L::G;
-  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, SUB, false, false);
   constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
 
   extern __shared__ uint8_t smem_raw[];
@@ -316,10 +303,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   B.k_empty = B.k_full + KST;
   B.v_full = B.k_empty + KST;
   B.v_empty = B.v_full + VST;
-  B.s_ready = B.v_empty + VST;  // [2 heads]
-  B.p_ready = B.s_ready + 2;
-  B.o_ready = B.p_ready + 2;
-  B.bnd_ready = B.o_ready + 2;
+  B.s_ready = B.v_empty + VST;  // [2 heads][2 halves]
+  B.p_ready = B.s_ready + 4;    // [2 heads][2 halves]
+  B.o_ready = B.p_ready + 4;
+  B.o_final = B.o_ready + 2;  // completes once, after the last PV of the head
+  B.bnd_ready = B.o_final + 2;
   B.bnd_done = B.bnd_ready + 2;
   B.drain = B.bnd_done + 2;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
@@ -346,24 +334,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(B.q_full, 1);
     for (int s = 0; s < KST; ++s) {
       mbar_init(&B.k_full[s], 1);
-      mbar_init(&B.k_empty[s], 1);
+      mbar_init(&B.k_empty[s], nslot);  // one commit per head's MMA warp
     }
     for (int s = 0; s < VST; ++s) {
       mbar_init(&B.v_full[s], 1);
-      mbar_init(&B.v_empty[s], 1);
+      mbar_init(&B.v_empty[s], nslot);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&B.s_ready[s], 1);
       mbar_init(&B.p_ready[s], 4);  // one arrival per softmax warp
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&B.o_ready[s], 1);
+      mbar_init(&B.o_final[s], 1);
       mbar_init(&B.bnd_ready[s], 1);
       mbar_init(&B.bnd_done[s], 4);
     }
-    mbar_init(B.drain, 1);
+    mbar_init(&B.drain[0], 1);
+    mbar_init(&B.drain[1], 1);
     fence_barrier_init();
   }
-  // Tile table: key tile t = key block qb - t.
-  for (int t = threadIdx.x; t <= qb; t += NTHREADS) ttab[t] = static_cast<uint16_t>(tile_masks(a, G, qb, qb - t));
+  // Sub-tile table: sub-tile u = 2t + h holds the keys of 64-key block
+  // 2(qb - t) + h, i.e. half h of key tile t.
+  for (int u = threadIdx.x; u < 2 * (qb + 1); u += NTHREADS)
+    ttab[u] = static_cast<uint16_t>(sub_masks(a, G, qb, 2 * (qb - u / 2) + (u & 1)));
   if (warp == MMA_WARP) {
     tmem_alloc(tmem_base_slot, TMEM_COLS);
     tmem_relinquish();
@@ -373,6 +367,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
   const int nkb = *abort_flag ? 0 : qb + 1;  // key tiles qb, qb-1, ..., 0 (BM == BN)
+  const int nsub = 2 * nkb;
 
   if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
@@ -413,8 +408,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         break;
       }
       const int kb = qb - t;
-      const uint32_t tm = ttab[t];
-      const uint32_t need = (tm | (tm >> 8)) & 0xffu;
+      const uint32_t m0 = ttab[2 * t], m1 = ttab[2 * t + 1];
+      const uint32_t need = (m0 | (m0 >> 8) | m1 | (m1 >> 8)) & 0xffu;  // groups either half computes
       if (leader) {
         mbar_arrive_expect_tx(&B.k_full[st], __popc(need) * GROUP_TILE_BYTES);
         for (uint32_t m = need; m; m &= m - 1) {
@@ -439,10 +434,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int last = s + ((v_issued - 1 - s) / VST) * VST;
       warp_wait(&B.v_full[s], (last / VST) & 1, lim, nullptr);
     }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the issue loop: control flow and descriptors are
-    // warp-uniform, and one elected lane issues each tcgen05.mma / commit.
+  } else if (warp >= MMA_WARP && warp < MMA_WARP + nslot) {
+    // ------------------------------------------------------- MMA issuers
+    // Warp MMA_WARP + s issues head slot s: the whole warp runs the issue
+    // loop (control flow and descriptors are warp-uniform) and one elected
+    // lane issues each group of tcgen05.mma / commit in one branch. The two
+    // heads' loops run side by side; tcgen05.commit tracks the MMAs of the
+    // issuing thread only, so each head's barriers see its own MMAs.
+    const int s = warp - MMA_WARP;
     const bool leader = elect_one();
     // Descriptor bases; a byte offset within shared memory is added to the
     // start-address field (bits 0-13, in 16-byte units).
@@ -451,11 +450,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // V tile: 128 keys x D, dims contiguous (MN-major), 128-byte swizzle;
     // 8-key row groups 1024 B apart, 64-dim chunks 16 KB apart.
     const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), V_CHUNK_BYTES, 1024, SMEM_SWIZZLE_128B);
-    int bnd_cnt[2] = {0, 0};
+    int bnd_cnt = 0;
     bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
 
-    // One MMA per group of `groups` (issued by the elected lane alone, in one
-    // branch), accumulating after the first.
+    // One MMA (M=128, N=64, K=16) per group of `groups`, accumulating after
+    // the first.
     auto issue_groups = [&](uint32_t s_col, uint64_t qs_desc, uint64_t kst_desc, uint32_t groups, uint32_t acc) {
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -466,12 +465,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     };
-    // QK of head slot s for key tile t (its K stage already loaded).
-    auto issue_qk = [&](int s, int t) -> bool {
-      const uint32_t tm = ttab[t];
-      const uint32_t s_col = tmem + col_s(s);
+    // QK of this head for sub-tile u into S half u & 1 (its K stage loaded).
+    auto issue_qk = [&](int u) -> bool {
+      const uint32_t tm = ttab[u];
+      const int t = u >> 1, hh = u & 1;
+      const uint32_t s_col = tmem + col_s(s) + SUB * hh;
       const uint64_t qs_desc = q_desc + ((s * L::Q_SLOT) >> 4);
-      const uint64_t kst_desc = k_desc + (((t % KST) * L::K_STAGE) >> 4);
+      // key rows 64*hh.. of every K group tile (32 bytes per row)
+      const uint64_t kst_desc = k_desc + (((t % KST) * L::K_STAGE + hh * SUB * 32) >> 4);
       uint32_t acc = 0;
       const uint32_t bnd = tm >> 8;
       if (bnd) {
@@ -486,15 +487,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           acc = 1;
           __syncwarp();
-          if (!warp_wait(&B.bnd_done[s], bnd_cnt[s] & 1, lim, abort_flag)) return false;
+          if (!warp_wait(&B.bnd_done[s], bnd_cnt & 1, lim, abort_flag)) return false;
           tc_fence_after();
-          ++bnd_cnt[s];
+          ++bnd_cnt;
           prev = W;
         }
       }
       if (leader) {
         issue_groups(s_col, qs_desc, kst_desc, tm & 0xffu, acc);
-        umma_commit(&B.s_ready[s]);
+        umma_commit(&B.s_ready[2 * s + hh]);
       }
       __syncwarp();
       return true;
@@ -504,54 +505,63 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ok = warp_wait(&B.k_full[0], 0, lim, abort_flag);
       if (ok) {
         tc_fence_after();
-        for (int s = 0; ok && s < nslot; ++s) ok = issue_qk(s, 0);
+        ok = issue_qk(0);
+        if (ok) ok = issue_qk(1);
         if (ok && leader) umma_commit(&B.k_empty[0]);
         __syncwarp();
       }
     }
-    for (int t = 0; ok && t < nkb; ++t) {
+    // Per sub-tile u and head: PV(u) as soon as P(u) is in TMEM, then
+    // QK(u + 2) into the S half that P(u) frees (the tensor core runs them in
+    // order); S(u + 1) was issued one step earlier, so the softmax never
+    // waits for the MMAs that follow its own P.
+    for (int u = 0; ok && u < nsub; ++u) {
+      const int t = u >> 1, hh = u & 1;
       const int vst = t % VST;
-      if (!warp_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
+      if (hh == 0 && !warp_wait(&B.v_full[vst], (t / VST) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       const uint64_t vst_desc = v_desc + ((vst * L::V_STAGE) >> 4);
-      for (int s = 0; ok && s < nslot; ++s) {
-        if (!warp_wait(&B.p_ready[s], t & 1, lim, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t p_col = tmem + col_s(s);
-        if (leader) {
+      // one barrier per S half: the softmax of the other half may already
+      // have arrived for the next sub-tile
+      if (!warp_wait(&B.p_ready[2 * s + hh], t & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t p_col = tmem + col_s(s) + SUB * hh;
+      if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_ts(tmem + col_o(s), p_col + kk * 8, vst_desc + kk * (2048 >> 4), IDESC_PV,
-                    (t > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&B.o_ready[s]);
-          if (s == nslot - 1) umma_commit(&B.v_empty[vst]);
+        for (int kk = 0; kk < SUB / 16; ++kk)
+          umma_ts(tmem + col_o(s), p_col + kk * 8, vst_desc + (hh * (SUB / 16) + kk) * (2048 >> 4), IDESC_PV,
+                  (u > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&B.o_ready[s]);
+        if (u == nsub - 1) umma_commit(&B.o_final[s]);
+        if (hh == 1) umma_commit(&B.v_empty[vst]);
+      }
+      __syncwarp();
+      if (u + 2 < nsub) {
+        if (hh == 0) {
+          // QK(u + 2) opens key tile t + 1
+          if (!warp_wait(&B.k_full[(t + 1) % KST], ((t + 1) / KST) & 1, lim, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
         }
-        __syncwarp();
-        if (t + 1 < nkb) {
-          if (s == 0) {
-            if (!warp_wait(&B.k_full[(t + 1) % KST], ((t + 1) / KST) & 1, lim, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          ok = issue_qk(s, t + 1);
-          if (ok && s == nslot - 1) {
-            if (leader) umma_commit(&B.k_empty[(t + 1) % KST]);
-            __syncwarp();
-          }
+        ok = issue_qk(u + 2);
+        if (ok && hh == 1) {
+          // QK(u + 2) closed key tile t + 1
+          if (leader) umma_commit(&B.k_empty[(t + 1) % KST]);
+          __syncwarp();
         }
       }
     }
     // Every MMA this warp issued must finish before TMEM is released.
-    if (leader) umma_commit(B.drain);
+    if (leader) umma_commit(&B.drain[s]);
     __syncwarp();
-    warp_wait(B.drain, 0, lim, nullptr);
+    warp_wait(&B.drain[s], 0, lim, nullptr);
   } else if (warp / 4 < nslot) {
     // ------------------------------------------------------- softmax warps
     // Every tcgen05.ld/st/wait below is .sync.aligned: the whole warp must
@@ -564,21 +574,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int h = h0 + slot;
     const int64_t i = static_cast<int64_t>(qb) * BM + r;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const uint32_t s_addr = lane_addr + col_s(slot);
     const uint32_t o_addr = lane_addr + col_o(slot);
     const float c2 = a.scale_log2;  // logits to base-2 exponent units
     const uint64_t c2x2 = pack_f2(c2, c2);
     float m_run = -INFINITY, l_run = 0.f;  // running max (base-2 units) and sum
     int bnd_cnt = 0;
     bool ok = true;
-    for (int t = 0; t < nkb; ++t) {
-      const int kb = qb - t;
-      const uint32_t tm = ttab[t];
+    for (int u = 0; u < nsub; ++u) {
+      const int t = u >> 1, hh = u & 1;
+      const int64_t k0 = static_cast<int64_t>(qb - t) * BN + SUB * hh;  // first key of the sub-tile
+      const uint32_t s_addr = lane_addr + col_s(slot) + SUB * hh;
+      const uint32_t tm = ttab[u];
       const uint32_t bnd = tm >> 8;
       const bool any_group = (tm & 0xffffu) != 0;
       if (bnd) {
         // Mask S in place after each boundary class: keep column c iff
-        // (i - kb*BN) - c <= W, i.e. c >= cmin; otherwise 0.
+        // (i - k0) - c <= W, i.e. c >= cmin; otherwise 0.
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
@@ -586,18 +597,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = warp_wait(&B.bnd_ready[slot], bnd_cnt & 1, lim, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const int64_t cmin64 = i - static_cast<int64_t>(kb) * BN - W;
-          const int cmin = cmin64 < 0 ? 0 : (cmin64 > BN ? BN : static_cast<int>(cmin64));
+          const int64_t cmin64 = i - k0 - W;
+          const int cmin = cmin64 < 0 ? 0 : (cmin64 > SUB ? SUB : static_cast<int>(cmin64));
+          uint32_t su[64];
+          tmem_ld64(s_addr, su);
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t su[64];
-            tmem_ld64(s_addr + 64 * hf, su);
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (64 * hf + c < cmin) su[c] = 0u;
-            tmem_st32(s_addr + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
-            tmem_st32(s_addr + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
-          }
+          for (int c = 0; c < 64; ++c)
+            if (c < cmin) su[c] = 0u;
+          tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+          tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -607,68 +615,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (!ok) break;
       }
-      if (!warp_wait(&B.s_ready[slot], t & 1, lim, abort_flag)) {
+      if (!warp_wait(&B.s_ready[2 * slot + hh], t & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t su[64];
+      load_half(s_addr, any_group, su);
+      if (t == 0) causal_mask(su, SUB * hh, r);  // diagonal tile
+      const float m_half = half_max(su) * c2;    // scale > 0, so the max commutes with it
+      if (u == 0) {
+        m_run = m_half;  // key 0 of the diagonal tile is in every row's window
+      } else if (__any_sync(FULL, m_half > m_run + RESCALE_THRESHOLD)) {
+        // Some row's max grew by more than 2^8 (rare): rescale O (it holds the
+        // sum through sub-tile u - 1: wait for that PV) and the row sum.
+        const float m_new = fmaxf(m_run, m_half);
+        const float alpha = fast_exp2(m_run - m_new);
+        if (!warp_wait(&B.o_ready[slot], (u - 1) & 1, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        scale_cols_f32(o_addr, D / 32, alpha);
+        l_run *= alpha;
+        m_run = m_new;
+      }
       const uint64_t zero2 = 0ull;
       uint64_t acc[4] = {zero2, zero2, zero2, zero2};
-      if (t == 0) {
-        // Diagonal tile: causal mask, and the row max from both halves first
-        // (the running max starts here), then a second read for the exps.
-        float mx = -INFINITY;
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t su[64];
-          load_half(s_addr + 64 * hf, any_group, su);
-          causal_mask(su, 64 * hf, r);
-          mx = fmaxf(mx, half_max(su));
-        }
-        m_run = mx * c2;  // scale > 0, so the max commutes with it
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t su[64];
-          load_half(s_addr + 64 * hf, any_group, su);
-          causal_mask(su, 64 * hf, r);
-          exp_half(su, c2x2, m_run, acc, s_addr + 32 * hf);
-        }
-      } else {
-        // One read of S per half: exponentiate against the running max right
-        // away, unless some row's max grew by more than 2^8 (rare): then O, the
-        // row sum and the P already written for the first half are rescaled.
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t su[64];
-          load_half(s_addr + 64 * hf, any_group, su);
-          const float m_half = half_max(su) * c2;
-          if (__any_sync(FULL, m_half > m_run + RESCALE_THRESHOLD)) {
-            const float m_new = fmaxf(m_run, m_half);
-            const float alpha = fast_exp2(m_run - m_new);
-            // O holds the sum through key tile t-1: wait for that PV.
-            if (!warp_wait(&B.o_ready[slot], (t - 1) & 1, lim, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            scale_cols_f32(o_addr, D / 32, alpha);
-            if (hf == 1) scale_cols_bf16x2(s_addr, alpha);  // P of keys 0-63
-            float a0, a1;
-            unpack_f2(acc[0], a0, a1);
-            acc[0] = pack_f2(a0 * alpha, a1 * alpha);
-            unpack_f2(acc[1], a0, a1);
-            acc[1] = pack_f2(a0 * alpha, a1 * alpha);
-            unpack_f2(acc[2], a0, a1);
-            acc[2] = pack_f2(a0 * alpha, a1 * alpha);
-            unpack_f2(acc[3], a0, a1);
-            acc[3] = pack_f2(a0 * alpha, a1 * alpha);
-            l_run *= alpha;
-            m_run = m_new;
-          }
-          exp_half(su, c2x2, m_run, acc, s_addr + 32 * hf);
-        }
-        if (!ok) break;
-      }
+      exp_half(su, c2x2, m_run, acc, s_addr);  // P: the sub-tile's first 32 columns
       float s0, s1, s2, s3, s4, s5, s6, s7;
       unpack_f2(acc[0], s0, s1);
       unpack_f2(acc[1], s2, s3);
@@ -678,22 +652,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();  // the warp's TMEM stores are ordered before lane 0's arrival
-      if (lane == 0) mbar_arrive(&B.p_ready[slot]);
+      if (lane == 0) mbar_arrive(&B.p_ready[2 * slot + hh]);
     }
-    if (ok && nkb > 0 && warp_wait(&B.o_ready[slot], (nkb - 1) & 1, lim, abort_flag)) {
+    // o_ready may trail by two phases here (the last two PVs can both be in
+    // flight), so the end of the last PV has a barrier of its own.
+    if (ok && nsub > 0 && warp_wait(&B.o_final[slot], 0, lim, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
       __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t u[32];
-        tmem_ld32(o_addr + 32 * c4, u);
-        tmem_wait_ld(u);
+        uint32_t u32[32];
+        tmem_ld32(o_addr + 32 * c4, u32);
+        tmem_wait_ld(u32);
         uint4 pk4[4];
         uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          pw[k] = pack_bf16x2(__uint_as_float(u[2 * k]) * inv_l, __uint_as_float(u[2 * k + 1]) * inv_l);
+          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * inv_l, __uint_as_float(u32[2 * k + 1]) * inv_l);
         if (i < a.N) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c4);
 #pragma unroll
@@ -716,7 +692,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_dealloc(tmem, TMEM_COLS);
   }
 }
-
 }  // namespace
 
 template <int D>
