@@ -292,7 +292,7 @@ def cpu_baseline(path: Path, target_s: float):
         return flops, time.perf_counter() - t0
 
     f0, t0 = sample(32, 1)
-    nrows = int(min(8192, max(32, 32 * target_s / max(t0, 1e-3))))
+    nrows = int(min(65536, max(32, 32 * target_s / max(t0, 1e-3))))
     f1, t1 = sample(nrows, 2)
     return {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"{nrows} random query rows (all heads) of the 32K prefill, fp64, {t1:.1f} s"}

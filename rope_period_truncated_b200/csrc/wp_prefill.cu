@@ -8,38 +8,44 @@
 //
 // How. One CTA takes one 128-row query tile of two query heads that share a
 // KV head (GQA), so every K/V tile it loads feeds both, and visits the key
-// tiles from the diagonal backwards. §2.3's skip / full / boundary class of
-// every (key tile, group) is the same for both heads and comes from a per-CTA
-// table built once in shared memory.
-//   warp 8  TMA producer: Q of both heads once (one 16-dim box per group); per
-//           key tile only the K column slices of non-skipped groups (16-dim
-//           boxes, 32-byte swizzle) and all of V (64-dim boxes, 128-byte
-//           swizzle).
-//   warp 9  MMA issuer (one elected lane, warp-uniform loop). Per key tile and
-//           head: one tcgen05.mma (M=128, N=128, K=16) per non-skipped group
-//           into that head's S accumulator in TMEM, then P (bf16, written back
-//           into S's columns by the softmax warps) times V into its O
-//           accumulator. The two heads ping-pong: PV(head 0), QK(head 0, next
-//           tile), PV(head 1), QK(head 1, next tile), so one head's softmax
-//           runs while the tensor core works for the other.
+// tiles from the diagonal backwards. Each 128-key tile is handled as two
+// 64-key sub-tiles u = 2t + h; §2.3's skip / full / boundary class of
+// every (sub-tile, group) is the same for both heads and comes from a
+// per-CTA table built once in shared memory.
+//   warp 8   TMA producer: Q of both heads once (one 16-dim box per group);
+//            per key tile only the K column slices of groups either half
+//            computes (16-dim boxes, 32-byte swizzle) and all of V (64-dim
+//            boxes, 128-byte swizzle); two stages each.
+//   warp 9+s MMA issuer of head s (one elected lane, warp-uniform loop). S of
+//            a head is double-buffered: two 64-column halves of TMEM, half h
+//            holding sub-tiles u = h mod 2. Per sub-tile u: once P(u) is in
+//            TMEM, PV(u) (4 MMAs, K = 16 keys each, into O) and then QK(u+2)
+//            into the half P(u) frees (one M=128, N=64, K=16 MMA per
+//            non-skipped group). The tensor core runs one thread's MMAs in
+//            order, so QK(u+2) overwrites P(u) only after PV(u) has read it,
+//            and S(u+1) was issued one step earlier: the softmax of u+1 runs
+//            while the MMAs that follow u do.
 //   warps 0-3 / 4-7  softmax of head 0 / head 1, one thread per query row:
-//           causal mask on the diagonal tile, online softmax in base 2 with
-//           the scale folded into one FMA, P to TMEM, O rescaled only when a
-//           row max grows by more than 2^8; epilogue O/l -> bf16 and
-//           LSE = ln(sum exp).
-// Boundary groups: the groups whose cutoff falls inside the tile's distance
-// range go first, one distinct cutoff at a time in ascending order; after each
-// class the softmax warps mask S in place (keep iff i - j <= W, else 0), and
-// the full groups then accumulate on top unmasked. Masks of ascending cutoffs
-// are nested, so m2*(m1*S1 + S2) = m1*S1 + m2*S2: the exact per-class mask.
-// TMEM columns: head s uses [256s, 256s+128) for S / P and [256s+128, 256s+256)
-// for O. If H_q/H_kv is odd the CTA takes a single head.
+//            causal mask on the diagonal tile, online softmax in base 2 with
+//            the scale folded into one FMA, P (bf16) over the first 32
+//            columns of its S half, O rescaled only when a row max grows by
+//            more than 2^8; epilogue O/l -> bf16 and LSE = ln(sum exp).
+// Boundary groups: the groups whose cutoff falls inside the sub-tile's
+// distance range go first, one distinct cutoff at a time in ascending order;
+// after each class the softmax warps mask S in place (keep iff i - j <= W,
+// else 0), and the full groups then accumulate on top unmasked. Masks of
+// ascending cutoffs are nested, so m2*(m1*S1 + S2) = m1*S1 + m2*S2: the
+// exact per-class mask.
+// TMEM columns: head s uses [256s, 256s+64) and [256s+64, 256s+128) for the
+// two S / P halves and [256s+128, 256s+256) for O. If H_q/H_kv is odd the CTA
+// takes a single head.
 //
-// The softmax's exponentials (16384 per head and tile) compete with the MUFU
-// unit's 16 per SM per clock, so POLY_PAIRS of every 8 pairs take 2^x on the
-// FMA pipe instead, in packed f32x2 arithmetic: Cody-Waite reduction x = j + f, |f| <= 1/2, and a degree-3 minimax
-// polynomial for 2^f (coefficients from a Remez fit, max relative error
-// 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in the exponent field.
+// The softmax's exponentials compete with the MUFU unit's 16 per SM per
+// clock, so POLY_PAIRS of every 8 pairs take 2^x on the FMA pipe instead, in
+// packed f32x2 arithmetic: Cody-Waite reduction x = j + f, |f| <= 1/2, and a
+// degree-3 minimax polynomial for 2^f (coefficients from a Remez fit, max
+// relative error 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in the
+// exponent field.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -68,7 +74,7 @@ constexpr uint32_t FULL = 0xffffffffu;
 // Row-max growth (base-2 units) below which O is not rescaled.
 constexpr float RESCALE_THRESHOLD = 8.0f;
 #ifndef WP_POLY_PAIRS
-#define WP_POLY_PAIRS 1
+#define WP_POLY_PAIRS 2
 #endif
 constexpr int POLY_PAIRS = WP_POLY_PAIRS;  // of every 8 exponent pairs, on the FMA pipe
 static_assert(POLY_PAIRS >= 0 && POLY_PAIRS <= 8, "POLY_PAIRS counts pairs out of 8");
