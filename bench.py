@@ -93,6 +93,26 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def profiled_traffic(summary: str, source: str):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or
+    None when the kernel source has changed since it was captured."""
+    import hashlib
+    try:
+        kv = {}
+        with open(os.path.join(ROOT, "profiles", summary)) as f:
+            for line in f:
+                if ":" in line and not line.startswith("#"):
+                    key, val = line.split(":", 1)
+                    kv[key.strip()] = val.strip()
+        with open(os.path.join(ROOT, source), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+        if kv.get("source_sha256_16") != digest:
+            return None
+        return int(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def prefill_flops(N, d, Hq, B, wg):
     """(tile-level, pair-exact) useful FLOPs of one causal prefill.
 
@@ -457,7 +477,10 @@ def run_ours(args, rank, world, local):
             "frac": round(achieved / peak_t, 4),
             "peak_kind": f"{peak_kind} bf16 dense burst",
             "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
-            "traffic": None,
+            "traffic": (profiled_traffic("prefill_grouped_kernel_32k_dram.txt",
+                                         "rope_period_truncated_b200/csrc/wp_prefill.cu")
+                        if args.prefill_n in (0, 32768) else None),
+            "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "kernel_ms": round(prefill_ms, 4),
             "flops_per_launch": tile_flops,
             "pair_exact_flops_per_launch": pair_flops,
