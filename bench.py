@@ -56,6 +56,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--kcache", choices=["group-major", "rows"], default="group-major",
+                   help="layout of the decode K cache in HBM")
     p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                    help="restrict the step (profiling a single kernel)")
     p.add_argument("--prefill-n", type=int, default=0,
@@ -213,7 +215,7 @@ class ClockSampler:
 class Path:
     """Device buffers and launches of one hot-path step."""
 
-    def __init__(self, device, prefill_n=0):
+    def __init__(self, device, prefill_n=0, kcache_layout="group-major"):
         import dataclasses
         import rope_period_truncated_b200 as wp
         self.wp = wp
@@ -233,7 +235,12 @@ class Path:
         self.host_decode = (dq, lens)
         self.dq = dq.to(device).reshape(dw.B, 1, dw.Hq, dw.d)
         self.dqr = torch.empty_like(self.dq)
-        self.kc, self.vc = kc.to(device), vc.to(device)
+        # the K cache is stored group-major ([B, Hkv, d/16, L, 16]) unless asked
+        # for rows: the keys a group skips are then contiguous and never read
+        self.kc = kc.to(device)
+        if kcache_layout == "group-major":
+            self.kc = wp.wp_kcache_group_major(self.kc)
+        self.vc = vc.to(device)
         self.lens_host = lens
         self.lens = lens.to(device)
         self.pos = (lens - 1).to(torch.int32).reshape(dw.B, 1).to(device)
@@ -324,7 +331,7 @@ def run_ours(args, rank, world, local):
     wpbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    path = Path(dev, args.prefill_n)
+    path = Path(dev, args.prefill_n, args.kcache)
     peaks, peak_kind = load_peaks()
     do_prefill = args.only in ("all", "prefill")
     do_decode = args.only in ("all", "decode")
@@ -467,6 +474,8 @@ def run_ours(args, rank, world, local):
             "l2": "inputs larger than L2 each step (384 MiB prefill Q/K/V, 2 GiB KV cache); no flush",
             "parallelism": f"replicas x{world} (independent heads/sequences, no collective)",
             "group_cutoffs": [int(x) for x in path.wg],
+            "decode_kcache": ("group-major [B,Hkv,d/16,L,16]" if args.kcache == "group-major"
+                              else "rows [B,Hkv,L,d]"),
         },
         "roofline": {
             "kernel": "wp_prefill (grouped, tcgen05)",

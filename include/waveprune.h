@@ -165,6 +165,44 @@ int wp_decode(const void *q, const void *kcache, const void *vcache, const int32
               void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * K cache layouts of wp_decode_kl.
+ *   WP_KCACHE_ROWS          [B, H_kv, Lmax, d_h]: one row of d_h per key (the
+ *                           layout of wp_decode).
+ *   WP_KCACHE_GROUP_MAJOR   [B, H_kv, d_h/16, Lmax, 16]: the 16 dims of group g
+ *                           of all keys are contiguous 32-byte records. [RN
+ *                           §2.3, table row 1] says a skipped group's K bytes
+ *                           are not read in decode; in this layout the keys a
+ *                           group skips are one contiguous range, which DRAM
+ *                           then never moves (in rows they are 32-byte holes
+ *                           inside 256-byte rows that travel with their line).
+ *                           The pages fix no layout; this one is a choice of
+ *                           this library.
+ */
+enum wp_kcache_layout { WP_KCACHE_ROWS = 0, WP_KCACHE_GROUP_MAJOR = 1 };
+
+/*
+ * wp_kcache_group_major — copy a K cache from WP_KCACHE_ROWS to
+ * WP_KCACHE_GROUP_MAJOR.
+ *   k_rows  device bf16 [B, H_kv, Lmax, d_h], 16-byte aligned (read only).
+ *   k_gm    device bf16 out [B, H_kv, d_h/16, Lmax, 16], 16-byte aligned, the
+ *           same size, caller-owned, not overlapping k_rows.
+ *   d_h in {64, 128}. Asynchronous on `stream`.
+ * Errors: WP_ERR_ARG (null, misaligned, same buffer, bad sizes),
+ * WP_ERR_UNSUPPORTED (d_h), WP_ERR_CUDA.
+ */
+int wp_kcache_group_major(const void *k_rows, void *k_gm, int B, int H_kv, int Lmax, int d_h, void *stream);
+
+/*
+ * wp_decode_kl — wp_decode with the K cache in layout `k_layout`
+ * (wp_kcache_layout); V stays [B, H_kv, Lmax, d_h]. All other arguments,
+ * results and errors are those of wp_decode; a k_layout outside the enum is
+ * WP_ERR_ARG. Both layouts give bit-identical results.
+ */
+int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
+                 int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+                 void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * wp_decode_static — wp_decode without a workspace argument, for callers that
  * cannot allocate device memory (for example a serving engine whose device
  * memory is planned up front and handed out by its own pool, or a decode loop

@@ -24,7 +24,7 @@ __all__ = [
     "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
     "WavePruneError", "library_path", "load_library",
     "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
-    "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES",
+    "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES", "wp_kcache_group_major", "KCACHE_ROWS", "KCACHE_GROUP_MAJOR",
     "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
 ]
 
@@ -36,6 +36,7 @@ CUTOFF_INF = 2 ** 31 - 1
 DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 WP_OK, WP_ERR_ARG, WP_ERR_UNSUPPORTED, WP_ERR_CUDA, WP_ERR_TIMEOUT = range(5)
+KCACHE_ROWS, KCACHE_GROUP_MAJOR = 0, 1  # wp_kcache_layout
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libwaveprune.so")
@@ -76,6 +77,10 @@ def load_library():
     lib.wp_decode.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
     lib.wp_decode_static.restype = I
     lib.wp_decode_static.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P]
+    lib.wp_decode_kl.restype = I
+    lib.wp_decode_kl.argtypes = [P, P, I, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
+    lib.wp_kcache_group_major.restype = I
+    lib.wp_kcache_group_major.argtypes = [P, P, I, I, I, I, P]
     lib.wp_device_status.restype = I
     lib.wp_device_status.argtypes = [P]
     lib.wp_set_wait_limit.restype = ctypes.c_longlong
@@ -216,19 +221,44 @@ def wp_decode_workspace_bytes(B: int, Hq: int, d_h: int, Lmax: int) -> int:
     return int(load_library().wp_decode_workspace_bytes(B, Hq, d_h, Lmax))
 
 
+def wp_kcache_group_major(kcache: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """K cache [B,Hkv,Lmax,d] bf16 (rows) -> [B,Hkv,d/16,Lmax,16] (group-major)."""
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    B, Hkv, Lmax, d = kcache.shape
+    if out is None:
+        out = torch.empty((B, Hkv, d // 16, Lmax, 16), dtype=torch.bfloat16, device=kcache.device)
+    _need(out, "out", torch.bfloat16, 5)
+    if tuple(out.shape) != (B, Hkv, d // 16, Lmax, 16):
+        raise ValueError("out shape mismatch")
+    _check("wp_kcache_group_major", load_library().wp_kcache_group_major(
+        _ptr(kcache), _ptr(out), B, Hkv, Lmax, d, _stream(stream)))
+    return out
+
+
 def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens: torch.Tensor, group_cut=None,
               softmax_scale: float = 0.0, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, want_lse: bool = True, stream=None):
-    """Split-KV decode. q [B,Hq,d] (rotated), caches [B,Hkv,Lmax,d] bf16, lens
-    int32 [B] (device). Returns (o [B,Hq,d] bf16, lse [B,Hq] fp32)."""
+    """Split-KV decode. q [B,Hq,d] (rotated), V cache [B,Hkv,Lmax,d] bf16, K
+    cache the same (rows) or [B,Hkv,d/16,Lmax,16] (group-major, from
+    wp_kcache_group_major), lens int32 [B] (device). Returns (o [B,Hq,d] bf16,
+    lse [B,Hq] fp32)."""
     _need(q, "q", torch.bfloat16, 3)
-    _need(kcache, "kcache", torch.bfloat16, 4)
     _need(vcache, "vcache", torch.bfloat16, 4)
     _need(lens, "lens", torch.int32, 1)
     B, Hq, d = q.shape
-    _, Hkv, Lmax, _ = kcache.shape
-    if tuple(kcache.shape) != (B, Hkv, Lmax, d) or tuple(vcache.shape) != tuple(kcache.shape):
+    _, Hkv, Lmax, _ = vcache.shape
+    if tuple(vcache.shape) != (B, Hkv, Lmax, d):
         raise ValueError("cache shape mismatch")
+    if kcache.dim() == 5:
+        _need(kcache, "kcache", torch.bfloat16, 5)
+        if tuple(kcache.shape) != (B, Hkv, d // 16, Lmax, 16):
+            raise ValueError("group-major K cache shape mismatch")
+        k_layout = KCACHE_GROUP_MAJOR
+    else:
+        _need(kcache, "kcache", torch.bfloat16, 4)
+        if tuple(kcache.shape) != tuple(vcache.shape):
+            raise ValueError("cache shape mismatch")
+        k_layout = KCACHE_ROWS
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
@@ -239,8 +269,8 @@ def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens:
     if workspace.numel() * workspace.element_size() < ws_bytes:
         raise ValueError("workspace too small")
     cut_a, cut_p = _host_i32(group_cut, d // 16)
-    _check("wp_decode", load_library().wp_decode(
-        _ptr(q), _ptr(kcache), _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
+    _check("wp_decode", load_library().wp_decode_kl(
+        _ptr(q), _ptr(kcache), k_layout, _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 

@@ -235,12 +235,13 @@ size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {
   return decode_workspace_bytes(B, H_q, nsplit, d_h);
 }
 
-int wp_decode(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B, int H_q,
-              int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
-              void *workspace, size_t ws_bytes, void *stream) {
+int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
+                 int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+                 void *workspace, size_t ws_bytes, void *stream) {
   if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr ||
       workspace == nullptr)
     return WP_ERR_ARG;
+  if (k_layout != WP_KCACHE_ROWS && k_layout != WP_KCACHE_GROUP_MAJOR) return WP_ERR_ARG;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || (reinterpret_cast<uintptr_t>(lens) & 3u) != 0 ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
@@ -270,12 +271,30 @@ int wp_decode(const void *q, const void *kcache, const void *vcache, const int32
   a.Lmax = Lmax;
   a.nsplit = nsplit;
   a.chunk = DECODE_CHUNK;
+  a.k_group_major = k_layout == WP_KCACHE_GROUP_MAJOR ? 1 : 0;
   for (int g = 0; g < 8; ++g) {
     a.cut[g] = (group_cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : group_cut[g];
     if (a.cut[g] < 0) return WP_ERR_ARG;
   }
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
   return from_cuda(launch_decode(a, d_h, static_cast<cudaStream_t>(stream)));
+}
+
+int wp_decode(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B, int H_q,
+              int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+              void *workspace, size_t ws_bytes, void *stream) {
+  return wp_decode_kl(q, kcache, WP_KCACHE_ROWS, vcache, lens, Lmax, B, H_q, H_kv, d_h, group_cut, softmax_scale, o,
+                      lse, workspace, ws_bytes, stream);
+}
+
+int wp_kcache_group_major(const void *k_rows, void *k_gm, int B, int H_kv, int Lmax, int d_h, void *stream) {
+  if (k_rows == nullptr || k_gm == nullptr || !aligned16(k_rows) || !aligned16(k_gm)) return WP_ERR_ARG;
+  if (B <= 0 || H_kv <= 0 || Lmax <= 0) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  if (k_rows == k_gm) return WP_ERR_ARG;  // not in place
+  return from_cuda(launch_kcache_group_major(static_cast<const __nv_bfloat16 *>(k_rows),
+                                             static_cast<__nv_bfloat16 *>(k_gm), static_cast<int64_t>(B) * H_kv,
+                                             Lmax, d_h, static_cast<cudaStream_t>(stream)));
 }
 
 int wp_device_status(void *stream) {

@@ -15,7 +15,11 @@
 // copied with source size 0 (no bytes read, slot zero-filled), so the group
 // adds exactly 0 to the logit. In the row layout [Lmax, d] the skipped K
 // bytes only leave HBM untouched where a whole 128-byte line is out of
-// window; finer holes are fetched with their line. The GQA query heads of the
+// window; finer holes are fetched with their line. In the group-major K layout
+// [D/16, Lmax, 16] a group's keys are contiguous 32-byte records, so the keys
+// a group skips form one contiguous range that is not read at all; there a
+// warp loads one group of a 16-key block (512 contiguous bytes) per
+// instruction. The GQA query heads of the
 // KV head (H_q/H_kv <= 8) form the rows of warp-level bf16 mma.sync products
 // (scores Q.K^T and P.V, fp32 accumulation); the online softmax keeps the row
 // max and row sum with warp shuffles. The 4 warps merge their states in
@@ -86,7 +90,7 @@ __device__ __forceinline__ uint32_t piece_off(int r, int p) {
   return static_cast<uint32_t>(r) * DecLayout<D>::ROWB + static_cast<uint32_t>((p ^ (r & 7)) * 16);
 }
 
-template <int D, int R>
+template <int D, int R, bool KGM>
 __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeArgs a) {
   using L = DecLayout<D>;
   constexpr int PIECES = L::PIECES;
@@ -125,7 +129,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
     }
   }
 
-  const __nv_bfloat16 *kbase = a.kc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;
+  const __nv_bfloat16 *kbase = a.kc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;  // either layout
   const __nv_bfloat16 *vbase = a.vc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;
   const uint32_t ring = smem_u32(dsmem) + warp * L::WARP_BYTES;
 
@@ -138,14 +142,29 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
       const int r = idx / PIECES, p = idx % PIECES;
       const int key = kb0 + r;
       const bool valid = key < end;
-      const int64_t dist = qpos - key;
-      const bool kin = valid && dist <= static_cast<int64_t>(a.cut[p >> 1]);
-      // An out-of-window K piece is copied with source size 0: nothing is
-      // read and its shared-memory slot is zero-filled, so the group adds
-      // exactly 0 to the score.
       const int64_t row = valid ? key : kb0;  // any in-range address when nothing is read
-      cp_async16(kdst + piece_off<D>(r, p), kbase + row * D + 8 * p, kin ? 16u : 0u);
+      if (!KGM) {
+        const int64_t dist = qpos - key;
+        const bool kin = valid && dist <= static_cast<int64_t>(a.cut[p >> 1]);
+        // An out-of-window K piece is copied with source size 0: nothing is
+        // read and its shared-memory slot is zero-filled, so the group adds
+        // exactly 0 to the score.
+        cp_async16(kdst + piece_off<D>(r, p), kbase + row * D + 8 * p, kin ? 16u : 0u);
+      }
       cp_async16(vdst + piece_off<D>(r, p), vbase + row * D + 8 * p, valid ? 16u : 0u);
+    }
+    if (KGM) {
+      // group-major K: iteration it takes group it, lane = 2 * key + half
+#pragma unroll
+      for (int gi = 0; gi < D / 16; ++gi) {
+        const int r = lane >> 1, half = lane & 1;
+        const int key = kb0 + r;
+        const bool valid = key < end;
+        const int64_t row = valid ? key : kb0;
+        const bool kin = valid && qpos - key <= static_cast<int64_t>(a.cut[gi]);
+        cp_async16(kdst + piece_off<D>(r, 2 * gi + half), kbase + (static_cast<int64_t>(gi) * a.Lmax + row) * 16 + 8 * half,
+                   kin ? 16u : 0u);
+      }
     }
   };
 
@@ -285,15 +304,38 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   if (d == 0 && a.lse != nullptr) a.lse[bh] = (M + log2f(Lsum)) * 0.69314718055994531f;
 }
 
-template <int D, int R>
-cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+template <int D, int R, bool KGM>
+cudaError_t launch_split_l(const DecodeArgs &a, cudaStream_t stream) {
   const uint32_t smem = DecLayout<D>::BYTES;
   cudaError_t e =
-      cudaFuncSetAttribute(decode_split_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(decode_split_kernel<D, R, KGM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nsplit, a.Hkv, a.B);
-  decode_split_kernel<D, R><<<grid, DEC_THREADS, smem, stream>>>(a);
+  decode_split_kernel<D, R, KGM><<<grid, DEC_THREADS, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int R>
+cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+  return a.k_group_major ? launch_split_l<D, R, true>(a, stream) : launch_split_l<D, R, false>(a, stream);
+}
+
+// One thread per 16-byte piece of the group-major output, in output order:
+// consecutive threads write consecutive bytes.
+template <int D>
+__global__ void kcache_group_major_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int64_t BH,
+                                          int Lmax) {
+  constexpr int G = D / 16;
+  const int64_t n = BH * G * Lmax * 2;
+  for (int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; o < n;
+       o += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int half = static_cast<int>(o & 1);
+    const int64_t key = (o >> 1) % Lmax;
+    const int64_t bg = (o >> 1) / Lmax;  // bh * G + g
+    const int g = static_cast<int>(bg % G);
+    const int64_t bh = bg / G;
+    dst[o] = src[(bh * Lmax + key) * (D / 8) + 2 * g + half];
+  }
 }
 
 template <int D>
@@ -307,6 +349,19 @@ cudaError_t launch_split_r(const DecodeArgs &a, int R, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int64_t BH, int Lmax, int D,
+                                      cudaStream_t stream) {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const uint4 *s = reinterpret_cast<const uint4 *>(src);
+  uint4 *d = reinterpret_cast<uint4 *>(dst);
+  if (D == 128)
+    kcache_group_major_kernel<128><<<nsm * 8, 256, 0, stream>>>(s, d, BH, Lmax);
+  else
+    kcache_group_major_kernel<64><<<nsm * 8, 256, 0, stream>>>(s, d, BH, Lmax);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream) {
   const int R = a.Hq / a.Hkv;

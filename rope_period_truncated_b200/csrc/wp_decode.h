@@ -13,13 +13,14 @@ constexpr int DECODE_CHUNK = 1024;
 
 struct DecodeArgs {
   const __nv_bfloat16 *q;            // [B, Hq, D]
-  const __nv_bfloat16 *kc, *vc;      // [B, Hkv, Lmax, D]
+  const __nv_bfloat16 *kc, *vc;      // V [B, Hkv, Lmax, D]; K the same or group-major [B, Hkv, D/16, Lmax, 16]
   const int32_t *lens;               // [B]
   __nv_bfloat16 *o;                  // [B, Hq, D]
   float *lse;                        // [B, Hq] or null
   float *o_part;                     // [B, Hq, nsplit, D]
   float *lse_part;                   // [B, Hq, nsplit], base-2
   int B, Hq, Hkv, Lmax, nsplit, chunk;
+  int k_group_major;                 // K cache layout: 0 rows, 1 group-major
   int32_t cut[8];                    // group cutoffs
   float scale_log2;
 };
@@ -34,5 +35,9 @@ inline size_t decode_workspace_bytes(int B, int Hq, int nsplit, int D) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream);
+
+// K cache rows [BH, Lmax, D] -> group-major [BH, D/16, Lmax, 16] (BH = B * H_kv).
+cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int64_t BH, int Lmax, int D,
+                                      cudaStream_t stream);
 
 }  // namespace wp

@@ -150,6 +150,30 @@ def test_decode_rejects_bad_arguments(lib):
     assert call(4, 0) == wp.WP_ERR_ARG                  # Lmax
 
 
+def test_decode_kl_and_kcache_conversion_reject_bad_arguments(lib):
+    f = lib.wp_decode_kl
+    ws = lib.wp_decode_workspace_bytes(2, 8, 128, 4096)
+    args = [FAKE, FAKE, wp.KCACHE_GROUP_MAJOR, FAKE, FAKE, 4096, 2, 8, 2, 128, None, ctypes.c_float(0.0), FAKE,
+            None, FAKE, ws, None]
+
+    def call(i, val):
+        a = list(args)
+        a[i] = val
+        return f(*a)
+
+    assert call(2, 2) == wp.WP_ERR_ARG                  # layout outside the enum
+    assert call(2, -1) == wp.WP_ERR_ARG
+    assert call(1, None) == wp.WP_ERR_ARG               # K cache NULL
+    assert call(15, ws - 1) == wp.WP_ERR_ARG            # workspace too small
+    assert call(9, 80) == wp.WP_ERR_UNSUPPORTED         # d_h
+    g = lib.wp_kcache_group_major
+    assert g(None, FAKE, 1, 2, 100, 128, None) == wp.WP_ERR_ARG
+    assert g(FAKE, FAKE, 1, 2, 100, 128, None) == wp.WP_ERR_ARG      # in place
+    assert g(FAKE, FAKE + 8, 1, 2, 100, 128, None) == wp.WP_ERR_ARG  # misaligned
+    assert g(FAKE, FAKE + 4096, 0, 2, 100, 128, None) == wp.WP_ERR_ARG
+    assert g(FAKE, FAKE + 4096, 1, 2, 100, 80, None) == wp.WP_ERR_UNSUPPORTED
+
+
 def test_rope_rejects_bad_arguments(lib):
     f = lib.wp_rope_apply
     assert f(None, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG

@@ -94,3 +94,54 @@ def test_decode_bad_length_gives_nan_rows():
     torch.cuda.synchronize()
     assert torch.isnan(o[0].float()).all() and torch.isnan(lse[0]).all()
     assert torch.allclose(o[1].float(), torch.ones_like(o[1].float()))
+
+
+def test_kcache_group_major_layout():
+    """wp_kcache_group_major is the permutation [B,Hkv,L,G,16] -> [B,Hkv,G,L,16]."""
+    g = torch.Generator().manual_seed(11)
+    for d in (64, 128):
+        kc = torch.randn(3, 2, 1000, d, generator=g).to(torch.bfloat16).cuda()
+        gm = wp.wp_kcache_group_major(kc)
+        torch.cuda.synchronize()
+        want = kc.reshape(3, 2, 1000, d // 16, 16).permute(0, 1, 3, 2, 4).contiguous()
+        assert torch.equal(gm, want)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_group_major_kcache(d):
+    """The group-major K cache gives results bit-identical to the row layout,
+    and both match the oracle (ragged lengths, boundary cutoffs)."""
+    g = torch.Generator().manual_seed(31 + d)
+    B, Hq, Hkv, Lmax = 4, 8, 2, 3000
+    lens = torch.tensor([1, 2999, 1500, 1025], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    _, wg = oracle.cutoffs(d, 1e4, oracle.HALF_SPLIT)
+    wg = np.minimum(wg, [5, 40, 300, 1100, 2000, 10 ** 6, 7, 1024][: d // 16]).astype(np.int32)
+    o_rows, lse_rows = _gpu_decode(q, kc, vc, lens, wg)
+    kgm = wp.wp_kcache_group_major(kc.cuda())
+    o_gm, lse_gm = wp.wp_decode(q.cuda(), kgm, vc.cuda(), lens.cuda(), wg)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    assert torch.equal(o_gm, o_rows) and torch.equal(lse_gm, lse_rows)
+    ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o_gm, lse_gm, ro, rl, f"decode group-major d={d}")
+
+
+def test_decode_group_major_workload():
+    """The 32K decode workload with a group-major K cache: every row checked
+    against the oracle."""
+    w = syn.workload("decode_32k")
+    q, kc, vc, lens = syn.decode_inputs(w)
+    _, wg = oracle.cutoffs(w.d, w.theta, w.layout)
+    pos = (lens - 1).to(torch.int32).reshape(w.B, 1)
+    qr = wp.wp_rope_apply(q.cuda().reshape(w.B, 1, w.Hq, w.d), w.theta, w.layout, pos=pos.cuda())
+    kgm = wp.wp_kcache_group_major(kc.cuda())
+    o, lse = wp.wp_decode(qr.reshape(w.B, w.Hq, w.d), kgm, vc.cuda(), lens.cuda(), wg)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    qo = oracle.rope(widen(q).reshape(w.B, 1, w.Hq, w.d), w.theta, w.layout, pos=pos.numpy())
+    qo = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qo)).reshape(w.B, w.Hq, w.d)
+    ro, rl = oracle.decode(qo, widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o, lse, ro, rl, "decode_32k group-major")
