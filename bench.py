@@ -318,9 +318,12 @@ def cpu_baseline(path: Path, target_s: float):
                               oracle.MODE_GROUPED, pw.layout, nthreads=threads)
         return flops, time.perf_counter() - t0
 
-    f0, t0 = sample(32, 1)
-    nrows = int(min(65536, max(32, 32 * target_s / max(t0, 1e-3))))
+    f0, t0 = sample(256, 1)
+    nrows = int(min(65536, max(32, 256 * target_s / max(t0, 1e-3))))
     f1, t1 = sample(nrows, 2)
+    if t1 < 0.5 * target_s and nrows < 65536:  # the small sample overestimated the per-row time
+        nrows = int(min(65536, nrows * target_s / max(t1, 1e-3)))
+        f1, t1 = sample(nrows, 3)
     return {"value": f1 / t1 / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"{nrows} random query rows (all heads) of the 32K prefill, fp64, {t1:.1f} s"}
 
@@ -397,10 +400,16 @@ def run_ours(args, rank, world, local):
     # dense comparison: the same kernels with every cutoff infinite
     dense = None
     if not args.no_dense and args.only == "all":
-        dpf = time_kernel(lambda: path.prefill_only("dense"), 5, 2)
-        ddc = time_kernel(lambda: path.decode_only("dense"), 20, 5)
-        wpf = time_kernel(lambda: path.prefill_only("wave"), 5, 2)
-        wdc = time_kernel(lambda: path.decode_only("wave"), 20, 5)
+        # dense and wave alternate (A B B A ...) so that the clock drift of the
+        # power cap falls on both alike
+        dps, wps, dds, wds = [], [], [], []
+        for r in range(4):
+            order = [("dense", dps, dds), ("wave", wps, wds)]
+            for cut, pl, dl in (order if r % 2 == 0 else order[::-1]):
+                pl.append(time_kernel(lambda: path.prefill_only(cut), 3, 1))
+                dl.append(time_kernel(lambda: path.decode_only(cut), 10, 3))
+        dpf, wpf = statistics.median(dps), statistics.median(wps)
+        ddc, wdc = statistics.median(dds), statistics.median(wds)
         dense = {"prefill_ms": round(dpf, 4), "decode_ms": round(ddc, 5),
                  "prefill_speedup": round(dpf / wpf, 4), "decode_speedup": round(ddc / wdc, 4),
                  "prefill_dense_tflops": round(dense_tile_flops / (dpf * 1e-3) / 1e12, 2),
