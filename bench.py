@@ -58,6 +58,9 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--kcache", choices=["group-major", "rows"], default="group-major",
                    help="layout of the decode K cache in HBM")
+    p.add_argument("--grouping", choices=["half-split", "paired"], default="half-split",
+                   help="paired: Q/K of the half-split model rotated into the interleaved order, groups of 8 "
+                        "whole channels (the pages' grouping, Table 12 cutoffs)")
     p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                    help="restrict the step (profiling a single kernel)")
     p.add_argument("--prefill-n", type=int, default=0,
@@ -215,7 +218,7 @@ class ClockSampler:
 class Path:
     """Device buffers and launches of one hot-path step."""
 
-    def __init__(self, device, prefill_n=0, kcache_layout="group-major"):
+    def __init__(self, device, prefill_n=0, kcache_layout="group-major", grouping="half-split"):
         import dataclasses
         import rope_period_truncated_b200 as wp
         self.wp = wp
@@ -230,7 +233,12 @@ class Path:
         self.qr, self.kr = torch.empty_like(self.q), torch.empty_like(self.k)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((pw.B, pw.Hq, pw.N), dtype=torch.float32, device=device)
-        _, self.wg = wp.wp_cutoffs(pw.d, pw.theta, pw.layout, scale_all=pw.scale_all)
+        # "paired": Q/K rotated half-split but written in the interleaved order, so
+        # the groups hold whole channels and take the interleaved cutoffs
+        paired = grouping == "paired" and pw.layout == wp.ROPE_HALF_SPLIT
+        self.rope_layout = wp.ROPE_HALF_SPLIT_PAIRED if paired else pw.layout
+        self.cut_layout = wp.ROPE_INTERLEAVED if paired else pw.layout
+        _, self.wg = wp.wp_cutoffs(pw.d, pw.theta, self.cut_layout, scale_all=pw.scale_all)
         dq, kc, vc, lens = syn.decode_inputs(dw)
         self.host_decode = (dq, lens)
         self.dq = dq.to(device).reshape(dw.B, 1, dw.Hq, dw.d)
@@ -248,22 +256,23 @@ class Path:
         self.dlse = torch.empty((dw.B, dw.Hq), dtype=torch.float32, device=device)
         self.ws = torch.empty(wp.wp_decode_workspace_bytes(dw.B, dw.Hq, dw.d, dw.Lmax), dtype=torch.uint8,
                               device=device)
-        _, self.dwg = wp.wp_cutoffs(dw.d, dw.theta, dw.layout)
+        self.d_rope_layout = wp.ROPE_HALF_SPLIT_PAIRED if paired and dw.layout == wp.ROPE_HALF_SPLIT else dw.layout
+        _, self.dwg = wp.wp_cutoffs(dw.d, dw.theta, wp.ROPE_INTERLEAVED if paired else dw.layout)
         self.launches_per_step = 6  # rope Q, rope K, prefill, rope q(decode), decode split, combine
 
     def prefill(self, cut="wave"):
         wp, pw = self.wp, self.pw
-        wp.wp_rope_apply(self.q, pw.theta, pw.layout, scale_all=pw.scale_all, out=self.qr)
-        wp.wp_rope_apply(self.k, pw.theta, pw.layout, scale_all=pw.scale_all, out=self.kr)
+        wp.wp_rope_apply(self.q, pw.theta, self.rope_layout, scale_all=pw.scale_all, out=self.qr)
+        wp.wp_rope_apply(self.k, pw.theta, self.rope_layout, scale_all=pw.scale_all, out=self.kr)
         return self.prefill_only(cut)
 
     def prefill_only(self, cut="wave"):
         return self.wp.wp_prefill(self.qr, self.kr, self.v, self.wg if cut == "wave" else None,
-                                  self.wp.MODE_GROUPED, self.pw.layout, out=self.o, lse=self.lse)
+                                  self.wp.MODE_GROUPED, self.cut_layout, out=self.o, lse=self.lse)
 
     def decode(self, cut="wave"):
         wp, dw = self.wp, self.dw
-        wp.wp_rope_apply(self.dq, dw.theta, dw.layout, pos=self.pos, out=self.dqr)
+        wp.wp_rope_apply(self.dq, dw.theta, self.d_rope_layout, pos=self.pos, out=self.dqr)
         return self.decode_only(cut)
 
     def decode_only(self, cut="wave"):
@@ -334,7 +343,7 @@ def run_ours(args, rank, world, local):
     wpbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    path = Path(dev, args.prefill_n, args.kcache)
+    path = Path(dev, args.prefill_n, args.kcache, args.grouping)
     peaks, peak_kind = load_peaks()
     do_prefill = args.only in ("all", "prefill")
     do_decode = args.only in ("all", "decode")
@@ -348,8 +357,8 @@ def run_ours(args, rank, world, local):
         elif evp is None:
             path.prefill()
         else:
-            wp.wp_rope_apply(path.q, pw.theta, pw.layout, scale_all=pw.scale_all, out=path.qr)
-            wp.wp_rope_apply(path.k, pw.theta, pw.layout, scale_all=pw.scale_all, out=path.kr)
+            wp.wp_rope_apply(path.q, pw.theta, path.rope_layout, scale_all=pw.scale_all, out=path.qr)
+            wp.wp_rope_apply(path.k, pw.theta, path.rope_layout, scale_all=pw.scale_all, out=path.kr)
             evp[0].record()
             path.prefill_only()
             evp[1].record()
@@ -358,7 +367,7 @@ def run_ours(args, rank, world, local):
         elif evd is None:
             path.decode()
         else:
-            wp.wp_rope_apply(path.dq, dw.theta, dw.layout, pos=path.pos, out=path.dqr)
+            wp.wp_rope_apply(path.dq, dw.theta, path.d_rope_layout, pos=path.pos, out=path.dqr)
             evd[0].record()
             path.decode_only()
             evd[1].record()
@@ -489,6 +498,8 @@ def run_ours(args, rank, world, local):
             "group_cutoffs": [int(x) for x in path.wg],
             "decode_kcache": ("group-major [B,Hkv,d/16,L,16]" if args.kcache == "group-major"
                               else "rows [B,Hkv,L,d]"),
+            "grouping": ("half-split groups (max over channels c and c+64)" if args.grouping == "half-split"
+                         else "paired: 8 whole channels per group (interleaved order after rope)"),
         },
         "roofline": {
             "kernel": "wp_prefill (grouped, tcgen05)",
@@ -503,7 +514,7 @@ def run_ours(args, rank, world, local):
             "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
             "traffic": (profiled_traffic("prefill_grouped_kernel_32k_dram.txt",
                                          "rope_period_truncated_b200/csrc/wp_prefill.cu")
-                        if args.prefill_n in (0, 32768) else None),
+                        if args.prefill_n in (0, 32768) and args.grouping == "half-split" else None),
             "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
             "kernel_ms": round(prefill_ms, 4),
             "flops_per_launch": tile_flops,
@@ -529,7 +540,7 @@ def run_ours(args, rank, world, local):
     }
     if args.only != "all" or args.prefill_n:
         out["note"] = "restricted profiling case, not a bench line"
-    if rank == 0 and not args.no_cpu_baseline and world == 1 and args.only == "all":
+    if rank == 0 and not args.no_cpu_baseline and world == 1 and args.only == "all" and args.grouping == "half-split":
         out["cpu_baseline"] = cpu_baseline(path, args.cpu_seconds)
     return out
 

@@ -44,8 +44,17 @@ typedef enum {
 
 /* RoPE rotation layouts. Interleaved [KC, RoPE matrix]: channel c rotates the
  * dim pair (2c, 2c+1). Half-split: channel c rotates (c, c + d_h/2), the
- * rotate_half convention of Llama/Qwen checkpoints. */
-enum { WP_ROPE_INTERLEAVED = 0, WP_ROPE_HALF_SPLIT = 1 };
+ * rotate_half convention of Llama/Qwen checkpoints.
+ * WP_ROPE_HALF_SPLIT_PAIRED is for wp_rope_apply only: it rotates a half-split
+ * input exactly as WP_ROPE_HALF_SPLIT and writes channel c's pair to dims
+ * (2c, 2c+1) of the output, i.e. in the interleaved order. Q.K^T is unchanged
+ * when Q and K are permuted alike (V is untouched), so attention on paired Q
+ * and K is attention on the half-split model; wp_cutoffs, wp_prefill and
+ * wp_decode then take WP_ROPE_INTERLEAVED, and every 16-dim group holds 8
+ * whole channels: the group-end cutoffs of [RN §2.3, Table 12]
+ * (28, 160, 900, 5063, ... at theta 1e6) instead of the half-split groups'
+ * max over channels c and c + d_h/2. */
+enum { WP_ROPE_INTERLEAVED = 0, WP_ROPE_HALF_SPLIT = 1, WP_ROPE_HALF_SPLIT_PAIRED = 2 };
 
 /* Logit modes. Channel mode is the exact per-channel rule [RN §2.1, Eq. (6)];
  * grouped mode gives each 16-dim group the largest cutoff of the channels
@@ -87,6 +96,8 @@ int wp_cutoffs(int d_h, double theta, const double *freq_scale, double scale_all
  *   pos         device int32 [B, N] positions, or NULL: position = pos0 + t.
  *   theta, freq_scale (host, [d_h/2] or NULL), scale_all, layout: as in
  *               wp_cutoffs; frequencies are formed in fp64 on the host.
+ *   layout      also WP_ROPE_HALF_SPLIT_PAIRED (see its enum); then y must not
+ *               overlap x at all (WP_ERR_ARG).
  * The angle is formed and reduced modulo 2*pi in fp64, the rotation is fp32,
  * the result rounds to bf16. d_h in {64, 128}. Errors: WP_ERR_ARG,
  * WP_ERR_UNSUPPORTED, WP_ERR_CUDA.

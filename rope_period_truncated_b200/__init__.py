@@ -21,7 +21,7 @@ import numpy as np
 import torch
 
 __all__ = [
-    "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
+    "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "ROPE_HALF_SPLIT_PAIRED", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
     "WavePruneError", "library_path", "load_library",
     "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
     "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES", "wp_kcache_group_major", "KCACHE_ROWS", "KCACHE_GROUP_MAJOR",
@@ -30,6 +30,7 @@ __all__ = [
 
 ROPE_INTERLEAVED = 0
 ROPE_HALF_SPLIT = 1
+ROPE_HALF_SPLIT_PAIRED = 2  # wp_rope_apply only: half-split rotation written in the interleaved order
 MODE_GROUPED = 0
 MODE_CHANNEL = 1
 CUTOFF_INF = 2 ** 31 - 1

@@ -152,9 +152,11 @@ int wp_rope_apply(const void *x, void *y, int B, int N, int H, int d_h, const in
                   const double *freq_scale, double scale_all, int layout, void *stream) {
   if (x == nullptr || y == nullptr || !aligned16(x) || !aligned16(y)) return WP_ERR_ARG;
   if (B <= 0 || N <= 0 || H <= 0) return WP_ERR_ARG;
-  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
+  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT && layout != WP_ROPE_HALF_SPLIT_PAIRED)
+    return WP_ERR_ARG;
   if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
   if (!freq_args_ok(d_h, theta, freq_scale, scale_all)) return WP_ERR_ARG;
+  if (layout == WP_ROPE_HALF_SPLIT_PAIRED && x == y) return WP_ERR_ARG;  // permutes dims: not in place
   if (x != y) {  // only exact in-place aliasing is allowed
     const uintptr_t a0 = reinterpret_cast<uintptr_t>(x), b0 = reinterpret_cast<uintptr_t>(y);
     const uintptr_t n = static_cast<uintptr_t>(B) * N * H * d_h * 2;

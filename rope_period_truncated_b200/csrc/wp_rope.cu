@@ -81,7 +81,10 @@ __global__ void __launch_bounds__(ROPE_THREADS) rope_interleaved_kernel(const Ro
 
 // Half-split: thread (token, chunk) owns channels [8*chunk, 8*chunk + 8),
 // whose dims are [8*chunk, +8) and [C + 8*chunk, +8), C = D/2.
-template <int D>
+// PAIRED: write channel c's rotated pair to dims 2c, 2c+1 (the interleaved
+// order) instead of back to c, c + D/2; then every 16-dim group holds 8 whole
+// channels. Not in place (the writes land on other threads' inputs).
+template <int D, bool PAIRED>
 __global__ void __launch_bounds__(ROPE_THREADS) rope_half_split_kernel(const RopeArgs a) {
   constexpr int C = D / 2;
   constexpr int CHUNKS = C / 8;
@@ -108,8 +111,22 @@ __global__ void __launch_bounds__(ROPE_THREADS) rope_half_split_kernel(const Rop
       u[t] = f[t] * cs[t] - g[t] * sn[t];
       v[t] = f[t] * sn[t] + g[t] * cs[t];
     }
-    y[lo] = pack8(u);
-    y[hi] = pack8(v);
+    if (PAIRED) {
+      float w0[8], w1[8];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        w0[2 * t] = u[t];
+        w0[2 * t + 1] = v[t];
+        w1[2 * t] = u[t + 4];
+        w1[2 * t + 1] = v[t + 4];
+      }
+      const int64_t out = (token * a.H * D + static_cast<int64_t>(hh) * D + 16 * chunk) / 8;
+      y[out] = pack8(w0);
+      y[out + 1] = pack8(w1);
+    } else {
+      y[lo] = pack8(u);
+      y[hi] = pack8(v);
+    }
   }
 }
 
@@ -125,11 +142,16 @@ cudaError_t launch_rope(const RopeArgs &a, int d_h, int layout, cudaStream_t str
       rope_interleaved_kernel<128><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
     else
       rope_interleaved_kernel<64><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
+  } else if (layout == 1) {
+    if (d_h == 128)
+      rope_half_split_kernel<128, false><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
+    else
+      rope_half_split_kernel<64, false><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
   } else {
     if (d_h == 128)
-      rope_half_split_kernel<128><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
+      rope_half_split_kernel<128, true><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
     else
-      rope_half_split_kernel<64><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
+      rope_half_split_kernel<64, true><<<static_cast<unsigned>(blocks), ROPE_THREADS, 0, stream>>>(a);
   }
   return cudaGetLastError();
 }

@@ -180,7 +180,9 @@ def test_rope_rejects_bad_arguments(lib):
     assert f(FAKE, FAKE + 64, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG  # partial overlap
     assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 0.5, None, 1.0, 0, None) == wp.WP_ERR_ARG       # theta
     assert f(FAKE, FAKE, 1, 4, 2, 48, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_UNSUPPORTED
-    assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 2, None) == wp.WP_ERR_ARG       # layout
+    assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 3, None) == wp.WP_ERR_ARG       # layout
+    # the paired half-split order permutes dims: never in place
+    assert f(FAKE, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, wp.ROPE_HALF_SPLIT_PAIRED, None) == wp.WP_ERR_ARG
 
 
 def test_status_strings(lib):

@@ -86,3 +86,54 @@ def test_rope_full_size_sampled_tokens(name):
     xs = q[0, tok].unsqueeze(0)          # [1, 512, H, d]
     ys = y[0, tok.cuda()].unsqueeze(0)
     _check(ys, xs, w.theta, w.layout, pos=tok.numpy().reshape(1, -1), scale_all=w.scale_all)
+
+
+def _paired_perm(d):
+    """Output dim 2c takes half-split dim c, dim 2c+1 takes dim c + d/2."""
+    C = d // 2
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2] = np.arange(C)
+    perm[1::2] = np.arange(C) + C
+    return perm
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rope_half_split_paired_is_a_permutation(d):
+    """WP_ROPE_HALF_SPLIT_PAIRED is the half-split rotation with channel c's
+    pair moved to dims (2c, 2c+1): bit-identical to permuting the half-split
+    result."""
+    g = torch.Generator().manual_seed(50 + d)
+    x = torch.randn(2, 300, 3, d, generator=g).to(torch.bfloat16).cuda()
+    pos = torch.randint(0, 40000, (2, 300), generator=g).to(torch.int32).cuda()
+    hs = wp.wp_rope_apply(x, 1e6, wp.ROPE_HALF_SPLIT, pos=pos)
+    pr = wp.wp_rope_apply(x, 1e6, wp.ROPE_HALF_SPLIT_PAIRED, pos=pos)
+    torch.cuda.synchronize()
+    perm = torch.from_numpy(_paired_perm(d)).cuda()
+    assert torch.equal(pr, hs[..., perm])
+
+
+def test_prefill_paired_grouping_matches_oracle():
+    """Paper-equivalent grouping of a half-split model: Q and K rotated into
+    the interleaved order, then the interleaved group cutoffs (8 whole
+    channels per group, [RN §2.3, Table 12]). The oracle rotates half-split
+    in fp64, permutes the same way and applies the grouped rule with the
+    interleaved cutoffs."""
+    g = torch.Generator().manual_seed(77)
+    B, N, Hq, Hkv, d, theta = 1, 700, 4, 2, 128, 1e6
+    q = torch.randn(B, N, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, N, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, N, Hkv, d, generator=g).to(torch.bfloat16)
+    _, wg = oracle.cutoffs(d, theta, oracle.INTERLEAVED)
+    wg = np.asarray(wg) // 40  # shrink the windows so that N = 700 spans several cutoffs
+    wg = np.maximum(wg, 0).astype(np.int32)
+    qp = wp.wp_rope_apply(q.cuda(), theta, wp.ROPE_HALF_SPLIT_PAIRED)
+    kp = wp.wp_rope_apply(k.cuda(), theta, wp.ROPE_HALF_SPLIT_PAIRED)
+    o, lse = wp.wp_prefill(qp, kp, v.cuda(), wg, wp.MODE_GROUPED, wp.ROPE_INTERLEAVED)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    perm = _paired_perm(d)
+    qo = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(oracle.rope(widen(q), theta, oracle.HALF_SPLIT)))[..., perm]
+    ko = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(oracle.rope(widen(k), theta, oracle.HALF_SPLIT)))[..., perm]
+    ro, rl = oracle.attention(qo, ko, widen(v), wg, oracle.MODE_GROUPED, oracle.INTERLEAVED)
+    from parity import assert_attention_close
+    assert_attention_close(o, lse, ro, rl, "paired grouping")
