@@ -98,6 +98,22 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def bench_config(args, world, wg):
+    """The workload description both arms print."""
+    return {
+        "workload": "prefill long_32k (B1 Hq32/Hkv8 N32768 d128 theta1e6 half-split, grouped cutoffs) + "
+                    "decode_32k (16 seqs Hq32/Hkv8 d128 L~U[16384,32768]); step = rope Q,K + prefill + "
+                    "rope q + split-KV decode",
+        "l2": "inputs larger than L2 each step (384 MiB prefill Q/K/V, 2 GiB KV cache); no flush",
+        "parallelism": f"replicas x{world} (independent heads/sequences, no collective)",
+        "group_cutoffs": [int(x) for x in wg],
+        "decode_kcache": ("group-major [B,Hkv,d/16,L,16]" if args.kcache == "group-major"
+                          else "rows [B,Hkv,L,d]"),
+        "grouping": ("half-split groups (max over channels c and c+64)" if args.grouping == "half-split"
+                     else "paired: 8 whole channels per group (interleaved order after rope)"),
+    }
+
+
 def profiled_traffic(summary: str, source: str):
     """DRAM bytes per launch from a committed ncu summary under profiles/, or
     None when the kernel source has changed since it was captured."""
@@ -489,18 +505,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": "prefill long_32k (B1 Hq32/Hkv8 N32768 d128 theta1e6 half-split, grouped cutoffs) + "
-                        "decode_32k (16 seqs Hq32/Hkv8 d128 L~U[16384,32768]); step = rope Q,K + prefill + "
-                        "rope q + split-KV decode",
-            "l2": "inputs larger than L2 each step (384 MiB prefill Q/K/V, 2 GiB KV cache); no flush",
-            "parallelism": f"replicas x{world} (independent heads/sequences, no collective)",
-            "group_cutoffs": [int(x) for x in path.wg],
-            "decode_kcache": ("group-major [B,Hkv,d/16,L,16]" if args.kcache == "group-major"
-                              else "rows [B,Hkv,L,d]"),
-            "grouping": ("half-split groups (max over channels c and c+64)" if args.grouping == "half-split"
-                         else "paired: 8 whole channels per group (interleaved order after rope)"),
-        },
+        "config": bench_config(args, world, path.wg),
         "roofline": {
             "kernel": "wp_prefill (grouped, tcgen05)",
             "bound": "tensor",
@@ -547,7 +552,7 @@ def run_ours(args, rank, world, local):
 
 # ----------------------------------------------------------------------------- reference arm
 
-def run_reference(args):
+def run_reference(args, world=1):
     """The fp64 oracle as the reference arm: each step is a bounded sample of
     query rows of the 32K prefill, timed on the host cores."""
     import oracle
@@ -592,7 +597,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "prefill long_32k sampled rows (B1 Hq32/Hkv8 N32768 d128 theta1e6 half-split)"},
+        "config": bench_config(args, world, wg),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -603,7 +608,7 @@ def main():
     rank, world, local = dist_env()
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args)), flush=True)
+            print(json.dumps(run_reference(args, world)), flush=True)
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
