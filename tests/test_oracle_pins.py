@@ -399,3 +399,29 @@ def test_tile_classes_ragged_vs_numpy(N, BM, BN):
                 if want < 3:
                     want_counts[g, want] += 1
     assert np.array_equal(counts, want_counts)
+
+
+def test_paired_order_is_the_half_split_model_in_channel_mode():
+    """Moving channel c's half-split pair (c, c + d/2) to dims (2c, 2c+1) of
+    both Q and K leaves the exact per-channel rule unchanged ([RN §2.1, Eq.
+    (6)] depends on channels, not on where their dims sit): the interleaved
+    layout on the permuted data gives the half-split result on the original."""
+    rng = np.random.default_rng(5)
+    B, N, Hq, Hkv, d = 1, 40, 2, 1, 32
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    wc, _ = oracle.cutoffs(d, 30.0, oracle.HALF_SPLIT)
+    assert len(set(np.asarray(wc).tolist())) > 3  # several distinct windows inside N
+    C = d // 2
+    perm = np.empty(d, dtype=np.int64)
+    perm[0::2], perm[1::2] = np.arange(C), np.arange(C) + C
+    o1, l1 = oracle.attention(q, k, v, wc, oracle.MODE_CHANNEL, oracle.HALF_SPLIT)
+    o2, l2 = oracle.attention(q[..., perm], k[..., perm], v, wc, oracle.MODE_CHANNEL, oracle.INTERLEAVED)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=1e-12, atol=1e-12)
+    # and the paired order's groups are the interleaved groups: each holds 8
+    # whole channels, so its cutoff is the largest of those 8 channel cutoffs
+    wc_i, wg_i = oracle.cutoffs(d, 30.0, oracle.INTERLEAVED)
+    assert np.array_equal(np.asarray(wc_i), np.asarray(wc))
+    assert wg_i[0] == max(wc[:8]) and wg_i[1] == max(wc[8:])
