@@ -74,6 +74,9 @@ SMALL = [
     (384, 64, 4, 2, 1e4, wp.ROPE_INTERLEAVED, "mixed"),
     (300, 128, 2, 2, 1e6, wp.ROPE_HALF_SPLIT, "zero"),
     (300, 128, 2, 2, 1e6, wp.ROPE_HALF_SPLIT, "dense"),
+    (190, 128, 6, 2, 1e4, wp.ROPE_HALF_SPLIT, "wave"),    # 3 query heads per KV head: one head per CTA;
+                                                          # last tile of 62 rows (< one 64-key half)
+    (200, 64, 6, 3, 1e4, wp.ROPE_INTERLEAVED, "mixed"),   # 2 per KV head; last tile of 72 rows
 ]
 
 
