@@ -58,6 +58,8 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--kcache", choices=["group-major", "rows"], default="group-major",
                    help="layout of the decode K cache in HBM")
+    p.add_argument("--page-size", type=int, default=0,
+                   help="decode from a paged KV cache with pages of this many keys (0: contiguous)")
     p.add_argument("--grouping", choices=["half-split", "paired"], default="half-split",
                    help="paired: Q/K of the half-split model rotated into the interleaved order, groups of 8 "
                         "whole channels (the pages' grouping, Table 12 cutoffs)")
@@ -111,6 +113,8 @@ def bench_config(args, world, wg):
                           else "rows [B,Hkv,L,d]"),
         "grouping": ("half-split groups (max over channels c and c+64)" if args.grouping == "half-split"
                      else "paired: 8 whole channels per group (interleaved order after rope)"),
+        **({"decode_kv_pages": f"{args.page_size} keys per page, pages shuffled in the pool"}
+           if args.page_size else {}),
     }
 
 
@@ -234,7 +238,7 @@ class ClockSampler:
 class Path:
     """Device buffers and launches of one hot-path step."""
 
-    def __init__(self, device, prefill_n=0, kcache_layout="group-major", grouping="half-split"):
+    def __init__(self, device, prefill_n=0, kcache_layout="group-major", grouping="half-split", page_size=0):
         import dataclasses
         import rope_period_truncated_b200 as wp
         self.wp = wp
@@ -265,6 +269,27 @@ class Path:
         if kcache_layout == "group-major":
             self.kc = wp.wp_kcache_group_major(self.kc)
         self.vc = vc.to(device)
+        self.page_size = page_size
+        if page_size:
+            # the same keys in a paged pool: pages shuffled, one block table per sequence
+            B_, Hkv_, L_, d_ = vc.shape
+            mp = L_ // page_size
+            perm = torch.randperm(B_ * mp, generator=torch.Generator().manual_seed(7)).to(device)
+            vpg = self.vc.reshape(B_, Hkv_, mp, page_size, d_).permute(0, 2, 1, 3, 4).reshape(B_ * mp, Hkv_,
+                                                                                              page_size, d_)
+            self.v_pages = torch.empty_like(vpg)
+            self.v_pages[perm] = vpg
+            if kcache_layout == "group-major":
+                G_ = d_ // 16
+                kpg = self.kc.reshape(B_, Hkv_, G_, mp, page_size, 16).permute(0, 3, 1, 2, 4, 5).reshape(
+                    B_ * mp, Hkv_, G_, page_size, 16)
+            else:
+                kpg = self.kc.reshape(B_, Hkv_, mp, page_size, d_).permute(0, 2, 1, 3, 4).reshape(
+                    B_ * mp, Hkv_, page_size, d_)
+            self.k_pages = torch.empty_like(kpg)
+            self.k_pages[perm] = kpg
+            self.block_table = perm.to(torch.int32).reshape(B_, mp).contiguous()
+            del vpg, kpg
         self.lens_host = lens
         self.lens = lens.to(device)
         self.pos = (lens - 1).to(torch.int32).reshape(dw.B, 1).to(device)
@@ -293,6 +318,10 @@ class Path:
 
     def decode_only(self, cut="wave"):
         dw = self.dw
+        if self.page_size:
+            return self.wp.wp_decode_paged(self.dqr.reshape(dw.B, dw.Hq, dw.d), self.k_pages, self.v_pages,
+                                           self.block_table, self.lens, self.dwg if cut == "wave" else None,
+                                           out=self.do, lse=self.dlse, workspace=self.ws)
         return self.wp.wp_decode(self.dqr.reshape(dw.B, dw.Hq, dw.d), self.kc, self.vc, self.lens,
                                  self.dwg if cut == "wave" else None, out=self.do, lse=self.dlse,
                                  workspace=self.ws)
@@ -359,7 +388,7 @@ def run_ours(args, rank, world, local):
     wpbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    path = Path(dev, args.prefill_n, args.kcache, args.grouping)
+    path = Path(dev, args.prefill_n, args.kcache, args.grouping, args.page_size)
     peaks, peak_kind = load_peaks()
     do_prefill = args.only in ("all", "prefill")
     do_decode = args.only in ("all", "decode")

@@ -214,6 +214,35 @@ int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vc
                  void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * wp_decode_paged — wp_decode_kl over a paged KV cache, as serving engines
+ * keep it: the keys of a sequence live in fixed-size pages from a shared pool,
+ * listed per sequence in a block table. (The pages' decode reads one
+ * contiguous cache; paging only changes where each key block is read from.)
+ *   k_pages     device bf16 K pool of n_pages pages, each [H_kv, page_size,
+ *               d_h] in WP_KCACHE_ROWS or [H_kv, d_h/16, page_size, 16] in
+ *               WP_KCACHE_GROUP_MAJOR (k_layout).
+ *   v_pages     device bf16 V pool of n_pages pages, each [H_kv, page_size, d_h].
+ *   page_size   keys per page, a multiple of 16 (>= 16).
+ *   block_table device int32 [B, max_pages]: entry j of sequence b is the page
+ *               holding its keys [j*page_size, (j+1)*page_size); only the
+ *               entries below ceil(lens[b] / page_size) are read. An entry
+ *               read outside [0, n_pages) makes the kernel write NaN rows for
+ *               that sequence (nothing is read from it).
+ *   lens        device int32 [B], each in 1..max_pages*page_size.
+ *   workspace   at least wp_decode_workspace_bytes(B, H_q, d_h,
+ *               max_pages*page_size) bytes, 256-byte aligned.
+ * Everything else as in wp_decode; results are bit-identical to wp_decode_kl
+ * on the same keys stored contiguously. Errors: WP_ERR_ARG (also: block_table
+ * NULL or not 4-byte aligned, n_pages/max_pages < 1, page_size not a positive
+ * multiple of 16), WP_ERR_UNSUPPORTED (also: max_pages*page_size > 2^30),
+ * WP_ERR_CUDA.
+ */
+int wp_decode_paged(const void *q, const void *k_pages, int k_layout, const void *v_pages, int n_pages, int page_size,
+                    const int32_t *block_table, int max_pages, const int32_t *lens, int B, int H_q, int H_kv, int d_h,
+                    const int32_t *group_cut, float softmax_scale, void *o, float *lse, void *workspace,
+                    size_t ws_bytes, void *stream);
+
+/*
  * wp_decode_static — wp_decode without a workspace argument, for callers that
  * cannot allocate device memory (for example a serving engine whose device
  * memory is planned up front and handed out by its own pool, or a decode loop

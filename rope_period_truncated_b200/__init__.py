@@ -25,6 +25,7 @@ __all__ = [
     "WavePruneError", "library_path", "load_library",
     "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
     "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES", "wp_kcache_group_major", "KCACHE_ROWS", "KCACHE_GROUP_MAJOR",
+    "wp_decode_paged",
     "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
 ]
 
@@ -80,6 +81,8 @@ def load_library():
     lib.wp_decode_static.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P]
     lib.wp_decode_kl.restype = I
     lib.wp_decode_kl.argtypes = [P, P, I, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
+    lib.wp_decode_paged.restype = I
+    lib.wp_decode_paged.argtypes = [P, P, I, P, I, I, P, I, P, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
     lib.wp_kcache_group_major.restype = I
     lib.wp_kcache_group_major.argtypes = [P, P, I, I, I, I, P]
     lib.wp_device_status.restype = I
@@ -273,6 +276,49 @@ def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens:
     _check("wp_decode", load_library().wp_decode_kl(
         _ptr(q), _ptr(kcache), k_layout, _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
         _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out, lse
+
+
+def wp_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                    lens: torch.Tensor, group_cut=None, softmax_scale: float = 0.0, out: torch.Tensor | None = None,
+                    lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None, want_lse: bool = True,
+                    stream=None):
+    """Split-KV decode over a paged cache. q [B,Hq,d]; v_pages [n_pages,Hkv,P,d];
+    k_pages the same (rows) or [n_pages,Hkv,d/16,P,16] (group-major);
+    block_table int32 [B, max_pages] (device); lens int32 [B] (device)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(v_pages, "v_pages", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(lens, "lens", torch.int32, 1)
+    B, Hq, d = q.shape
+    n_pages, Hkv, P, _ = v_pages.shape
+    if tuple(v_pages.shape) != (n_pages, Hkv, P, d) or block_table.shape[0] != B:
+        raise ValueError("paged cache shape mismatch")
+    if k_pages.dim() == 5:
+        _need(k_pages, "k_pages", torch.bfloat16, 5)
+        if tuple(k_pages.shape) != (n_pages, Hkv, d // 16, P, 16):
+            raise ValueError("group-major K pages shape mismatch")
+        k_layout = KCACHE_GROUP_MAJOR
+    else:
+        _need(k_pages, "k_pages", torch.bfloat16, 4)
+        if tuple(k_pages.shape) != tuple(v_pages.shape):
+            raise ValueError("K pages shape mismatch")
+        k_layout = KCACHE_ROWS
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = wp_decode_workspace_bytes(B, Hq, d, max_pages * P)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < ws_bytes:
+        raise ValueError("workspace too small")
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    _check("wp_decode_paged", load_library().wp_decode_paged(
+        _ptr(q), _ptr(k_pages), k_layout, _ptr(v_pages), n_pages, P, _ptr(block_table), max_pages, _ptr(lens), B, Hq,
+        Hkv, d, cut_p, float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 

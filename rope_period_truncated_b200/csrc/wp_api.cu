@@ -237,9 +237,12 @@ size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {
   return decode_workspace_bytes(B, H_q, nsplit, d_h);
 }
 
-int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
-                 int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
-                 void *workspace, size_t ws_bytes, void *stream) {
+// Shared argument checks and launch of the split-KV decode; block_table null
+// = contiguous caches of Lmax keys, else pages of page_size keys.
+static int decode_launch(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens,
+                         int Lmax, int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale,
+                         void *o, float *lse, void *workspace, size_t ws_bytes, const int32_t *block_table,
+                         int max_pages, int page_size, int n_pages, void *stream) {
   if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr ||
       workspace == nullptr)
     return WP_ERR_ARG;
@@ -274,12 +277,35 @@ int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vc
   a.nsplit = nsplit;
   a.chunk = DECODE_CHUNK;
   a.k_group_major = k_layout == WP_KCACHE_GROUP_MAJOR ? 1 : 0;
+  a.block_table = block_table;
+  a.max_pages = max_pages;
+  a.page_size = page_size;
+  a.n_pages = n_pages;
   for (int g = 0; g < 8; ++g) {
     a.cut[g] = (group_cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : group_cut[g];
     if (a.cut[g] < 0) return WP_ERR_ARG;
   }
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
   return from_cuda(launch_decode(a, d_h, static_cast<cudaStream_t>(stream)));
+}
+
+int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
+                 int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,
+                 void *workspace, size_t ws_bytes, void *stream) {
+  return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, group_cut, softmax_scale, o, lse,
+                       workspace, ws_bytes, nullptr, 0, 0, 0, stream);
+}
+
+int wp_decode_paged(const void *q, const void *k_pages, int k_layout, const void *v_pages, int n_pages, int page_size,
+                    const int32_t *block_table, int max_pages, const int32_t *lens, int B, int H_q, int H_kv, int d_h,
+                    const int32_t *group_cut, float softmax_scale, void *o, float *lse, void *workspace,
+                    size_t ws_bytes, void *stream) {
+  if (block_table == nullptr || (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0) return WP_ERR_ARG;
+  if (n_pages <= 0 || max_pages <= 0 || page_size < 16 || page_size % 16 != 0) return WP_ERR_ARG;
+  const int64_t Lmax = static_cast<int64_t>(max_pages) * page_size;
+  if (Lmax > (1ll << 30)) return WP_ERR_UNSUPPORTED;
+  return decode_launch(q, k_pages, k_layout, v_pages, lens, static_cast<int>(Lmax), B, H_q, H_kv, d_h, group_cut,
+                       softmax_scale, o, lse, workspace, ws_bytes, block_table, max_pages, page_size, n_pages, stream);
 }
 
 int wp_decode(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B, int H_q,

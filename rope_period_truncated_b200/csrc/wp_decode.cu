@@ -90,7 +90,7 @@ __device__ __forceinline__ uint32_t piece_off(int r, int p) {
   return static_cast<uint32_t>(r) * DecLayout<D>::ROWB + static_cast<uint32_t>((p ^ (r & 7)) * 16);
 }
 
-template <int D, int R, bool KGM>
+template <int D, int R, bool KGM, bool PAGED>
 __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeArgs a) {
   using L = DecLayout<D>;
   constexpr int PIECES = L::PIECES;
@@ -109,6 +109,19 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
   if (start >= len) {
     if (threadIdx.x < R) a.lse_part[part + static_cast<int64_t>(threadIdx.x) * a.nsplit] = -INFINITY;
     return;
+  }
+  if (PAGED) {
+    // A block-table entry outside [0, n_pages) poisons this split (LSE +inf):
+    // the combine then writes NaN rows for the sequence; nothing is read.
+    bool bad = false;
+    for (int j = start / a.page_size + lane; j <= (end - 1) / a.page_size; j += 32) {
+      const int pg = a.block_table[static_cast<int64_t>(b) * a.max_pages + j];
+      bad = bad || pg < 0 || pg >= a.n_pages;
+    }
+    if (__any_sync(0xffffffffu, bad)) {
+      if (threadIdx.x < R) a.lse_part[part + static_cast<int64_t>(threadIdx.x) * a.nsplit] = INFINITY;
+      return;
+    }
   }
   const int g = lane >> 2, t = lane & 3;
   const int64_t qpos = len - 1;
@@ -131,39 +144,59 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
 
   const __nv_bfloat16 *kbase = a.kc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;  // either layout
   const __nv_bfloat16 *vbase = a.vc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.Lmax * D;
+  // Where the 16 keys from kb0 on live: K (row of kb0, or group 0 of kb0 in
+  // the group-major layout, groups kgs elements apart) and V (row of kb0). A
+  // paged cache holds page_size keys per page; a 16-key block never crosses a
+  // page (page_size is a multiple of 16).
+  auto block_src = [&](int kb0, const __nv_bfloat16 *&kblk, const __nv_bfloat16 *&vblk, int64_t &kgs) {
+    if (PAGED) {
+      const int64_t page = a.block_table[static_cast<int64_t>(b) * a.max_pages + kb0 / a.page_size];
+      const int off = kb0 % a.page_size;
+      const int64_t pbase = (page * a.Hkv + hk) * a.page_size * D;  // both layouts: one page per (page, head)
+      kblk = a.kc + pbase + (KGM ? static_cast<int64_t>(off) * 16 : static_cast<int64_t>(off) * D);
+      vblk = a.vc + pbase + static_cast<int64_t>(off) * D;
+      kgs = static_cast<int64_t>(a.page_size) * 16;
+    } else {
+      kblk = kbase + (KGM ? static_cast<int64_t>(kb0) * 16 : static_cast<int64_t>(kb0) * D);
+      vblk = vbase + static_cast<int64_t>(kb0) * D;
+      kgs = static_cast<int64_t>(a.Lmax) * 16;
+    }
+  };
   const uint32_t ring = smem_u32(dsmem) + warp * L::WARP_BYTES;
 
   // Issue the loads of one 16-key block into stage `st`.
   auto load_block = [&](int kb0, int st) {
     const uint32_t kdst = ring + st * L::STAGE, vdst = kdst + L::TILE;
+    const __nv_bfloat16 *kblk, *vblk;
+    int64_t kgs;
+    block_src(kb0, kblk, vblk, kgs);
 #pragma unroll
     for (int it = 0; it < KEYS * PIECES / 32; ++it) {
       const int idx = it * 32 + lane;
       const int r = idx / PIECES, p = idx % PIECES;
       const int key = kb0 + r;
       const bool valid = key < end;
-      const int64_t row = valid ? key : kb0;  // any in-range address when nothing is read
+      const int64_t rr = valid ? r : 0;  // any in-range address when nothing is read
       if (!KGM) {
         const int64_t dist = qpos - key;
         const bool kin = valid && dist <= static_cast<int64_t>(a.cut[p >> 1]);
         // An out-of-window K piece is copied with source size 0: nothing is
         // read and its shared-memory slot is zero-filled, so the group adds
         // exactly 0 to the score.
-        cp_async16(kdst + piece_off<D>(r, p), kbase + row * D + 8 * p, kin ? 16u : 0u);
+        cp_async16(kdst + piece_off<D>(r, p), kblk + rr * D + 8 * p, kin ? 16u : 0u);
       }
-      cp_async16(vdst + piece_off<D>(r, p), vbase + row * D + 8 * p, valid ? 16u : 0u);
+      cp_async16(vdst + piece_off<D>(r, p), vblk + rr * D + 8 * p, valid ? 16u : 0u);
     }
     if (KGM) {
-      // group-major K: iteration it takes group it, lane = 2 * key + half
+      // group-major K: iteration gi takes group gi, lane = 2 * key + half
 #pragma unroll
       for (int gi = 0; gi < D / 16; ++gi) {
         const int r = lane >> 1, half = lane & 1;
         const int key = kb0 + r;
         const bool valid = key < end;
-        const int64_t row = valid ? key : kb0;
+        const int64_t rr = valid ? r : 0;
         const bool kin = valid && qpos - key <= static_cast<int64_t>(a.cut[gi]);
-        cp_async16(kdst + piece_off<D>(r, 2 * gi + half), kbase + (static_cast<int64_t>(gi) * a.Lmax + row) * 16 + 8 * half,
-                   kin ? 16u : 0u);
+        cp_async16(kdst + piece_off<D>(r, 2 * gi + half), kblk + gi * kgs + rr * 16 + 8 * half, kin ? 16u : 0u);
       }
     }
   };
@@ -304,20 +337,22 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   if (d == 0 && a.lse != nullptr) a.lse[bh] = (M + log2f(Lsum)) * 0.69314718055994531f;
 }
 
-template <int D, int R, bool KGM>
+template <int D, int R, bool KGM, bool PAGED>
 cudaError_t launch_split_l(const DecodeArgs &a, cudaStream_t stream) {
   const uint32_t smem = DecLayout<D>::BYTES;
-  cudaError_t e =
-      cudaFuncSetAttribute(decode_split_kernel<D, R, KGM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, R, KGM, PAGED>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nsplit, a.Hkv, a.B);
-  decode_split_kernel<D, R, KGM><<<grid, DEC_THREADS, smem, stream>>>(a);
+  decode_split_kernel<D, R, KGM, PAGED><<<grid, DEC_THREADS, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 template <int D, int R>
 cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
-  return a.k_group_major ? launch_split_l<D, R, true>(a, stream) : launch_split_l<D, R, false>(a, stream);
+  if (a.block_table != nullptr)
+    return a.k_group_major ? launch_split_l<D, R, true, true>(a, stream) : launch_split_l<D, R, false, true>(a, stream);
+  return a.k_group_major ? launch_split_l<D, R, true, false>(a, stream) : launch_split_l<D, R, false, false>(a, stream);
 }
 
 // One thread per 16-byte piece of the group-major output, in output order:

@@ -21,6 +21,8 @@ struct DecodeArgs {
   float *lse_part;                   // [B, Hq, nsplit], base-2
   int B, Hq, Hkv, Lmax, nsplit, chunk;
   int k_group_major;                 // K cache layout: 0 rows, 1 group-major
+  const int32_t *block_table;        // paged cache: [B, max_pages] page of each page_size-key block, or null
+  int max_pages, page_size, n_pages;
   int32_t cut[8];                    // group cutoffs
   float scale_log2;
 };

@@ -174,6 +174,30 @@ def test_decode_kl_and_kcache_conversion_reject_bad_arguments(lib):
     assert g(FAKE, FAKE + 4096, 1, 2, 100, 80, None) == wp.WP_ERR_UNSUPPORTED
 
 
+def test_decode_paged_rejects_bad_arguments(lib):
+    f = lib.wp_decode_paged
+    ws = lib.wp_decode_workspace_bytes(2, 8, 128, 64 * 64)
+    # q, k_pages, k_layout, v_pages, n_pages, page_size, block_table, max_pages, lens, B, Hq, Hkv, d, cut, scale,
+    # o, lse, ws, ws_bytes, stream
+    args = [FAKE, FAKE, wp.KCACHE_ROWS, FAKE, 100, 64, FAKE, 64, FAKE, 2, 8, 2, 128, None, ctypes.c_float(0.0),
+            FAKE, None, FAKE, ws, None]
+
+    def call(i, val):
+        a = list(args)
+        a[i] = val
+        return f(*a)
+
+    assert call(6, None) == wp.WP_ERR_ARG               # block table NULL
+    assert call(6, FAKE + 2) == wp.WP_ERR_ARG           # block table misaligned
+    assert call(5, 8) == wp.WP_ERR_ARG                  # page size below 16
+    assert call(5, 40) == wp.WP_ERR_ARG                 # page size not a multiple of 16
+    assert call(4, 0) == wp.WP_ERR_ARG                  # empty pool
+    assert call(7, 0) == wp.WP_ERR_ARG                  # no pages per sequence
+    assert call(2, 5) == wp.WP_ERR_ARG                  # K layout
+    assert call(18, ws - 1) == wp.WP_ERR_ARG            # workspace too small for max_pages * page_size keys
+    assert call(7, 1 << 26) == wp.WP_ERR_UNSUPPORTED    # 2^32 keys per sequence
+
+
 def test_rope_rejects_bad_arguments(lib):
     f = lib.wp_rope_apply
     assert f(None, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG

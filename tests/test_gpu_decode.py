@@ -145,3 +145,71 @@ def test_decode_group_major_workload():
     qo = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qo)).reshape(w.B, w.Hq, w.d)
     ro, rl = oracle.decode(qo, widen(kc), widen(vc), lens.numpy(), wg)
     assert_attention_close(o, lse, ro, rl, "decode_32k group-major")
+
+
+def _paged(kc, vc, P, extra, seed):
+    """Contiguous caches [B,Hkv,L,d] (L a multiple of P) -> shuffled page pools
+    [n_pages,Hkv,P,d] and the block table [B, L/P]."""
+    B, Hkv, L, d = kc.shape
+    mp = L // P
+
+    def pool_of(x):
+        pages = x.reshape(B, Hkv, mp, P, d).permute(0, 2, 1, 3, 4).reshape(B * mp, Hkv, P, d)
+        return pages
+
+    g = torch.Generator().manual_seed(seed)
+    n_pages = B * mp + extra
+    perm = torch.randperm(n_pages, generator=g)[: B * mp]
+    kp = torch.zeros((n_pages, Hkv, P, d), dtype=kc.dtype)
+    vp = torch.zeros((n_pages, Hkv, P, d), dtype=vc.dtype)
+    kp[perm] = pool_of(kc)
+    vp[perm] = pool_of(vc)
+    table = perm.to(torch.int32).reshape(B, mp)
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("P", [16, 64, 256])
+@pytest.mark.parametrize("group_major", [False, True])
+def test_decode_paged_matches_contiguous(P, group_major):
+    """A paged cache (shuffled pages in a larger pool) gives results
+    bit-identical to the same keys stored contiguously, in both K layouts."""
+    g = torch.Generator().manual_seed(61 + P)
+    B, Hq, Hkv, d, L = 3, 8, 2, 128, 3072
+    lens = torch.tensor([1, 3072, 1700], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, L, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, L, d, generator=g).to(torch.bfloat16)
+    _, wg = oracle.cutoffs(d, 1e4, oracle.HALF_SPLIT)
+    wg = np.minimum(wg, [5, 40, 300, 1100, 2000, 10 ** 6, 7, 1024]).astype(np.int32)
+    kp, vp, table = _paged(kc, vc, P, extra=5, seed=P)
+    kcd, kpd = kc.cuda(), kp.cuda()
+    if group_major:
+        kcd = wp.wp_kcache_group_major(kcd)
+        n = kp.shape[0]
+        kpd = kpd.reshape(n, Hkv, P, d // 16, 16).permute(0, 1, 3, 2, 4).contiguous()
+    o_ref, l_ref = wp.wp_decode(q.cuda(), kcd, vc.cuda(), lens.cuda(), wg)
+    o, lse = wp.wp_decode_paged(q.cuda(), kpd, vp.cuda(), table.cuda(), lens.cuda(), wg)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
+    ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o, lse, ro, rl, f"paged P={P} gm={group_major}")
+
+
+def test_decode_paged_bad_page_gives_nan_rows():
+    """A block-table entry outside the pool poisons only its own sequence."""
+    g = torch.Generator().manual_seed(9)
+    B, Hq, Hkv, d, L, P = 2, 4, 2, 64, 512, 64
+    lens = torch.tensor([512, 300], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, L, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, L, d, generator=g).to(torch.bfloat16)
+    kp, vp, table = _paged(kc, vc, P, extra=0, seed=1)
+    table[1, 2] = kp.shape[0] + 7  # a page of sequence 1 that does not exist
+    o, lse = wp.wp_decode_paged(q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), lens.cuda(), None)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    o = o.float().cpu()
+    assert torch.isnan(o[1]).all()
+    ro, rl = oracle.decode(widen(q[:1]), widen(kc[:1]), widen(vc[:1]), lens[:1].numpy(), np.full(d // 16, 2 ** 31 - 1))
+    assert_attention_close(o[:1].to(torch.bfloat16), lse[:1], ro, rl, "paged, sequence with valid pages")
