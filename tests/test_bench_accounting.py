@@ -1,0 +1,82 @@
+"""The bench's work accounting (useful FLOPs, required decode bytes, the ncu
+traffic lookup) checked against brute-force enumeration on small cases and
+against the figures the scope table states for the 32K workload. Host only."""
+import os
+
+import numpy as np
+import pytest
+
+import bench
+
+
+def _brute_pair_exact(N, d, wg):
+    total = 0
+    for i in range(N):
+        for j in range(i + 1):
+            total += 2 * 16 * sum(1 for w in wg if i - j <= w) + 2 * d
+    return total
+
+
+def _brute_tile_level(N, d, wg, BM=128, BN=128):
+    total = 0
+    nqb = (N + BM - 1) // BM
+    for qb in range(nqb):
+        qs, qe = qb * BM, min(qb * BM + BM, N) - 1
+        for kb in range(qb + 1):
+            ks, ke = kb * BN, min(kb * BN + BN, N) - 1
+            if ks > qe:
+                continue
+            dmax, dmin = qe - ks, (qs - ke if qs > ke else 0)
+            live = sum(1 for w in wg if dmin <= w)  # not skipped: full or boundary
+            total += live * 2 * BM * BN * 16 + 2 * BM * BN * d
+    return total
+
+
+@pytest.mark.parametrize("N", [1, 127, 300, 513])
+def test_prefill_flops_match_enumeration(N):
+    d, wg = 64, [0, 3, 130, 1000]
+    tile, pair, dense = bench.prefill_flops(N, d, 2, 3, wg)
+    assert pair == _brute_pair_exact(N, d, wg) * 2 * 3
+    assert tile == _brute_tile_level(N, d, wg) * 2 * 3
+    assert dense == _brute_tile_level(N, d, [10 ** 9] * (d // 16)) * 2 * 3  # every group kept
+
+
+def test_prefill_flops_32k_figures():
+    """Scope table: 6.922 TFLOP pair-exact useful work for the 32K prefill, and
+    8.796 TFLOP dense causal (same count with every group kept)."""
+    wg = [160, 5063, 160114, 5063255] * 2
+    _, pair, _ = bench.prefill_flops(32768, 128, 32, 1, wg)
+    _, pair_dense, _ = bench.prefill_flops(32768, 128, 32, 1, [2 ** 31 - 1] * 8)
+    assert abs(pair / 1e12 - 6.922) < 5e-4
+    assert abs(pair_dense / 1e12 - 8.796) < 5e-4
+
+
+def test_decode_required_bytes_match_enumeration():
+    rng = np.random.default_rng(3)
+    lens = rng.integers(1, 400, size=5)
+    wg = [2, 17, 100, 10 ** 6]
+    B, Hq, Hkv, d = 5, 8, 2, 64
+    req, dense = bench.decode_required_bytes(lens, wg, B, Hq, Hkv, d)
+    kv = 0
+    for L in lens:
+        q = L - 1
+        for j in range(L):
+            kv += 32 * sum(1 for w in wg if q - j <= w) + 2 * d  # K of in-window groups + V row
+    io = B * Hq * d * 2 * 2 + B * Hq * 4
+    assert req == kv * Hkv + io
+    assert dense == sum(4 * d * L for L in lens) * Hkv + io
+
+
+def test_profiled_traffic_follows_the_source(tmp_path, monkeypatch):
+    import hashlib
+    src = tmp_path / "kernel.cu"
+    src.write_text("kernel v1\n")
+    h = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "k.txt").write_text(
+        f"# comment: with a colon\nsource_sha256_16: {h}\ndram_bytes_per_launch: 12345\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k.txt", "kernel.cu") == 12345
+    src.write_text("kernel v2\n")  # the kernel changed since the capture
+    assert bench.profiled_traffic("k.txt", "kernel.cu") is None
+    assert bench.profiled_traffic("missing.txt", "kernel.cu") is None
