@@ -142,9 +142,9 @@ int wp_schedule(int N, int BM, int BN, const int32_t *cut, int n_cut, uint8_t *c
  *   softmax_scale  > 0, or <= 0 for 1/sqrt(d_h) [RN §2.1, detail 3].
  * d_h in {64, 128}. Masked channels add 0 to the logit (the pair still takes
  * part in the softmax) [RN §2.1, detail 1]. Errors: WP_ERR_ARG,
- * WP_ERR_UNSUPPORTED (also: B*H_kv or ceil(N/128) above 65535), WP_ERR_CUDA
- * (also: grouped mode with N beyond what one CTA's shared memory can hold the
- * key-block table for, about 1.1M tokens at d_h = 128).
+ * WP_ERR_UNSUPPORTED (also: B*H_kv above 65535; grouped mode with N above
+ * 2^20, the longest sequence whose key-block table fits one CTA's shared
+ * memory), WP_ERR_CUDA.
  */
 int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int N, int H_q, int H_kv,
                int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream);

@@ -223,6 +223,8 @@ int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
   a.scale_log2 = scale_log2;
   a.wait_limit = g_wait_limit;
   if ((N + 127) / 128 > 65535 || static_cast<int64_t>(H_kv) * B > 65535) return WP_ERR_UNSUPPORTED;
+  // the kernel keeps one key-block table per CTA in shared memory: 2^20 tokens fit at every d_h
+  if (N > (1 << 20)) return WP_ERR_UNSUPPORTED;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, B, N, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
       !make_map(&tk, k, B, N, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||

@@ -123,6 +123,7 @@ def test_prefill_rejects_bad_arguments(lib):
     assert call(d=96) == wp.WP_ERR_UNSUPPORTED
     assert call(d=100) == wp.WP_ERR_ARG
     assert call(mode=5) == wp.WP_ERR_ARG
+    assert call(N=(1 << 20) + 1) == wp.WP_ERR_UNSUPPORTED  # key-block table beyond shared memory
     assert call(layout=3) == wp.WP_ERR_ARG
     negcut = (ctypes.c_int32 * 8)(*([-1] * 8))
     assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 64, 4, 2, 128, 0, negcut, 1, ctypes.c_float(0.0), None) == wp.WP_ERR_ARG
