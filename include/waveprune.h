@@ -20,7 +20,11 @@
  *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
  *   - A kernel that waits longer than the wait limit on one of its internal
  *     barriers stops, records WP_ERR_TIMEOUT in a device status word and
- *     returns; wp_device_status() reads and clears that word.
+ *     returns; wp_device_status() reads and clears that word. The word
+ *     carries over between calls: while it is set, every wp_prefill on that
+ *     device skips its work and writes NaN to all its O rows and LSE entries
+ *     (the call itself still returns WP_OK), until wp_device_status() has
+ *     read and cleared it. Outputs are never left holding stale values.
  *   - bf16 is IEEE bfloat16 (raw 16-bit patterns); outputs round to nearest
  *     even.
  */
@@ -261,9 +265,11 @@ int wp_decode_paged(const void *q, const void *k_pages, int k_layout, const void
  *   Every call on a device shares the one array and leaves its contents
  *   behind; nothing in it needs to start at zero. Calls whose kernels overlap
  *   on the GPU (e.g. on two streams without ordering) race on the array.
- *   Errors: WP_ERR_UNSUPPORTED when wp_decode_workspace_bytes(B, H_q, d_h,
- *   Lmax) exceeds WP_DECODE_STATIC_SCRATCH_BYTES (nothing is launched);
- *   otherwise those of wp_decode.
+ *   Errors: WP_ERR_ARG for a null or misaligned q, kcache, vcache, lens, o
+ *   or lse (checked first, whatever the sizes); WP_ERR_UNSUPPORTED when
+ *   wp_decode_workspace_bytes(B, H_q, d_h, Lmax) exceeds
+ *   WP_DECODE_STATIC_SCRATCH_BYTES, or on a device ordinal of 64 or more
+ *   (nothing is launched); otherwise those of wp_decode.
  */
 #define WP_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
 int wp_decode_static(const void *q, const void *kcache, const void *vcache, const int32_t *lens, int Lmax, int B,

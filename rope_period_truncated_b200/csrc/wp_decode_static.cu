@@ -27,10 +27,12 @@ void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_decode_scratch on the current device. In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device with that device current, and cached.
+// per device with that device current, and cached. Device ordinals from
+// kMaxDevices on are not served.
 int scratch_address(void **out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WP_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return WP_ERR_CUDA;
+  if (dev >= kMaxDevices) return WP_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_scratch_addr[dev] == nullptr) {
     void *p = nullptr;
@@ -46,6 +48,13 @@ int scratch_address(void **out) {
 extern "C" int wp_decode_static(const void *q, const void *kcache, const void *vcache, const int32_t *lens,
                                 int Lmax, int B, int H_q, int H_kv, int d_h, const int32_t *group_cut,
                                 float softmax_scale, void *o, float *lse, void *stream) {
+  // The pointer checks of wp_decode come first, so a bad pointer is reported
+  // as such whatever the batch size.
+  const auto misaligned = [](const void *p, uintptr_t m) { return (reinterpret_cast<uintptr_t>(p) & m) != 0; };
+  if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr) return WP_ERR_ARG;
+  if (misaligned(q, 15) || misaligned(kcache, 15) || misaligned(vcache, 15) || misaligned(o, 15) ||
+      misaligned(lens, 3) || (lse != nullptr && misaligned(lse, 3)))
+    return WP_ERR_ARG;
   const size_t need = wp_decode_workspace_bytes(B, H_q, d_h, Lmax);
   if (need == 0) return WP_ERR_ARG;
   if (need > kScratchBytes) return WP_ERR_UNSUPPORTED;  // batch too large for the fixed scratch

@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const long long lim = a.wait_limit;
 
   if (threadIdx.x == 0) {
-    // An earlier CTA already gave up: skip the work, the call has failed.
+    // A kernel of this library has given up since the status word was last
+    // read (this call or an earlier one): skip the work and write NaN rows.
     *abort_flag = *reinterpret_cast<volatile int *>(&g_status) != 0 ? 1 : 0;
     mbar_init(B.q_full, 1);
     for (int s = 0; s < KST; ++s) {
@@ -685,8 +686,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (i < a.N && a.lse != nullptr)
         a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     } else {
-      // Tell the other roles to stop waiting for this warp's progress.
+      // Tell the other roles to stop waiting for this warp's progress, and
+      // never leave the caller's buffers with stale rows: an aborted CTA
+      // writes NaN to its O rows and LSE entries.
       *abort_flag = 1;
+      if (i < a.N) {
+        __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) reinterpret_cast<uint4 *>(orow)[k] = nan4;
+        if (a.lse != nullptr) a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = __int_as_float(0x7FC00000);
+      }
     }
   }
 

@@ -31,6 +31,15 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(cons
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (a.Hq / a.Hkv);
   if (i >= a.N) return;
+  if (*reinterpret_cast<volatile int *>(&g_status) != 0) {
+    // A kernel of this library has given up since the status word was last
+    // read: write NaN rows rather than leave stale outputs.
+    __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+    for (int t = lane; t < D; t += 32) orow[t] = __ushort_as_bfloat16(0x7FC0);
+    if (lane == 0 && a.lse != nullptr)
+      a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = __int_as_float(0x7FC00000);
+    return;
+  }
   const __nv_bfloat16 *qrow = a.q + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
   for (int t = lane; t < D; t += 32) q_s[warp][t] = __bfloat162float(qrow[t]);
   __syncwarp();

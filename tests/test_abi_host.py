@@ -199,6 +199,26 @@ def test_decode_paged_rejects_bad_arguments(lib):
     assert call(7, 1 << 26) == wp.WP_ERR_UNSUPPORTED    # 2^32 keys per sequence
 
 
+def test_decode_static_checks_pointers_before_sizes(lib):
+    """A null or misaligned pointer is WP_ERR_ARG even for a batch too large
+    for the fixed scratch; a well-formed oversized batch is WP_ERR_UNSUPPORTED.
+    Neither reaches the GPU."""
+    f = lib.wp_decode_static
+    big = [FAKE, FAKE, FAKE, FAKE, 131072, 64, 64, 8, 128, None, ctypes.c_float(0.0), FAKE, None, None]
+    assert lib.wp_decode_workspace_bytes(64, 64, 128, 131072) > wp.DECODE_STATIC_SCRATCH_BYTES
+
+    def call(i, val):
+        a = list(big)
+        a[i] = val
+        return f(*a)
+
+    assert call(0, None) == wp.WP_ERR_ARG               # q NULL
+    assert call(3, None) == wp.WP_ERR_ARG               # lens NULL
+    assert call(11, FAKE + 8) == wp.WP_ERR_ARG          # o misaligned
+    assert call(12, FAKE + 2) == wp.WP_ERR_ARG          # lse misaligned
+    assert f(*big) == wp.WP_ERR_UNSUPPORTED
+
+
 def test_rope_rejects_bad_arguments(lib):
     f = lib.wp_rope_apply
     assert f(None, FAKE, 1, 4, 2, 128, None, 0, 1e4, None, 1.0, 0, None) == wp.WP_ERR_ARG

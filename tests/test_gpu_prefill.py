@@ -1,9 +1,10 @@
 """GPU parity of wp_prefill (grouped tcgen05 path and exact channel path)
 against the fp64 oracle, on the same seeded inputs.
 
-Small cases run the oracle on every row (several 128-row tiles plus ragged
-tails, multiple boundary cutoffs per tile, all-masked and dense tables); the
-full-size workloads are checked on sampled rows, through the same launch
+Small cases and the Qwen3-shaped 4K workload run the oracle on every row
+(several 128-row tiles plus ragged tails, multiple boundary cutoffs per tile,
+all-masked and dense tables); the 32K and 128K workloads are checked on
+sampled rows, through the same launch
 (rope of Q and K, then prefill) that the bench times."""
 import numpy as np
 import pytest
@@ -113,9 +114,18 @@ def _sampled_check(name, per_head):
     return assert_attention_close(og, lg, ro, rl, name)
 
 
-def test_qwen3_shaped_sampled_rows():
-    """B2 H32/8 N4096 d128 theta 1e6 half-split, per-dim Q/K scales."""
-    _sampled_check("qwen3_8b_4k", 64)
+def test_qwen3_shaped_every_row():
+    """B2 H32/8 N4096 d128 theta 1e6 half-split, per-dim Q/K scales: every
+    row of every head (262,144 rows) against the oracle, through the same
+    rope + prefill launches the bench times."""
+    w = syn.workload("qwen3_8b_4k")
+    q, k, v = syn.prefill_inputs(w)
+    _, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
+    o, lse = _gpu_path(q, k, v, w.theta, w.layout, wg, wp.MODE_GROUPED, scale_all=w.scale_all)
+    qr = _oracle_rotated(q, w.theta, w.layout, w.scale_all)
+    kr = _oracle_rotated(k, w.theta, w.layout, w.scale_all)
+    ro, rl = oracle.attention(qr, kr, widen(v), wg, oracle.MODE_GROUPED, w.layout)
+    assert_attention_close(o, lse, ro, rl, "qwen3_8b_4k every row")
 
 
 def test_long_32k_sampled_rows():

@@ -2,9 +2,10 @@
 (e.g. an engine whose device memory is planned up front and served by its own
 pool, or a decode loop that must not reach cudaMalloc/cudaFree). Its split
 partials live in the library's fixed 16 MiB device scratch instead of a
-caller workspace. Checked through the C ABI against wp_decode on the same
-inputs, on two calls in a row (the second call reuses the scratch the first
-one left behind), and for the size limit.
+caller workspace. Checked through the C ABI against the fp64 oracle and
+against wp_decode on the same inputs, on three calls in a row (each reuses
+the scratch the one before left behind; the second has the first one's shape
+with fewer active splits), and for the size limit.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test."""
@@ -16,7 +17,7 @@ import torch
 
 import oracle
 import rope_period_truncated_b200 as wp
-from parity import O_MAX_ABS, O_MEAN_ABS, LSE_REL
+from parity import LSE_REL, O_MAX_ABS, O_MEAN_ABS, assert_attention_close, widen
 
 pytestmark = pytest.mark.gpu
 
@@ -46,11 +47,17 @@ def _close(o_a, l_a, o_b, l_b):
     assert (lerr <= LSE_REL * torch.clamp(l_b.abs(), min=1.0)).all()
 
 
-def test_static_scratch_decode_matches_workspace_decode_twice():
+def test_static_scratch_decode_matches_oracle_and_workspace_decode():
+    """Three calls in a row on the one scratch array: a long batch, then the
+    same shape with shorter sequences (fewer splits hold keys, so stale
+    partials of the first call sit beyond the active ones), then another
+    shape. Each result is checked against the fp64 oracle and against
+    wp_decode with a caller workspace."""
     lib = wp.load_library()
     _, wg = oracle.cutoffs(128, 1e6, oracle.HALF_SPLIT)
     cases = [
-        (31, 4, 8, 2, 128, 3000, [1, 2999, 1500, 1025]),
+        (31, 4, 8, 2, 128, 3000, [1, 2999, 1500, 3000]),
+        (33, 4, 8, 2, 128, 3000, [700, 1, 100, 1025]),
         (32, 3, 16, 2, 128, 5000, [4999, 7, 2048]),
     ]
     for seed, B, Hq, Hkv, d, Lmax, lens in cases:
@@ -62,6 +69,8 @@ def test_static_scratch_decode_matches_workspace_decode_twice():
         torch.cuda.synchronize()
         assert wp.wp_device_status() == wp.WP_OK
         _close(o, lse, o_ref, l_ref)
+        ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), np.asarray(lens, dtype=np.int32), wg)
+        assert_attention_close(o, lse, ro, rl, f"static decode lens={lens}")
 
 
 def test_static_scratch_rejects_oversized_batch():
@@ -69,7 +78,7 @@ def test_static_scratch_rejects_oversized_batch():
     lib = wp.load_library()
     B, Hq, Hkv, d, Lmax = 64, 64, 8, 128, 131072
     assert wp.wp_decode_workspace_bytes(B, Hq, d, Lmax) > wp.DECODE_STATIC_SCRATCH_BYTES
-    t = torch.empty(16, dtype=torch.bfloat16, device="cuda")  # never read: the size check comes first
+    t = torch.empty(16, dtype=torch.bfloat16, device="cuda")  # never read: nothing is launched
     p = ctypes.c_void_p(t.data_ptr())
     rc = lib.wp_decode_static(p, p, p, p, Lmax, B, Hq, Hkv, d, None, ctypes.c_float(0.0), p, p,
                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
