@@ -154,6 +154,43 @@ int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
                int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream);
 
 /*
+ * wp_prefill_ex — wp_prefill with one cutoff table per query head, and
+ * packed batches of sequences of different lengths. [RN §5] names
+ * head-specific thresholds as the next step after one table per model; the
+ * rule per head is the same as in wp_prefill.
+ *   cu_seqlens  NULL: a uniform batch, laid out as in wp_prefill (q, o
+ *               [B, N, H_q, d_h]; k, v [B, N, H_kv, d_h]; lse [B, H_q, N]);
+ *               total_tokens is ignored.
+ *               Otherwise device int32 [B+1], 4-byte aligned: sequence b is
+ *               rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of the packed
+ *               q, o [T, H_q, d_h] and k, v [T, H_kv, d_h] (T = total_tokens),
+ *               positions restart at 0 in every sequence, and lse is
+ *               [H_q, T]. N is an upper bound of the lengths (it sizes the
+ *               launch). A sequence whose offsets fall outside [0, T], run
+ *               backwards, or span more than N rows is skipped (its rows are
+ *               not written) and WP_ERR_ARG is recorded in the device status
+ *               word (see wp_device_status). Rows past the end of a sequence
+ *               are read only where the causal mask gives them weight exactly
+ *               0; V must therefore be finite in the whole buffer.
+ *   cut, cut_rows  cut_rows = 1: one table for every head (as in wp_prefill);
+ *               cut_rows = H_q: cut is [H_q][d_h/16] (grouped) or
+ *               [H_q][d_h/2] (channel mode), row h for query head h (two
+ *               heads that share a KV head share its K loads, which cover the
+ *               groups either of them keeps). cut may be NULL only with
+ *               cut_rows = 1 (dense).
+ * Everything else as in wp_prefill. Errors: those of wp_prefill, and
+ * WP_ERR_ARG (cut_rows not 1 or H_q; cu_seqlens misaligned or
+ * total_tokens <= 0 with cu_seqlens), WP_ERR_UNSUPPORTED (more than 2048
+ * table entries in all, i.e. cut_rows x d_h/16 or cut_rows x d_h/2;
+ * total_tokens of 2^31 - 256 or more; grouped mode with cut_rows = H_q and N
+ * above 2^19, where the two heads' key-block tables no longer fit one CTA's
+ * shared memory).
+ */
+int wp_prefill_ex(const void *q, const void *k, const void *v, void *o, float *lse, const int32_t *cu_seqlens,
+                  int B, int N, int64_t total_tokens, int H_q, int H_kv, int d_h, int mode, const int32_t *cut,
+                  int cut_rows, int layout, float softmax_scale, void *stream);
+
+/*
  * wp_decode_workspace_bytes — size of the scratch that wp_decode needs for
  * the split-KV partial results of a batch (fp32 partial O and LSE per split).
  */
@@ -279,7 +316,8 @@ int wp_decode_static(const void *q, const void *kcache, const void *vcache, cons
 /*
  * wp_device_status — synchronises `stream`, then reads and clears the device
  * status word of the current device. Returns WP_OK, WP_ERR_TIMEOUT (a kernel
- * gave up waiting since the last call) or WP_ERR_CUDA.
+ * gave up waiting since the last call), WP_ERR_ARG (a packed prefill met
+ * out-of-range cu_seqlens) or WP_ERR_CUDA.
  */
 int wp_device_status(void *stream);
 

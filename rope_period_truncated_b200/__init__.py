@@ -73,6 +73,8 @@ def load_library():
     lib.wp_schedule.argtypes = [I, I, I, P, I, P, P]
     lib.wp_prefill.restype = I
     lib.wp_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, F, P]
+    lib.wp_prefill_ex.restype = I
+    lib.wp_prefill_ex.argtypes = [P, P, P, P, P, P, I, I, ctypes.c_int64, I, I, I, I, P, I, I, F, P]
     lib.wp_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.wp_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.wp_decode.restype = I
@@ -195,29 +197,60 @@ def wp_rope_apply(x: torch.Tensor, theta: float, layout: int, pos: torch.Tensor 
 
 def wp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cut=None, mode: int = MODE_GROUPED,
                layout: int = ROPE_HALF_SPLIT, softmax_scale: float = 0.0, out: torch.Tensor | None = None,
-               lse: torch.Tensor | None = None, want_lse: bool = True, stream=None):
-    """Causal WavePrune prefill. q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 (rotated).
-    ``cut``: host group cutoffs [d/16] (grouped) or channel cutoffs [d/2]
-    (channel mode), None = dense. Returns (o [B,N,Hq,d] bf16, lse [B,Hq,N] fp32)."""
-    _need(q, "q", torch.bfloat16, 4)
-    _need(k, "k", torch.bfloat16, 4)
-    _need(v, "v", torch.bfloat16, 4)
-    B, N, Hq, d = q.shape
-    Hkv = k.shape[2]
-    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
-        raise ValueError("k/v shape mismatch")
+               lse: torch.Tensor | None = None, want_lse: bool = True, stream=None,
+               cu_seqlens: torch.Tensor | None = None, max_seqlen: int | None = None):
+    """Causal WavePrune prefill (wp_prefill_ex).
+
+    Uniform batch: q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16 (rotated); returns
+    (o [B,N,Hq,d] bf16, lse [B,Hq,N] fp32). Packed batch: q [T,Hq,d], k/v
+    [T,Hkv,d] with ``cu_seqlens`` (device int32 [B+1]) and ``max_seqlen`` (an
+    upper bound of the lengths); returns (o [T,Hq,d], lse [Hq,T]).
+    ``cut``: host cutoffs, one row [d/16] (grouped) or [d/2] (channel mode)
+    for every head, or one row per query head [Hq, n]; None = dense."""
+    packed = cu_seqlens is not None
+    nd = 3 if packed else 4
+    _need(q, "q", torch.bfloat16, nd)
+    _need(k, "k", torch.bfloat16, nd)
+    _need(v, "v", torch.bfloat16, nd)
+    if packed:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        T, Hq, d = q.shape
+        B = cu_seqlens.numel() - 1
+        if B < 1 or max_seqlen is None or int(max_seqlen) < 1:
+            raise ValueError("a packed batch needs cu_seqlens [B+1] and max_seqlen >= 1")
+        N = int(max_seqlen)
+        Hkv = k.shape[1]
+        if tuple(k.shape) != (T, Hkv, d) or tuple(v.shape) != (T, Hkv, d):
+            raise ValueError("k/v shape mismatch")
+        lse_shape = (Hq, T)
+    else:
+        B, N, Hq, d = q.shape
+        T = B * N
+        Hkv = k.shape[2]
+        if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
+            raise ValueError("k/v shape mismatch")
+        lse_shape = (B, Hq, N)
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", torch.bfloat16, 4)
+    _need(out, "out", torch.bfloat16, nd)
     if lse is None and want_lse:
-        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
     if lse is not None:
-        _need(lse, "lse", torch.float32, 3)
+        _need(lse, "lse", torch.float32, len(lse_shape))
     n_expected = d // 16 if mode == MODE_GROUPED else d // 2
-    cut_a, cut_p = _host_i32(cut, n_expected)
-    _check("wp_prefill", load_library().wp_prefill(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, N, Hq, Hkv, d, int(mode), cut_p, int(layout),
-        float(softmax_scale), _stream(stream)))
+    cut_rows = 1
+    if cut is not None:
+        arr = np.asarray(cut)
+        if arr.ndim == 2:
+            if arr.shape != (Hq, n_expected):
+                raise ValueError(f"per-head cutoffs must be [{Hq}, {n_expected}], got {arr.shape}")
+            cut_rows = Hq
+        cut_a, cut_p = _host_i32(arr.reshape(-1), cut_rows * n_expected)
+    else:
+        cut_a, cut_p = None, None
+    _check("wp_prefill", load_library().wp_prefill_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens), B, N, T, Hq, Hkv, d, int(mode), cut_p,
+        cut_rows, int(layout), float(softmax_scale), _stream(stream)))
     return out, lse
 
 

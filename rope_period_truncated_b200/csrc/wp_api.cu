@@ -174,20 +174,30 @@ int wp_rope_apply(const void *x, void *y, int B, int N, int H, int d_h, const in
   return from_cuda(launch_rope(a, d_h, layout, static_cast<cudaStream_t>(stream)));
 }
 
-int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int N, int H_q, int H_kv,
-               int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream) {
+int wp_prefill_ex(const void *q, const void *k, const void *v, void *o, float *lse, const int32_t *cu_seqlens,
+                  int B, int N, int64_t total_tokens, int H_q, int H_kv, int d_h, int mode, const int32_t *cut,
+                  int cut_rows, int layout, float softmax_scale, void *stream) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return WP_ERR_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return WP_ERR_ARG;
   if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return WP_ERR_ARG;
+  if (cu_seqlens != nullptr && ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0 || total_tokens <= 0))
+    return WP_ERR_ARG;
   if (B > 65535 || H_q > 65535) return WP_ERR_UNSUPPORTED;
   if (mode != WP_MODE_GROUPED && mode != WP_MODE_CHANNEL) return WP_ERR_ARG;
   if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
   if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
   if (!std::isfinite(softmax_scale)) return WP_ERR_ARG;
+  if (cut_rows != 1 && cut_rows != H_q) return WP_ERR_ARG;
+  if (cut_rows != 1 && cut == nullptr) return WP_ERR_ARG;
+  // the packed view is [T, H, d]: row coordinates of the tensor maps are int32
+  if (cu_seqlens != nullptr && total_tokens > (1ll << 31) - 256) return WP_ERR_UNSUPPORTED;
+  const int per_row = mode == WP_MODE_GROUPED ? d_h / 16 : d_h / 2;
+  if (static_cast<int64_t>(cut_rows) * per_row > PREFILL_CUT_CAP) return WP_ERR_UNSUPPORTED;
   const float scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(d_h)));
   const float scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t T = cu_seqlens != nullptr ? total_tokens : static_cast<int64_t>(B) * N;
 
   if (mode == WP_MODE_CHANNEL) {
     ChannelPrefillArgs a;
@@ -196,41 +206,63 @@ int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
     a.v = static_cast<const __nv_bfloat16 *>(v);
     a.o = static_cast<__nv_bfloat16 *>(o);
     a.lse = lse;
+    a.cu_seqlens = cu_seqlens;
     a.B = B;
     a.N = N;
+    a.T = T;
     a.Hq = H_q;
     a.Hkv = H_kv;
     a.layout = layout;
-    for (int c = 0; c < 64; ++c) {
-      a.cut[c] = (cut == nullptr || c >= d_h / 2) ? WP_CUTOFF_INF : cut[c];
-      if (a.cut[c] < 0) return WP_ERR_ARG;
+    a.cut_rows = cut_rows;
+    for (int e = 0; e < cut_rows * per_row; ++e) {
+      a.cut[e] = cut == nullptr ? WP_CUTOFF_INF : cut[e];
+      if (a.cut[e] < 0) return WP_ERR_ARG;
     }
     a.scale_log2 = scale_log2;
     return from_cuda(launch_prefill_channel(d_h, a, s));
   }
 
-  PrefillArgs a;
-  a.o = static_cast<__nv_bfloat16 *>(o);
-  a.lse = lse;
-  a.B = B;
-  a.N = N;
-  a.Hq = H_q;
-  a.Hkv = H_kv;
-  for (int g = 0; g < 8; ++g) {
-    a.cut[g] = (cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : cut[g];
-    if (a.cut[g] < 0) return WP_ERR_ARG;
-  }
-  a.scale_log2 = scale_log2;
-  a.wait_limit = g_wait_limit;
   if ((N + 127) / 128 > 65535 || static_cast<int64_t>(H_kv) * B > 65535) return WP_ERR_UNSUPPORTED;
   // the kernel keeps one key-block table per CTA in shared memory: 2^20 tokens fit at every d_h
   if (N > (1 << 20)) return WP_ERR_UNSUPPORTED;
+  // with one table per head, two tables share that space: 2^19 tokens
+  if (cut_rows != 1 && N > (1 << 19)) return WP_ERR_UNSUPPORTED;
+  PrefillArgs a;
+  a.o = static_cast<__nv_bfloat16 *>(o);
+  a.lse = lse;
+  a.cu_seqlens = cu_seqlens;
+  a.B = B;
+  a.N = N;
+  a.T = T;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  a.cut_rows = cut_rows;
+  for (int g = 0; g < 8; ++g) a.cut[g] = WP_CUTOFF_INF;
+  HeadCuts hc;
+  for (int e = 0; e < cut_rows * per_row; ++e) {
+    const int32_t w = cut == nullptr ? WP_CUTOFF_INF : cut[e];
+    if (w < 0) return WP_ERR_ARG;
+    if (cut_rows == 1)
+      a.cut[e] = w;
+    else
+      hc.cut[e] = w;
+  }
+  a.scale_log2 = scale_log2;
+  a.wait_limit = g_wait_limit;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, B, N, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !make_map(&tk, k, B, N, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-      !make_map(&tv, v, B, N, H_kv, d_h, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+  const int mB = cu_seqlens != nullptr ? 1 : B;
+  const int mN = cu_seqlens != nullptr ? static_cast<int>(total_tokens) : N;
+  if (!make_map(&tq, q, mB, mN, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map(&tk, k, mB, mN, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map(&tv, v, mB, mN, H_kv, d_h, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return WP_ERR_CUDA;
-  return from_cuda(launch_prefill_grouped(d_h, tq, tk, tv, a, s));
+  return from_cuda(launch_prefill_grouped(d_h, tq, tk, tv, a, cut_rows == 1 ? nullptr : &hc, s));
+}
+
+int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse, int B, int N, int H_q, int H_kv,
+               int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream) {
+  return wp_prefill_ex(q, k, v, o, lse, nullptr, B, N, 0, H_q, H_kv, d_h, mode, cut, 1, layout, softmax_scale,
+                       stream);
 }
 
 size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {

@@ -10,11 +10,12 @@
 // KV head (GQA), so every K/V tile it loads feeds both, and visits the key
 // tiles from the diagonal backwards. Each 128-key tile is handled as two
 // 64-key sub-tiles u = 2t + h; §2.3's skip / full / boundary class of
-// every (sub-tile, group) is the same for both heads and comes from a
-// per-CTA table built once in shared memory.
+// every (sub-tile, group) comes from a per-CTA table built once in shared
+// memory (one table for both heads, or one per head when each query head has
+// its own cutoff table).
 //   warp 8   TMA producer: Q of both heads once (one 16-dim box per group);
 //            per key tile only the K column slices of groups either half
-//            computes (16-dim boxes, 32-byte swizzle) and all of V (64-dim
+//            (of either head) computes (16-dim boxes, 32-byte swizzle) and all of V (64-dim
 //            boxes, 128-byte swizzle); two stages each.
 //   warp 9+s MMA issuer of head s (one elected lane, warp-uniform loop). S of
 //            a head is double-buffered: two 64-column halves of TMEM, half h
@@ -45,10 +46,17 @@
 // packed f32x2 arithmetic: Cody-Waite reduction x = j + f, |f| <= 1/2, and a
 // degree-3 minimax polynomial for 2^f (coefficients from a Remez fit, max
 // relative error 7.5e-5, far below bf16's 2^-9 for P), scaled by 2^j in the
-// exponent field.
+// exponent field. The diagonal tile takes every exponential on MUFU, so its
+// causally masked entries give exactly 0.
+//
+// Packed (varlen) batches: sequence b occupies rows cu_seqlens[b] ..
+// cu_seqlens[b+1]-1 of [T, H, d]; positions restart at 0 in every sequence.
+// A tile that runs past the sequence's end loads the next rows of the buffer,
+// which only the diagonal tile's causal mask ever sees (P exactly 0).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "wp_device.cuh"
 #include "wp_prefill.h"
@@ -96,8 +104,12 @@ struct Layout {
   // o_ready/o_final/bnd_ready/bnd_done, drain
   static constexpr uint32_t NUM_BARS = 1 + 2 * KST + 2 * VST + 2 * 4 + 2 * 4 + 2;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t TT_OFF = MISC_OFF + 16;  // sub-tile table: one uint16 per 64-key sub-tile
-  static uint32_t bytes(int nqb) { return TT_OFF + ((4u * nqb + 15u) & ~15u) + 1024u; }  // + alignment slack
+  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // cutoff rows of head slot 0 and 1: 2 x 8 int32
+  static constexpr uint32_t TT_OFF = CUT_OFF + 64;    // sub-tile tables: one uint16 per 64-key sub-tile
+  // One table per head slot when the two heads have their own cutoffs, one
+  // shared table otherwise.
+  static uint32_t table_bytes(int nqb, bool per_head) { return ((4u * nqb + 15u) & ~15u) * (per_head ? 2u : 1u); }
+  static uint32_t bytes(int nqb, bool per_head) { return TT_OFF + table_bytes(nqb, per_head) + 1024u; }  // + align
 };
 
 struct Barriers {
@@ -107,12 +119,22 @@ struct Barriers {
 
 // Class masks of the 128-query x 64-key block (qb, kb64): bits 0-7 full
 // groups, bits 8-15 boundary groups.
-__device__ __forceinline__ uint32_t sub_masks(const PrefillArgs &a, int G, int64_t qb, int64_t kb64) {
+// The per-head cutoff parameter of a kernel instantiation: the table, or a
+// placeholder when every head shares the table in PrefillArgs.
+struct NoHeadCuts {
+  int32_t unused;
+};
+template <bool PER_HEAD>
+using HeadCutsArg = typename std::conditional<PER_HEAD, HeadCuts, NoHeadCuts>::type;
+
+// Class masks of the 128-query x 64-key block (qb, kb64) under the cutoff
+// row `cut` (shared memory): bits 0-7 full groups, bits 8-15 boundary groups.
+__device__ __forceinline__ uint32_t sub_masks(const int32_t *cut, int G, int64_t N, int64_t qb, int64_t kb64) {
   int64_t dmin = 0, dmax = -1;
   uint32_t full = 0, bnd = 0;
-  if (tile_distance_range(a.N, BM, SUB, qb, kb64, &dmin, &dmax)) {
+  if (tile_distance_range(N, BM, SUB, qb, kb64, &dmin, &dmax)) {
     for (int g = 0; g < G; ++g) {
-      const int c = classify_cutoff(dmin, dmax, a.cut[g]);
+      const int c = classify_cutoff(dmin, dmax, cut[g]);
       if (c == TILE_FULL) full |= 1u << g;
       if (c == TILE_BOUNDARY) bnd |= 1u << g;
     }
@@ -123,18 +145,18 @@ __device__ __forceinline__ uint32_t sub_masks(const PrefillArgs &a, int G, int64
 // Smallest cutoff among the boundary groups in `bnd` that is > prev
 // (prev = -1 for the first); returns false when there is none. `mask` gets
 // the groups sharing that cutoff.
-__device__ __forceinline__ bool next_boundary_class(const PrefillArgs &a, uint32_t bnd, int64_t prev,
-                                                    int32_t *W, uint32_t *mask) {
+__device__ __forceinline__ bool next_boundary_class(const int32_t *cut, uint32_t bnd, int64_t prev, int32_t *W,
+                                                    uint32_t *mask) {
   int64_t best = INT64_MAX;
   for (uint32_t m = bnd; m; m &= m - 1) {
-    const int64_t w = a.cut[__ffs(m) - 1];
+    const int64_t w = cut[__ffs(m) - 1];
     if (w > prev && w < best) best = w;
   }
   if (best == INT64_MAX) return false;
   uint32_t mk = 0;
   for (uint32_t m = bnd; m; m &= m - 1) {
     const int g = __ffs(m) - 1;
-    if (static_cast<int64_t>(a.cut[g]) == best) mk |= 1u << g;
+    if (static_cast<int64_t>(cut[g]) == best) mk |= 1u << g;
   }
   *W = static_cast<int32_t>(best);
   *mask = mk;
@@ -255,6 +277,7 @@ __device__ __forceinline__ float half_max(const uint32_t (&su)[64]) {
 // pairs take the polynomial exp2, the rest the MUFU unit. Adds the p to the
 // four packed partial sums and writes them as bf16 pairs (32 TMEM columns)
 // to p_addr.
+template <bool USE_POLY>
 __device__ __forceinline__ void exp_half(const uint32_t (&su)[64], uint64_t c2x2, float m, uint64_t (&acc)[4],
                                          uint32_t p_addr) {
   const uint64_t negm = pack_f2(-m, -m);
@@ -265,7 +288,7 @@ __device__ __forceinline__ void exp_half(const uint32_t (&su)[64], uint64_t c2x2
     float x0, x1;
     unpack_f2(x2, x0, x1);
     float p0, p1;
-    if ((k & 7) >= 8 - POLY_PAIRS) {
+    if (USE_POLY && (k & 7) >= 8 - POLY_PAIRS) {
       poly_exp2x2(x2, p0, p1);
     } else {
       p0 = fast_exp2(x0);
@@ -291,10 +314,14 @@ __device__ __forceinline__ void scale_cols_f32(uint32_t taddr, int n32, float al
   tmem_wait_st();
 }
 
-template <int D>
+// PACKED: sequences located by cu_seqlens (else a uniform batch); PER_HEAD:
+// one cutoff row per query head (else one row for all). Both are template
+// parameters so that the plain case carries none of their bookkeeping.
+template <int D, bool PACKED, bool PER_HEAD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_grouped_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
+                           const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a,
+                           const HeadCutsArg<PER_HEAD> hc) {
   using L = Layout<D>;
   constexpr int G = L::G;
   constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, SUB, false, false);
@@ -318,7 +345,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   B.drain = B.bnd_done + 2;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
-  uint16_t *ttab = reinterpret_cast<uint16_t *>(smem + L::TT_OFF);
+  // Sub-tile class tables of head slot 0 and 1 (the same table unless the
+  // heads have their own cutoffs).
+  uint16_t *ttab0 = reinterpret_cast<uint16_t *>(smem + L::TT_OFF);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -332,6 +361,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int h0 = hk * rep + static_cast<int>(blockIdx.x) * nslot;  // head of slot s = h0 + s
   const int nqb = (a.N + BM - 1) / BM;
   const int qb = nqb - 1 - static_cast<int>(blockIdx.y);
+  // The sequence: batch entry b of a uniform batch (length a.N, coordinate b
+  // of the 4-D tensor view) or rows [row0, row0 + N) of a packed one.
+  int64_t N = a.N, row0 = 0;
+  if constexpr (PACKED) {
+    row0 = a.cu_seqlens[b];
+    const int64_t row1 = a.cu_seqlens[b + 1];
+    if (row0 < 0 || row1 < row0 || row1 > a.T || row1 - row0 > a.N) {
+      // Offsets out of range: nothing of this sequence can be located.
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && hk == 0) record_status(WP_ERR_ARG);
+      return;
+    }
+    N = row1 - row0;
+    if (static_cast<int64_t>(qb) * BM >= N) return;  // past this sequence's end (whole CTA)
+  }
+  // TMA row coordinate of query / key block x and the batch coordinate
+  const auto block_row = [&](int x) { return PACKED ? static_cast<int>(row0 + static_cast<int64_t>(x) * BM) : x * BM; };
+  const int bcoord = PACKED ? 0 : b;
+  // the cutoff rows of head slot 0 and 1, copied into shared memory below
+  int32_t *cut0 = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);
+  int32_t *cut1 = PER_HEAD ? cut0 + 8 : cut0;
+  uint16_t *ttab1 = PER_HEAD ? ttab0 + ((2 * qb + 2 + 7) & ~7) : ttab0;
   const long long lim = a.wait_limit;
 
   if (threadIdx.x == 0) {
@@ -361,10 +411,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&B.drain[1], 1);
     fence_barrier_init();
   }
+  if (threadIdx.x == 0) {  // the cutoff rows of both head slots (constant indices into the parameters)
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if constexpr (PER_HEAD) {
+        cut0[g] = g < G ? hc.cut[h0 * G + g] : WP_CUTOFF_INF;
+        cut0[8 + g] = g < G ? hc.cut[(h0 + nslot - 1) * G + g] : WP_CUTOFF_INF;
+      } else {
+        cut0[g] = a.cut[g];
+      }
+    }
+  }
+  __syncthreads();
   // Sub-tile table: sub-tile u = 2t + h holds the keys of 64-key block
   // 2(qb - t) + h, i.e. half h of key tile t.
-  for (int u = threadIdx.x; u < 2 * (qb + 1); u += NTHREADS)
-    ttab[u] = static_cast<uint16_t>(sub_masks(a, G, qb, 2 * (qb - u / 2) + (u & 1)));
+  for (int u = threadIdx.x; u < 2 * (qb + 1); u += NTHREADS) {
+    const int64_t kb64 = 2 * (qb - u / 2) + (u & 1);
+    ttab0[u] = static_cast<uint16_t>(sub_masks(cut0, G, N, qb, kb64));
+    if (PER_HEAD) ttab1[u] = static_cast<uint16_t>(sub_masks(cut1, G, N, qb, kb64));
+  }
   if (warp == MMA_WARP) {
     tmem_alloc(tmem_base_slot, TMEM_COLS);
     tmem_relinquish();
@@ -381,6 +446,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // The whole warp runs the loop (warp-uniform waits); one elected lane
     // issues each bulk copy.
     const bool leader = elect_one();
+    const int qrow = block_row(qb);
     if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -388,8 +454,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_arrive_expect_tx(B.q_full, nslot * G * GROUP_TILE_BYTES);
       for (int s = 0; s < nslot; ++s)
         for (int g = 0; g < G; ++g)
-          tma_load_4d(smem + L::Q_OFF + s * L::Q_SLOT + g * GROUP_TILE_BYTES, &tm_q, B.q_full, 16 * g, h0 + s,
-                      qb * BM, b);
+          tma_load_4d(smem + L::Q_OFF + s * L::Q_SLOT + g * GROUP_TILE_BYTES, &tm_q, B.q_full, 16 * g, h0 + s, qrow,
+                      bcoord);
     }
     __syncwarp();
     int k_issued = 0, v_issued = 0;
@@ -397,12 +463,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto load_v = [&](int t) -> bool {
       const int st = t % VST;
       if (t >= VST && !warp_wait(&B.v_empty[st], ((t / VST) - 1) & 1, lim, abort_flag)) return false;
-      const int kb = qb - t;
+      const int krow = block_row(qb - t);
       if (leader) {
         mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * V_CHUNK_BYTES);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(smem + L::V_OFF + st * L::V_STAGE + c * V_CHUNK_BYTES, &tm_v, &B.v_full[st], 64 * c, hk,
-                      kb * BN, b);
+          tma_load_4d(smem + L::V_OFF + st * L::V_STAGE + c * V_CHUNK_BYTES, &tm_v, &B.v_full[st], 64 * c, hk, krow,
+                      bcoord);
       }
       __syncwarp();
       ++v_issued;
@@ -414,15 +480,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ok = false;
         break;
       }
-      const int kb = qb - t;
-      const uint32_t m0 = ttab[2 * t], m1 = ttab[2 * t + 1];
-      const uint32_t need = (m0 | (m0 >> 8) | m1 | (m1 >> 8)) & 0xffu;  // groups either half computes
+      const int krow = block_row(qb - t);
+      // groups either half of the tile computes, for either head
+      const uint32_t m =
+          ttab0[2 * t] | ttab0[2 * t + 1] | (PER_HEAD && nslot == 2 ? ttab1[2 * t] | ttab1[2 * t + 1] : 0u);
+      const uint32_t need = (m | (m >> 8)) & 0xffu;
       if (leader) {
         mbar_arrive_expect_tx(&B.k_full[st], __popc(need) * GROUP_TILE_BYTES);
-        for (uint32_t m = need; m; m &= m - 1) {
-          const int g = __ffs(m) - 1;
-          tma_load_4d(smem + L::K_OFF + st * L::K_STAGE + g * GROUP_TILE_BYTES, &tm_k, &B.k_full[st], 16 * g,
-                      hk, kb * BN, b);
+        for (uint32_t mm = need; mm; mm &= mm - 1) {
+          const int g = __ffs(mm) - 1;
+          tma_load_4d(smem + L::K_OFF + st * L::K_STAGE + g * GROUP_TILE_BYTES, &tm_k, &B.k_full[st], 16 * g, hk,
+                      krow, bcoord);
         }
       }
       __syncwarp();
@@ -473,6 +541,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
     };
     // QK of this head for sub-tile u into S half u & 1 (its K stage loaded).
+    const uint16_t *ttab = s == 0 ? ttab0 : ttab1;
+    const int32_t *cut = s == 0 ? cut0 : cut1;
     auto issue_qk = [&](int u) -> bool {
       const uint32_t tm = ttab[u];
       const int t = u >> 1, hh = u & 1;
@@ -487,7 +557,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(a, bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, bnd, prev, &W, &cls)) {
           if (leader) {
             issue_groups(s_col, qs_desc, kst_desc, cls, acc);
             umma_commit(&B.bnd_ready[s]);
@@ -579,7 +649,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int q4 = warp % 4;
     const int r = q4 * 32 + lane;  // row of the query tile == TMEM lane
     const int h = h0 + slot;
-    const int64_t i = static_cast<int64_t>(qb) * BM + r;
+    const uint16_t *ttab = slot == 0 ? ttab0 : ttab1;
+    const int32_t *cut = slot == 0 ? cut0 : cut1;
+    const int64_t i = static_cast<int64_t>(qb) * BM + r;  // position in the sequence
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const uint32_t o_addr = lane_addr + col_o(slot);
     const float c2 = a.scale_log2;  // logits to base-2 exponent units
@@ -600,7 +672,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(a, bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, bnd, prev, &W, &cls)) {
           ok = warp_wait(&B.bnd_ready[slot], bnd_cnt & 1, lim, abort_flag);
           if (!ok) break;
           tc_fence_after();
@@ -649,7 +721,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       const uint64_t zero2 = 0ull;
       uint64_t acc[4] = {zero2, zero2, zero2, zero2};
-      exp_half(su, c2x2, m_run, acc, s_addr);  // P: the sub-tile's first 32 columns
+      // P: the sub-tile's first 32 columns. In a packed batch the diagonal
+      // tile takes every exponential on MUFU, so its causally masked entries
+      // (possibly the next sequence's keys) give exactly 0.
+      if (PACKED && t == 0)
+        exp_half<false>(su, c2x2, m_run, acc, s_addr);
+      else
+        exp_half<true>(su, c2x2, m_run, acc, s_addr);
       float s0, s1, s2, s3, s4, s5, s6, s7;
       unpack_f2(acc[0], s0, s1);
       unpack_f2(acc[1], s2, s3);
@@ -661,12 +739,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       __syncwarp();  // the warp's TMEM stores are ordered before lane 0's arrival
       if (lane == 0) mbar_arrive(&B.p_ready[2 * slot + hh]);
     }
+    __nv_bfloat16 *orow = a.o + (((PACKED ? row0 : static_cast<int64_t>(b) * a.N) + i) * a.Hq + h) * D;
+    float *lse_at = a.lse == nullptr
+                        ? nullptr
+                        : a.lse + (PACKED ? static_cast<int64_t>(h) * a.T + row0 + i
+                                                           : (static_cast<int64_t>(b) * a.Hq + h) * a.N + i);
     // o_ready may trail by two phases here (the last two PVs can both be in
     // flight), so the end of the last PV has a barrier of its own.
     if (ok && nsub > 0 && warp_wait(&B.o_final[slot], 0, lim, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
-      __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t u32[32];
@@ -677,25 +759,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int k = 0; k < 16; ++k)
           pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * inv_l, __uint_as_float(u32[2 * k + 1]) * inv_l);
-        if (i < a.N) {
+        if (i < N) {
           uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c4);
 #pragma unroll
           for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
         }
       }
-      if (i < a.N && a.lse != nullptr)
-        a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+      if (i < N && lse_at != nullptr) *lse_at = (m_run + log2f(l_run)) * 0.69314718055994531f;
     } else {
       // Tell the other roles to stop waiting for this warp's progress, and
       // never leave the caller's buffers with stale rows: an aborted CTA
       // writes NaN to its O rows and LSE entries.
       *abort_flag = 1;
-      if (i < a.N) {
-        __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+      if (i < N) {
         const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
 #pragma unroll
         for (int k = 0; k < D / 8; ++k) reinterpret_cast<uint4 *>(orow)[k] = nan4;
-        if (a.lse != nullptr) a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = __int_as_float(0x7FC00000);
+        if (lse_at != nullptr) *lse_at = __int_as_float(0x7FC00000);
       }
     }
   }
@@ -710,26 +790,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 }  // namespace
 
-template <int D>
+template <int D, bool PACKED, bool PER_HEAD>
 static cudaError_t launch_grouped(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                  const PrefillArgs &a, cudaStream_t stream) {
+                                  const PrefillArgs &a, const HeadCuts *head_cuts, cudaStream_t stream) {
   const int nqb = (a.N + BM - 1) / BM;
-  const uint32_t smem = Layout<D>::bytes(nqb);
+  const uint32_t smem = Layout<D>::bytes(nqb, a.cut_rows != 1);
   if (smem > 232448u) return cudaErrorInvalidValue;  // beyond 227 KB: N too large for the tile table
-  cudaError_t e = cudaFuncSetAttribute(prefill_grouped_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_grouped_kernel<D, PACKED, PER_HEAD>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int rep = a.Hq / a.Hkv;
   const int nslot = (rep % 2 == 0) ? 2 : 1;
   dim3 grid(rep / nslot, nqb, a.Hkv * a.B);
-  prefill_grouped_kernel<D><<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+  HeadCutsArg<PER_HEAD> hc;
+  if constexpr (PER_HEAD)
+    hc = *head_cuts;
+  else
+    hc.unused = 0;
+  prefill_grouped_kernel<D, PACKED, PER_HEAD><<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, a, hc);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_grouped(int d_h, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                                   const PrefillArgs &a, cudaStream_t stream) {
-  if (d_h == 128) return launch_grouped<128>(tq, tk, tv, a, stream);
-  return launch_grouped<64>(tq, tk, tv, a, stream);
+                                   const PrefillArgs &a, const HeadCuts *head_cuts, cudaStream_t stream) {
+  const bool packed = a.cu_seqlens != nullptr, per_head = head_cuts != nullptr;
+  if (d_h == 128) {
+    if (packed) return per_head ? launch_grouped<128, true, true>(tq, tk, tv, a, head_cuts, stream)
+                                : launch_grouped<128, true, false>(tq, tk, tv, a, head_cuts, stream);
+    return per_head ? launch_grouped<128, false, true>(tq, tk, tv, a, head_cuts, stream)
+                    : launch_grouped<128, false, false>(tq, tk, tv, a, head_cuts, stream);
+  }
+  if (packed) return per_head ? launch_grouped<64, true, true>(tq, tk, tv, a, head_cuts, stream)
+                              : launch_grouped<64, true, false>(tq, tk, tv, a, head_cuts, stream);
+  return per_head ? launch_grouped<64, false, true>(tq, tk, tv, a, head_cuts, stream)
+                  : launch_grouped<64, false, false>(tq, tk, tv, a, head_cuts, stream);
 }
 
 }  // namespace wp

@@ -22,7 +22,7 @@ namespace {
 constexpr int ROWS_PER_CTA = 4;
 
 template <int D>
-__global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(const ChannelPrefillArgs a) {
+__global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(const __grid_constant__ ChannelPrefillArgs a) {
   constexpr int C = D / 2;
   constexpr int PER_LANE = D / 32;
   __shared__ float q_s[ROWS_PER_CTA][D];
@@ -30,22 +30,37 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(cons
   const int64_t i = static_cast<int64_t>(blockIdx.x) * ROWS_PER_CTA + warp;
   const int h = blockIdx.y, b = blockIdx.z;
   const int hk = h / (a.Hq / a.Hkv);
-  if (i >= a.N) return;
+  // Rows of this sequence: [b*N, b*N + N) of a uniform batch, or
+  // [cu_seqlens[b], cu_seqlens[b+1]) of a packed one.
+  int64_t N = a.N, row0 = static_cast<int64_t>(b) * a.N;
+  if (a.cu_seqlens != nullptr) {
+    row0 = a.cu_seqlens[b];
+    const int64_t row1 = a.cu_seqlens[b + 1];
+    if (row0 < 0 || row1 < row0 || row1 > a.T || row1 - row0 > a.N) {
+      if (i == 0 && h == 0 && lane == 0) record_status(WP_ERR_ARG);
+      return;
+    }
+    N = row1 - row0;
+  }
+  if (i >= N) return;
+  const int32_t *cut = a.cut + (a.cut_rows == 1 ? 0 : h) * C;
+  __nv_bfloat16 *orow = a.o + ((row0 + i) * a.Hq + h) * D;
+  float *lse_at = a.lse == nullptr ? nullptr
+                                   : a.lse + (a.cu_seqlens != nullptr ? static_cast<int64_t>(h) * a.T + row0 + i
+                                                                      : (static_cast<int64_t>(b) * a.Hq + h) * a.N + i);
   if (*reinterpret_cast<volatile int *>(&g_status) != 0) {
     // A kernel of this library has given up since the status word was last
     // read: write NaN rows rather than leave stale outputs.
-    __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
     for (int t = lane; t < D; t += 32) orow[t] = __ushort_as_bfloat16(0x7FC0);
-    if (lane == 0 && a.lse != nullptr)
-      a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = __int_as_float(0x7FC00000);
+    if (lane == 0 && lse_at != nullptr) *lse_at = __int_as_float(0x7FC00000);
     return;
   }
-  const __nv_bfloat16 *qrow = a.q + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+  const __nv_bfloat16 *qrow = a.q + ((row0 + i) * a.Hq + h) * D;
   for (int t = lane; t < D; t += 32) q_s[warp][t] = __bfloat162float(qrow[t]);
   __syncwarp();
   const int64_t kstride = static_cast<int64_t>(a.Hkv) * D;
-  const __nv_bfloat16 *kbase = a.k + (static_cast<int64_t>(b) * a.N * a.Hkv + hk) * D;
-  const __nv_bfloat16 *vbase = a.v + (static_cast<int64_t>(b) * a.N * a.Hkv + hk) * D;
+  const __nv_bfloat16 *kbase = a.k + (row0 * a.Hkv + hk) * D;
+  const __nv_bfloat16 *vbase = a.v + (row0 * a.Hkv + hk) * D;
 
   float m_run = -INFINITY, l_run = 0.f;
   float o[PER_LANE];
@@ -60,7 +75,7 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(cons
       const int64_t dist = i - j;
       float acc = 0.f;
       for (int c = 0; c < C; ++c) {
-        if (dist > static_cast<int64_t>(a.cut[c])) continue;
+        if (dist > static_cast<int64_t>(cut[c])) continue;
         const int da = a.layout == WP_ROPE_INTERLEAVED ? 2 * c : c;
         const int db = a.layout == WP_ROPE_INTERLEAVED ? 2 * c + 1 : c + C;
         acc = fmaf(q_s[warp][da], __bfloat162float(krow[da]), acc);
@@ -89,12 +104,10 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) prefill_channel_kernel(cons
       for (int t = 0; t < PER_LANE; ++t) o[t] = fmaf(pk, __bfloat162float(vrow[lane + 32 * t]), o[t]);
     }
   }
-  __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
   const float inv_l = 1.f / l_run;
 #pragma unroll
   for (int t = 0; t < PER_LANE; ++t) orow[lane + 32 * t] = __float2bfloat16_rn(o[t] * inv_l);
-  if (lane == 0 && a.lse != nullptr)
-    a.lse[(static_cast<int64_t>(b) * a.Hq + h) * a.N + i] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+  if (lane == 0 && lse_at != nullptr) *lse_at = (m_run + log2f(l_run)) * 0.69314718055994531f;
 }
 
 }  // namespace

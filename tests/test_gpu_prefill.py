@@ -148,3 +148,129 @@ def test_dense_is_cutoff_infinity():
     o2, l2 = wp.wp_prefill(q, k, v, np.full(8, 2 ** 31 - 1, dtype=np.int32))
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _oracle_per_head(q, k, v, cut_rows, mode, layout):
+    """The oracle one query head at a time, each with its own cutoff row.
+    q [B,N,Hq,d], k/v [B,N,Hkv,d] (fp64 numpy); returns (o, lse) like attention."""
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N))
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        oh, lh = oracle.attention(q[:, :, h:h + 1], k[:, :, hk:hk + 1], v[:, :, hk:hk + 1], cut_rows[h], mode,
+                                  layout)
+        o[:, :, h:h + 1] = oh
+        lse[:, h] = lh[:, 0]
+    return o, lse
+
+
+def _per_head_table(Hq, d, theta, layout, mode, seed):
+    """Distinct cutoff rows per query head: the pages' table at several
+    period multiples alpha, and small random tables that put several
+    boundary cutoffs into one tile."""
+    rng = np.random.default_rng(seed)
+    n = d // 16 if mode == wp.MODE_GROUPED else d // 2
+    rows = []
+    for h in range(Hq):
+        if h % 3 == 2:
+            rows.append(rng.integers(0, 400, size=n).astype(np.int32))
+        else:
+            wc, wg = oracle.cutoffs(d, theta, layout, alpha=[2.0, 0.5, 8.0, 1.0][h % 4])
+            rows.append(wg if mode == wp.MODE_GROUPED else wc)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (6, 2), (4, 4)])
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_per_head_cutoff_tables(Hq, Hkv, mode):
+    """One cutoff row per query head ([H_q][G] or [H_q][C]); the two heads of
+    a GQA pair (or a single head when H_q/H_kv is odd) share K loads."""
+    N, d, theta, layout = 400, 128, 1e4, wp.ROPE_HALF_SPLIT
+    g = torch.Generator().manual_seed(200 + Hq + Hkv)
+    q = torch.randn(2, N, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(2, N, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(2, N, Hkv, d, generator=g).to(torch.bfloat16)
+    cut = _per_head_table(Hq, d, theta, layout, mode, seed=Hq)
+    o, lse = wp.wp_prefill(q.cuda(), k.cuda(), v.cuda(), cut, mode, layout)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    ro, rl = _oracle_per_head(widen(q), widen(k), widen(v), cut, mode, layout)
+    assert_attention_close(o, lse, ro, rl, f"per-head Hq={Hq} Hkv={Hkv} mode={mode}")
+
+
+VARLEN = [
+    # lengths, d, Hq, Hkv, layout
+    ([1, 127, 128, 129, 300, 513], 128, 4, 2, wp.ROPE_HALF_SPLIT),
+    ([200, 64, 1, 257], 64, 6, 2, wp.ROPE_INTERLEAVED),
+]
+
+
+@pytest.mark.parametrize("lens,d,Hq,Hkv,layout", VARLEN)
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+@pytest.mark.parametrize("per_head", [False, True])
+def test_packed_batch_of_ragged_sequences(lens, d, Hq, Hkv, layout, mode, per_head):
+    """Packed batch (cu_seqlens) of sequences of different lengths, none or
+    some multiples of the 128-row tile; positions restart in every sequence.
+    Every row of every sequence against the oracle run on that sequence."""
+    theta = 1e4
+    T = sum(lens)
+    g = torch.Generator().manual_seed(300 + T + d)
+    q = torch.randn(T, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(T, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(T, Hkv, d, generator=g).to(torch.bfloat16)
+    if per_head:
+        cut = _per_head_table(Hq, d, theta, layout, mode, seed=T)
+    else:
+        wc, wg = oracle.cutoffs(d, theta, layout)
+        cut = wg if mode == wp.MODE_GROUPED else wc
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+    o, lse = wp.wp_prefill(q.cuda(), k.cuda(), v.cuda(), cut, mode, layout, cu_seqlens=cu.cuda(),
+                           max_seqlen=max(lens))
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    assert tuple(o.shape) == (T, Hq, d) and tuple(lse.shape) == (Hq, T)
+    rows = cut if per_head else np.stack([cut] * Hq)
+    for b, (s0, s1) in enumerate(zip(cu[:-1].tolist(), cu[1:].tolist())):
+        qs, ks, vs = (widen(t[s0:s1]).reshape(1, s1 - s0, -1, d) for t in (q, k, v))
+        ro, rl = _oracle_per_head(qs, ks, vs, rows, mode, layout)
+        assert_attention_close(o[s0:s1].unsqueeze(0), lse[:, s0:s1].unsqueeze(0), ro, rl,
+                               f"seq {b} len {s1 - s0} mode={mode} per_head={per_head}")
+
+
+def test_packed_batch_of_equal_lengths_is_the_uniform_batch():
+    """A packed batch whose sequences all have length N gives the uniform
+    batch's results: only the tile coordinates differ, and the rounding of
+    the diagonal tile's exponentials (a packed batch takes them all on MUFU,
+    so that masked keys of the next sequence weigh exactly 0). A misplaced
+    row or tile would differ by O(1)."""
+    B, N, Hq, Hkv, d = 3, 333, 4, 2, 128
+    g = torch.Generator().manual_seed(17)
+    q = torch.randn(B, N, Hq, d, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(B, N, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(B, N, Hkv, d, generator=g).to(torch.bfloat16).cuda()
+    _, wg = oracle.cutoffs(d, 1e4, oracle.HALF_SPLIT)
+    o1, l1 = wp.wp_prefill(q, k, v, wg)
+    cu = torch.arange(0, B * N + 1, N, dtype=torch.int32, device="cuda")
+    o2, l2 = wp.wp_prefill(q.reshape(B * N, Hq, d), k.reshape(B * N, Hkv, d), v.reshape(B * N, Hkv, d), wg,
+                           cu_seqlens=cu, max_seqlen=N)
+    torch.cuda.synchronize()
+    assert (o1.reshape(B * N, Hq, d).float() - o2.float()).abs().max().item() <= 1e-2
+    assert (l1.permute(1, 0, 2).reshape(Hq, B * N) - l2).abs().max().item() <= 1e-4
+
+
+def test_packed_batch_bad_offsets_are_reported():
+    """Offsets that run backwards are not followed: the kernel records
+    WP_ERR_ARG in the status word (read and cleared by wp_device_status),
+    and a later correct call runs normally."""
+    T, Hq, Hkv, d = 400, 2, 2, 128
+    q = torch.randn(T, Hq, d, device="cuda").to(torch.bfloat16)
+    k = torch.randn(T, Hkv, d, device="cuda").to(torch.bfloat16)
+    cu_bad = torch.tensor([0, 300, 100, 400], dtype=torch.int32, device="cuda")
+    wp.wp_prefill(q, k, k, None, cu_seqlens=cu_bad, max_seqlen=300)
+    assert wp.wp_device_status() == wp.WP_ERR_ARG
+    cu = torch.tensor([0, 100, 400], dtype=torch.int32, device="cuda")
+    o, lse = wp.wp_prefill(q, k, k, None, cu_seqlens=cu, max_seqlen=300)
+    assert wp.wp_device_status() == wp.WP_OK
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
