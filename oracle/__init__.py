@@ -73,6 +73,8 @@ def _load():
                                            i32]
         lib.wpo_decode.restype = i32
         lib.wpo_decode.argtypes = [P, P, P, P, i64, i32, i32, i32, i64, P, f64, P, P, i32]
+        lib.wpo_attention_backward.restype = i32
+        lib.wpo_attention_backward.argtypes = [P, P, P, P, i64, i64, i32, i32, i32, i32, i32, P, f64, P, P, P, i32]
         lib.wpo_tile_classes.restype = i32
         lib.wpo_tile_classes.argtypes = [i64, i32, i32, P, i32, P, P]
         _lib = lib
@@ -178,6 +180,25 @@ def attention(q, k, v, cut, mode: int = MODE_GROUPED, layout: int = INTERLEAVED,
     rows = (bb.ravel(), hh.ravel(), tt.ravel())
     o, lse = attention_rows(q.reshape(-1, d), rows, k, v, Hq, cut, mode, layout, scale, nthreads)
     return o.reshape(B, N, Hq, d), lse.reshape(B, N, Hq).transpose(0, 2, 1).copy()
+
+
+def attention_backward(q, k, v, dout, cut, mode: int = MODE_GROUPED, layout: int = INTERLEAVED,
+                       scale: float | None = None, nthreads: int = 0):
+    """Gradients (dq, dk, dv) of sum(dout * O) for causal prefill, q/dout
+    [B,N,Hq,d], k/v [B,N,Hkv,d] (fp64). The chain rule through the forward
+    definition [RN §2.1 Eq. (6); §2.3 Eq. (8)]: masked units add 0 to the
+    gradients as they add 0 to the logit."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    scale = 1.0 / np.sqrt(d) if scale is None else scale
+    cut = np.ascontiguousarray(cut, dtype=np.int32)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _load().wpo_attention_backward(_p(q), _p(k), _p(v), _p(dout), B, N, Hq, Hkv, d, mode, layout, _p(cut),
+                                        scale, _p(dq), _p(dk), _p(dv), nthreads)
+    if rc:
+        raise ValueError(f"oracle backward: bad arguments (code {rc})")
+    return dq, dk, dv
 
 
 def decode(q, kc, vc, lens, group_cut, scale: float | None = None, nthreads: int = 0):

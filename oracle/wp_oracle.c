@@ -326,6 +326,121 @@ int wpo_decode(const double *q, const double *kc, const double *vc, const int32_
 }
 
 /* ------------------------------------------------------------------------- */
+/* Backward: gradients of the prefill definition                             */
+/* ------------------------------------------------------------------------- */
+
+/* [RN §2.3, the paragraph on the backward kernel; §4.6, Table 4] describes a
+ * backward kernel (gradient operands masked before the MMA, dQ and dK formed
+ * together under one mask) but prints no equations. The oracle therefore
+ * differentiates the forward definition itself, by the chain rule, one step
+ * per line of the forward pass:
+ *   forward   L_ij = scale * sum_u 1[i - j <= W_u] <q_i[u], k_j[u]>  (j <= i)
+ *             P_ij = exp(L_ij - LSE_i),   O_i = sum_j P_ij v_j
+ *   backward  dV_j += P_ij dO_i
+ *             dP_ij = <dO_i, v_j>
+ *             dL_ij = P_ij (dP_ij - D_i),   D_i = sum_j P_ij dP_ij = <dO_i, O_i>
+ *             dq_i[u] += scale * 1[i - j <= W_u] * dL_ij * k_j[u]
+ *             dk_j[u] += scale * 1[i - j <= W_u] * dL_ij * q_i[u]
+ * where u runs over channels (their two dims) in channel mode and over 16-dim
+ * groups in grouped mode. A masked unit contributes nothing to either
+ * gradient, exactly as it contributes 0 to the logit. */
+static void logit_grad(const double *q, const double *k, int64_t dist, int d_h, int mode, int layout,
+                       const int32_t *cut, double scale, double dl, double *dq, double *dk)
+{
+    double s = scale * dl;
+    if (mode == WPO_MODE_CHANNEL) {
+        int C = d_h / 2;
+        for (int c = 0; c < C; ++c) {
+            if (dist > (int64_t)cut[c])
+                continue;
+            int a, b;
+            channel_dims(c, d_h, layout, &a, &b);
+            dq[a] += s * k[a];
+            dq[b] += s * k[b];
+            dk[a] += s * q[a];
+            dk[b] += s * q[b];
+        }
+    } else {
+        int G = d_h / 16;
+        for (int g = 0; g < G; ++g) {
+            if (dist > (int64_t)cut[g])
+                continue;
+            for (int t = 16 * g; t < 16 * g + 16; ++t) {
+                dq[t] += s * k[t];
+                dk[t] += s * q[t];
+            }
+        }
+    }
+}
+
+/* Gradients of sum(dO * O) for causal prefill over positions 0..N-1.
+ * q, dout, dq: [B][N][Hq][d_h]; k, v, dk, dv: [B][N][Hkv][d_h]. The query
+ * heads sharing a KV head (GQA, h -> h / (Hq / Hkv)) add into its dk, dv.
+ * cut: channel cutoffs [d_h/2] (channel mode) or group cutoffs [d_h/16]. */
+int wpo_attention_backward(const double *q, const double *k, const double *v, const double *dout, int64_t B,
+                           int64_t N, int Hq, int Hkv, int d_h, int mode, int layout, const int32_t *cut,
+                           double scale, double *dq, double *dk, double *dv, int nthreads)
+{
+    if (Hkv <= 0 || Hq % Hkv != 0 || N <= 0 || B <= 0)
+        return 1;
+    int rep = Hq / Hkv;
+    int64_t qs = (int64_t)Hq * d_h, ks = (int64_t)Hkv * d_h;
+    for (int64_t e = 0; e < B * N * qs; ++e)
+        dq[e] = 0.0;
+    for (int64_t e = 0; e < B * N * ks; ++e)
+        dk[e] = dv[e] = 0.0;
+    int err = 0;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel
+    {
+        double *L = (double *)malloc(sizeof(double) * (size_t)N);
+        double *o = (double *)malloc(sizeof(double) * (size_t)d_h);
+        if (!L || !o) {
+#pragma omp atomic write
+            err = 2;
+        }
+        /* one thread per (b, KV head): it owns that head's dk, dv */
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bk = 0; bk < B * Hkv; ++bk) {
+            if (!L || !o)
+                continue;
+            int64_t b = bk / Hkv, hk = bk % Hkv;
+            const double *kb = k + (b * N * Hkv + hk) * d_h;
+            const double *vb = v + (b * N * Hkv + hk) * d_h;
+            double *dkb = dk + (b * N * Hkv + hk) * d_h;
+            double *dvb = dv + (b * N * Hkv + hk) * d_h;
+            for (int64_t h = hk * rep; h < (hk + 1) * rep; ++h)
+                for (int64_t i = 0; i < N; ++i) {
+                    const double *qi = q + ((b * N + i) * Hq + h) * d_h;
+                    const double *doi = dout + ((b * N + i) * Hq + h) * d_h;
+                    double *dqi = dq + ((b * N + i) * Hq + h) * d_h;
+                    double lse = attend_row(qi, kb, ks, vb, ks, i, d_h, mode, layout, cut, scale, L, o);
+                    double D = 0.0;
+                    for (int t = 0; t < d_h; ++t)
+                        D += doi[t] * o[t];
+                    for (int64_t j = 0; j <= i; ++j) {
+                        double p = exp(L[j] - lse);
+                        const double *vj = vb + j * ks;
+                        double dp = 0.0;
+                        for (int t = 0; t < d_h; ++t) {
+                            dp += doi[t] * vj[t];
+                            dvb[j * ks + t] += p * doi[t];
+                        }
+                        double dl = p * (dp - D);
+                        logit_grad(qi, kb + j * ks, i - j, d_h, mode, layout, cut, scale, dl, dqi, dkb + j * ks);
+                    }
+                }
+        }
+        free(L);
+        free(o);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Tile classes by brute force                                               */
 /* ------------------------------------------------------------------------- */
 

@@ -26,6 +26,13 @@ MUTANTS = {
     "tile skip rule": ("else if ((int64_t)cut[g] < lo)", "else if ((int64_t)cut[g] <= lo)"),
     "causal diagonal dropped": ("for (int64_t j = 0; j <= i; ++j) {\n        L[j]", "for (int64_t j = 0; j < i; ++j) {\n        L[j]"),
     "group width": ("for (int t = 16 * g; t < 16 * g + 16; ++t)", "for (int t = 16 * g; t < 16 * g + 15; ++t)"),
+    "backward: softmax correction dropped": ("double dl = p * (dp - D);", "double dl = p * dp;"),
+    "backward: dV without the weight": ("dvb[j * ks + t] += p * doi[t];", "dvb[j * ks + t] += doi[t];"),
+    "backward: dK from k": ("dk[t] += s * q[t];", "dk[t] += s * k[t];"),
+    "backward: dQ channel partner dim": ("dq[b] += s * k[b];", "dq[b] += s * k[a];"),
+    "backward: scale dropped": ("double s = scale * dl;", "double s = dl;"),
+    "backward: mask ignored": ("            if (dist > (int64_t)cut[g])\n                continue;\n            for (int t = 16 * g; t < 16 * g + 16; ++t) {\n                dq[t]",
+                               "            for (int t = 16 * g; t < 16 * g + 16; ++t) {\n                dq[t]"),
 }
 
 

@@ -425,3 +425,107 @@ def test_paired_order_is_the_half_split_model_in_channel_mode():
     wc_i, wg_i = oracle.cutoffs(d, 30.0, oracle.INTERLEAVED)
     assert np.array_equal(np.asarray(wc_i), np.asarray(wc))
     assert wg_i[0] == max(wc[:8]) and wg_i[1] == max(wc[8:])
+
+
+# --------------------------------------------------------------------------
+# Backward: gradients of the prefill definition
+# --------------------------------------------------------------------------
+
+def _bwd_case(seed, N=17, Hq=2, Hkv=1, d=32):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, N, Hq, d))
+    k = rng.standard_normal((1, N, Hkv, d))
+    v = rng.standard_normal((1, N, Hkv, d))
+    dout = rng.standard_normal((1, N, Hq, d))
+    return q, k, v, dout
+
+
+BWD_CASES = [
+    # mode, layout, cutoffs (small, so masks bite at distances < N)
+    (oracle.MODE_GROUPED, oracle.INTERLEAVED, [3, 9]),
+    (oracle.MODE_GROUPED, oracle.HALF_SPLIT, [0, 5]),
+    (oracle.MODE_CHANNEL, oracle.INTERLEAVED, [0, 1, 2, 3, 5, 7, 9, 12, 2, 4, 6, 8, 10, 11, 13, 20]),
+    (oracle.MODE_CHANNEL, oracle.HALF_SPLIT, [1, 3, 0, 6, 2, 8, 4, 11, 5, 7, 3, 9, 14, 2, 6, 10]),
+]
+
+
+@pytest.mark.parametrize("mode,layout,cut", BWD_CASES)
+def test_backward_central_differences(mode, layout, cut):
+    """Each gradient entry equals the central difference of the loss
+    sum(dout * O) computed with the oracle's forward pass (itself pinned to
+    SDPA, closed forms and invariants above): fp64, step 1e-6, on a random
+    subset of entries of q, k and v (GQA: two query heads per KV head)."""
+    cut = np.asarray(cut, dtype=np.int32)
+    q, k, v, dout = _bwd_case(7)
+    dq, dk, dv = oracle.attention_backward(q, k, v, dout, cut, mode, layout)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention(q_, k_, v_, cut, mode, layout)
+        return float((o * dout).sum())
+
+    rng = np.random.default_rng(1)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in zip(*[rng.integers(0, s, 25) for s in x.shape]):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - g[idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, g[idx])
+
+
+def _torch_wave_attention(q, k, v, cut, mode, layout):
+    """Independent torch statement of the forward rule: per-unit masked
+    logits summed, causal -inf, softmax, times V. q [N,Hq,d], k/v [N,Hkv,d]."""
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    rep = Hq // Hkv
+    kk = k.repeat_interleave(rep, dim=1)
+    vv = v.repeat_interleave(rep, dim=1)
+    dist = torch.arange(N)[:, None] - torch.arange(N)[None, :]
+    if mode == oracle.MODE_GROUPED:
+        units = [list(range(16 * g, 16 * g + 16)) for g in range(d // 16)]
+    elif layout == oracle.INTERLEAVED:
+        units = [[2 * c, 2 * c + 1] for c in range(d // 2)]
+    else:
+        units = [[c, c + d // 2] for c in range(d // 2)]
+    L = torch.zeros(Hq, N, N, dtype=q.dtype)
+    for u, dims in enumerate(units):
+        part = torch.einsum("ihe,jhe->hij", q[:, :, dims], kk[:, :, dims])
+        L = L + part * (dist <= int(cut[u])).to(q.dtype)
+    L = L / math.sqrt(d)
+    L = L.masked_fill(dist < 0, float("-inf"))
+    return torch.einsum("hij,jhe->ihe", torch.softmax(L, dim=-1), vv)
+
+
+@pytest.mark.parametrize("mode,layout,cut", BWD_CASES)
+def test_backward_matches_torch_autograd(mode, layout, cut):
+    """torch autograd through an independently written torch statement of the
+    same rule gives the oracle's gradients (fp64), including the sum over the
+    query heads that share a KV head."""
+    q, k, v, dout = _bwd_case(11, N=23, Hq=4, Hkv=2)
+    cut = np.asarray(cut, dtype=np.int32)
+    dq, dk, dv = oracle.attention_backward(q, k, v, dout, cut, mode, layout)
+    tq, tk, tv = (torch.tensor(x[0], requires_grad=True) for x in (q, k, v))
+    o = _torch_wave_attention(tq, tk, tv, cut, mode, layout)
+    (o * torch.tensor(dout[0])).sum().backward()
+    for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+        np.testing.assert_allclose(mine[0], ref.numpy(), rtol=0, atol=1e-10, err_msg=name)
+
+
+def test_backward_dense_is_sdpa_autograd():
+    """[RN §2.1]: alpha -> infinity (every cutoff >= N) is plain causal
+    attention, whose gradients torch's scaled_dot_product_attention gives."""
+    q, k, v, dout = _bwd_case(3, N=30, Hq=4, Hkv=2, d=64)
+    for mode, n in ((oracle.MODE_GROUPED, 4), (oracle.MODE_CHANNEL, 32)):
+        dq, dk, dv = oracle.attention_backward(q, k, v, dout, np.full(n, 2 ** 31 - 1, dtype=np.int32), mode,
+                                               oracle.INTERLEAVED)
+        tq, tk, tv = (torch.tensor(x[0].transpose(1, 0, 2), requires_grad=True) for x in (q, k, v))
+        o = torch.nn.functional.scaled_dot_product_attention(tq, tk.repeat_interleave(2, 0),
+                                                             tv.repeat_interleave(2, 0), is_causal=True)
+        (o * torch.tensor(dout[0].transpose(1, 0, 2))).sum().backward()
+        for name, mine, ref in (("dq", dq, tq.grad), ("dk", dk, tk.grad), ("dv", dv, tv.grad)):
+            np.testing.assert_allclose(mine[0], ref.numpy().transpose(1, 0, 2), rtol=0, atol=1e-10,
+                                       err_msg=f"{name} mode={mode}")
