@@ -55,6 +55,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-backward", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--kcache", choices=["group-major", "rows"], default="group-major",
                    help="layout of the decode K cache in HBM")
@@ -156,6 +157,19 @@ def prefill_flops(N, d, Hq, B, wg):
     pair_exact = float((pairs * (2 * 16 * active + 2 * d)).sum()) * B * Hq
     dense_tile = float(tiles * (2 * BM * BN * d * 2)) * B * Hq
     return tile_level, pair_exact, dense_tile
+
+
+def backward_flops(N, d, Hq, B, wg):
+    """Useful FLOPs of one prefill backward, pair exact: per pair j <= i the
+    three products over the in-window groups (S = Q K^T, dQ = dS K,
+    dK = dS^T Q: 2*16 each per group) and the two full ones (dP = dO V^T,
+    dV = P^T dO: 2*d each)."""
+    delta = np.arange(N, dtype=np.int64)
+    pairs = (N - delta).astype(np.float64)
+    active = (delta[:, None] <= np.asarray(wg, dtype=np.int64)[None, :]).sum(1)
+    useful = float((pairs * (3 * 2 * 16 * active + 2 * 2 * d)).sum()) * B * Hq
+    dense = float((pairs * (3 * 2 * d + 2 * 2 * d)).sum()) * B * Hq
+    return useful, dense
 
 
 def decode_required_bytes(lens, wg, B, Hq, Hkv, d):
@@ -570,6 +584,37 @@ def run_ours(args, rank, world, local):
                        "frac": round(rows_gbs / peaks["hbm_gbs"], 4), "kernel_ms": round(rows_ms, 5),
                        "required_bytes": dec_bytes}
 
+    # backward of the 32K prefill (wp_prefill_backward), wave and dense
+    backward = None
+    if args.only == "all" and not args.no_backward:
+        dout = torch.randn(path.o.shape, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).to(dev)
+        dq, dk, dv = torch.empty_like(path.qr), torch.empty_like(path.kr), torch.empty_like(path.v)
+        bw_useful, bw_dense = backward_flops(pw.N, pw.d, pw.Hq, pw.B, path.wg)
+        path.prefill()  # O and LSE of the wave forward for the backward's inputs
+        times = {}
+        for cut in ("wave", "dense", "wave", "dense"):
+            if cut == "dense":
+                path.prefill_only("dense")
+            else:
+                path.prefill_only("wave")
+            t = time_kernel(lambda: wp.wp_prefill_backward(path.qr, path.kr, path.v, path.o, path.lse, dout,
+                                                           path.wg if cut == "wave" else None, dq=dq, dk=dk,
+                                                           dv=dv), 2, 1)
+            times.setdefault(cut, []).append(t)
+        wave_ms, dense_ms = min(times["wave"]), min(times["dense"])
+        wave_ms, dense_ms = max_over_ranks([wave_ms, dense_ms], dev)
+        backward = {"kernel": "wp_prefill_backward (delta + dQ + dK/dV, warp-level mma.sync)",
+                    "ms": round(wave_ms, 3), "dense_ms": round(dense_ms, 3),
+                    "useful_tflops": round(bw_useful / (wave_ms * 1e-3) / 1e12, 2),
+                    "dense_tflops": round(bw_dense / (dense_ms * 1e-3) / 1e12, 2),
+                    "speedup_over_dense": round(dense_ms / wave_ms, 4),
+                    "useful_flops": bw_useful, "peak": peaks["bf16_tflops"],
+                    "frac": round(bw_useful / (wave_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                    "note": "useful FLOPs pair exact: 3 group-masked products (S, dQ, dK) + 2 full (dP, dV); the "
+                            "kernels recompute S and dP in both passes (7 products)"}
+        del dout, dq, dk, dv
+        path.prefill()  # the wave forward's outputs again
+
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e and args.only == "all":
@@ -631,6 +676,7 @@ def run_ours(args, rank, world, local):
                   "frac": round(rope_bytes / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                   "kernel_ms": round(rope_ms, 5), "bytes_per_step": rope_bytes} if do_prefill else None),
         "dense_comparison": dense,
+        "backward": backward,
         "e2e": e2e,
         "gpu_launches": {"all": 6, "prefill": 3, "decode": 3}[args.only] * K,
         "clocks": clk,

@@ -191,6 +191,46 @@ int wp_prefill_ex(const void *q, const void *k, const void *v, void *o, float *l
                   int cut_rows, int layout, float softmax_scale, void *stream);
 
 /*
+ * wp_prefill_backward_workspace_bytes — size of the scratch that
+ * wp_prefill_backward needs (one fp32 per query row and head).
+ */
+size_t wp_prefill_backward_workspace_bytes(int B, int N, int H_q);
+
+/*
+ * wp_prefill_backward — gradients of a grouped-mode wp_prefill: given dO, the
+ * gradients dQ, dK, dV of sum(dO * O) with respect to its inputs q (rotated),
+ * k (rotated) and v. [RN §2.3, the paragraph on the backward kernel]: in the
+ * backward the head dimension is the output axis of the dQ and dK products,
+ * so the group mask is applied to the gradient operand dS = P * (dP - D)
+ * before each product (full groups take dS as it is, skipped groups add
+ * nothing), and dQ and dK come from the same masked operands; [RN §4.6,
+ * Table 4] reports that the backward gains little. The pages print no
+ * backward equations: this is the chain rule through wp_prefill's definition,
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . V_j - D_i),  D_i = dO_i . O_i,
+ *   dQ_i[g] = scale sum_j 1[i-j <= W_g] dS_ij K_j[g],
+ *   dK_j[g] = scale sum_i 1[i-j <= W_g] dS_ij Q_i[g].
+ *   q, o, dout  device bf16 [B, N, H_q, d_h]: the forward's inputs q, its
+ *               output o and the incoming gradient.
+ *   k, v        device bf16 [B, N, H_kv, d_h].
+ *   lse         device fp32 [B, H_q, N]: the forward's LSE (natural log).
+ *   dq          device bf16 out [B, N, H_q, d_h]; dk, dv device bf16 out
+ *               [B, N, H_kv, d_h] (the query heads sharing a KV head add up).
+ *   workspace   device scratch of at least
+ *               wp_prefill_backward_workspace_bytes(B, N, H_q) bytes, 256-byte
+ *               aligned (holds D).
+ *   cut, cut_rows  group cutoffs as in wp_prefill_ex: cut_rows = 1 (cut
+ *               [d_h/16], or NULL: dense) or H_q ([H_q][d_h/16]).
+ *   softmax_scale  the forward's scale (<= 0: 1/sqrt(d_h)).
+ * Grouped mode only. The products run on warp-level tensor cores with bf16
+ * operands (P and dS rounded to bf16) and fp32 accumulation. d_h in
+ * {64, 128}. Errors: WP_ERR_ARG, WP_ERR_UNSUPPORTED (also: more than 2048
+ * table entries; more than 64 query heads per KV head), WP_ERR_CUDA.
+ */
+int wp_prefill_backward(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+                        void *dq, void *dk, void *dv, void *workspace, size_t ws_bytes, int B, int N, int H_q,
+                        int H_kv, int d_h, const int32_t *cut, int cut_rows, float softmax_scale, void *stream);
+
+/*
  * wp_decode_workspace_bytes — size of the scratch that wp_decode needs for
  * the split-KV partial results of a batch (fp32 partial O and LSE per split).
  */

@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "ROPE_INTERLEAVED", "ROPE_HALF_SPLIT", "ROPE_HALF_SPLIT_PAIRED", "MODE_GROUPED", "MODE_CHANNEL", "CUTOFF_INF",
     "WavePruneError", "library_path", "load_library",
-    "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_decode", "wp_decode_workspace_bytes",
+    "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_prefill_backward", "wp_decode",
+    "wp_decode_workspace_bytes",
     "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES", "wp_kcache_group_major", "KCACHE_ROWS", "KCACHE_GROUP_MAJOR",
     "wp_decode_paged",
     "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
@@ -75,6 +76,10 @@ def load_library():
     lib.wp_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, I, F, P]
     lib.wp_prefill_ex.restype = I
     lib.wp_prefill_ex.argtypes = [P, P, P, P, P, P, I, I, ctypes.c_int64, I, I, I, I, P, I, I, F, P]
+    lib.wp_prefill_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.wp_prefill_backward_workspace_bytes.argtypes = [I, I, I]
+    lib.wp_prefill_backward.restype = I
+    lib.wp_prefill_backward.argtypes = [P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, I, I, I, I, I, P, I, F, P]
     lib.wp_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.wp_decode_workspace_bytes.argtypes = [I, I, I, I]
     lib.wp_decode.restype = I
@@ -252,6 +257,46 @@ def wp_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cut=None, mode
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens), B, N, T, Hq, Hkv, d, int(mode), cut_p,
         cut_rows, int(layout), float(softmax_scale), _stream(stream)))
     return out, lse
+
+
+def wp_prefill_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                        dout: torch.Tensor, cut=None, softmax_scale: float = 0.0, dq: torch.Tensor | None = None,
+                        dk: torch.Tensor | None = None, dv: torch.Tensor | None = None,
+                        workspace: torch.Tensor | None = None, stream=None):
+    """Gradients (dq, dk, dv) of a grouped-mode wp_prefill: q/o/dout
+    [B,N,Hq,d], k/v [B,N,Hkv,d] bf16, lse [B,Hq,N] fp32 from the forward.
+    ``cut``: group cutoffs [d/16], per-head [Hq, d/16], or None (dense)."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, name, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (B, N, Hkv, d) or tuple(v.shape) != (B, N, Hkv, d):
+        raise ValueError("k/v shape mismatch")
+    if tuple(o.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("o/dout/lse shape mismatch")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, ref, name in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _need(t, name, torch.bfloat16, 4)
+        if t.shape != ref.shape:
+            raise ValueError(f"{name} shape mismatch")
+    lib = load_library()
+    ws_bytes = int(lib.wp_prefill_backward_workspace_bytes(B, N, Hq))
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    cut_rows = 1
+    cut_p = None
+    if cut is not None:
+        arr = np.asarray(cut)
+        cut_rows = Hq if arr.ndim == 2 else 1
+        cut_a, cut_p = _host_i32(arr.reshape(-1), cut_rows * (d // 16))
+    _check("wp_prefill_backward", lib.wp_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), B, N, Hq, Hkv, d, cut_p, cut_rows, float(softmax_scale),
+        _stream(stream)))
+    return dq, dk, dv
 
 
 def wp_decode_workspace_bytes(B: int, Hq: int, d_h: int, Lmax: int) -> int:

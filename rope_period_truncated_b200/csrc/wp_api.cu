@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "waveprune.h"
+#include "wp_backward.h"
 #include "wp_decode.h"
 #include "wp_device.cuh"
 #include "wp_prefill.h"
@@ -263,6 +264,58 @@ int wp_prefill(const void *q, const void *k, const void *v, void *o, float *lse,
                int d_h, int mode, const int32_t *cut, int layout, float softmax_scale, void *stream) {
   return wp_prefill_ex(q, k, v, o, lse, nullptr, B, N, 0, H_q, H_kv, d_h, mode, cut, 1, layout, softmax_scale,
                        stream);
+}
+
+size_t wp_prefill_backward_workspace_bytes(int B, int N, int H_q) {
+  if (B <= 0 || N <= 0 || H_q <= 0) return 0;
+  return (static_cast<size_t>(B) * H_q * N * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+int wp_prefill_backward(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
+                        void *dq, void *dk, void *dv, void *workspace, size_t ws_bytes, int B, int N, int H_q,
+                        int H_kv, int d_h, const int32_t *cut, int cut_rows, float softmax_scale, void *stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || dout == nullptr || lse == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return WP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return WP_ERR_ARG;
+  if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  if (B > 65535 || H_q > 65535 || H_kv > 65535) return WP_ERR_UNSUPPORTED;
+  if (!std::isfinite(softmax_scale)) return WP_ERR_ARG;
+  if (cut_rows != 1 && cut_rows != H_q) return WP_ERR_ARG;
+  if (cut_rows != 1 && cut == nullptr) return WP_ERR_ARG;
+  if (ws_bytes < wp_prefill_backward_workspace_bytes(B, N, H_q)) return WP_ERR_ARG;
+  const int G = d_h / 16;
+  if (static_cast<int64_t>(cut_rows) * G > PREFILL_CUT_CAP) return WP_ERR_UNSUPPORTED;
+  // the key-major kernel keeps the cutoff rows of the query heads of one KV head in shared memory
+  if (H_q / H_kv > 64) return WP_ERR_UNSUPPORTED;
+  const float scale = softmax_scale > 0.f ? softmax_scale : static_cast<float>(1.0 / std::sqrt(double(d_h)));
+  BackwardArgs a;
+  a.q = static_cast<const __nv_bfloat16 *>(q);
+  a.k = static_cast<const __nv_bfloat16 *>(k);
+  a.v = static_cast<const __nv_bfloat16 *>(v);
+  a.o = static_cast<const __nv_bfloat16 *>(o);
+  a.dout = static_cast<const __nv_bfloat16 *>(dout);
+  a.lse = lse;
+  a.delta = static_cast<float *>(workspace);
+  a.dq = static_cast<__nv_bfloat16 *>(dq);
+  a.dk = static_cast<__nv_bfloat16 *>(dk);
+  a.dv = static_cast<__nv_bfloat16 *>(dv);
+  a.B = B;
+  a.N = N;
+  a.Hq = H_q;
+  a.Hkv = H_kv;
+  a.cut_rows = cut_rows;
+  for (int e = 0; e < cut_rows * G; ++e) {
+    a.cut[e] = cut == nullptr ? WP_CUTOFF_INF : cut[e];
+    if (a.cut[e] < 0) return WP_ERR_ARG;
+  }
+  a.scale = scale;
+  a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
+  return from_cuda(launch_backward(d_h, a, static_cast<cudaStream_t>(stream)));
 }
 
 size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {

@@ -50,3 +50,31 @@ def assert_attention_close(o_gpu, lse_gpu, o_ref, lse_ref, tag: str = ""):
         assert not bad.any(), f"{tag}: LSE off at {np.argwhere(bad)[:5].tolist()} " \
                               f"max {np.abs(lse - lse_ref).max():.3e}"
     return float(err.max()), float(err.mean())
+
+
+# Gradients (wp_prefill_backward) against the fp64 oracle's: the kernel rounds
+# P and dS to bf16 (relative rounding 2^-9) before the dV, dQ and dK products
+# and takes D from the forward's bf16 O, so each entry carries a relative error
+# of a few 2^-9 of the terms it sums. The bounds are relative to the size of
+# the reference gradient, max |dG| <= 2e-2 max |G| + 1e-4 and
+# mean |dG| <= 1e-2 mean |G| + 1e-5; the small absolute terms cover gradients
+# that are exactly 0 (one key: dS = dP - D = 0), where the kernel leaves the
+# fp32 rounding of dP - D.
+GRAD_MAX_REL = 2e-2
+GRAD_MEAN_REL = 1e-2
+GRAD_MAX_ABS = 1e-4
+GRAD_MEAN_ABS = 1e-5
+
+
+def assert_grad_close(g_gpu, g_ref, tag: str = ""):
+    g = widen(g_gpu).reshape(g_ref.shape)
+    err = np.abs(g - g_ref)
+    assert np.all(np.isfinite(g)), f"{tag}: non-finite gradient"
+    ref_max, ref_mean = float(np.abs(g_ref).max()), float(np.abs(g_ref).mean())
+    assert err.max() <= GRAD_MAX_REL * ref_max + GRAD_MAX_ABS, \
+        f"{tag}: max |dG| {err.max():.3e} vs max |G| {ref_max:.3e}"
+    assert err.mean() <= GRAD_MEAN_REL * ref_mean + GRAD_MEAN_ABS, \
+        f"{tag}: mean |dG| {err.mean():.3e} vs mean |G| {ref_mean:.3e}"
+    print(f"{tag}: max |dG|/max |G| {err.max() / max(ref_max, 1e-30):.2e}, "
+          f"mean |dG|/mean |G| {err.mean() / max(ref_mean, 1e-30):.2e}")
+    return float(err.max() / max(ref_max, 1e-30)), float(err.mean() / max(ref_mean, 1e-30))

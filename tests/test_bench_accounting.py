@@ -51,6 +51,21 @@ def test_prefill_flops_32k_figures():
     assert abs(pair_dense / 1e12 - 8.796) < 5e-4
 
 
+@pytest.mark.parametrize("N", [1, 130, 400])
+def test_backward_flops_match_enumeration(N):
+    """Per causal pair: S, dQ and dK over the in-window groups (2*16 each per
+    group) and dP, dV in full (2*d each)."""
+    d, wg = 64, [0, 3, 130, 1000]
+    useful, dense = bench.backward_flops(N, d, 2, 3, wg)
+    tot = tot_dense = 0
+    for i in range(N):
+        for j in range(i + 1):
+            tot += 3 * 2 * 16 * sum(1 for w in wg if i - j <= w) + 2 * 2 * d
+            tot_dense += 3 * 2 * d + 2 * 2 * d
+    assert useful == tot * 2 * 3
+    assert dense == tot_dense * 2 * 3
+
+
 def test_decode_required_bytes_match_enumeration():
     rng = np.random.default_rng(3)
     lens = rng.integers(1, 400, size=5)
