@@ -297,6 +297,30 @@ int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vc
                  void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * wp_decode_ex — wp_decode_kl with the exact per-channel rule or one cutoff
+ * table per query head.
+ *   mode, cut, cut_rows, layout:
+ *     WP_MODE_GROUPED, cut_rows = 1: cut is group_cut [d_h/16] (as wp_decode).
+ *     WP_MODE_GROUPED, cut_rows = H_q: cut is [H_q][d_h/16], row h for query
+ *       head h ([RN §5]: head-specific thresholds). The K loads cover the
+ *       union of the heads' windows; each head's scores keep a group's
+ *       product only while the key is in that head's window.
+ *     WP_MODE_CHANNEL, cut_rows = 1: cut is chan_cut [d_h/2] (NULL: dense),
+ *       the exact rule of [RN §2.1, Eq. (6)]; layout (WP_ROPE_INTERLEAVED or
+ *       WP_ROPE_HALF_SPLIT) says which channel owns a dim. The decode query
+ *       has one position, so the dims of a channel out of window are zeroed
+ *       per key before the product; a group's K bytes are skipped beyond its
+ *       largest channel cutoff.
+ * Everything else as in wp_decode_kl. Errors: those of wp_decode_kl, and
+ * WP_ERR_ARG (mode, layout or cut_rows out of range, NULL cut with
+ * cut_rows = H_q), WP_ERR_UNSUPPORTED (channel mode with cut_rows = H_q;
+ * H_q x d_h/16 above 1024).
+ */
+int wp_decode_ex(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
+                 int B, int H_q, int H_kv, int d_h, int mode, const int32_t *cut, int cut_rows, int layout,
+                 float softmax_scale, void *o, float *lse, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * wp_decode_paged — wp_decode_kl over a paged KV cache, as serving engines
  * keep it: the keys of a sequence live in fixed-size pages from a shared pool,
  * listed per sequence in a block table. (The pages' decode reads one

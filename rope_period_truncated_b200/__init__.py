@@ -88,6 +88,8 @@ def load_library():
     lib.wp_decode_static.argtypes = [P, P, P, P, I, I, I, I, I, P, F, P, P, P]
     lib.wp_decode_kl.restype = I
     lib.wp_decode_kl.argtypes = [P, P, I, P, P, I, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
+    lib.wp_decode_ex.restype = I
+    lib.wp_decode_ex.argtypes = [P, P, I, P, P, I, I, I, I, I, I, P, I, I, F, P, P, P, ctypes.c_size_t, P]
     lib.wp_decode_paged.restype = I
     lib.wp_decode_paged.argtypes = [P, P, I, P, I, I, P, I, P, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
     lib.wp_kcache_group_major.restype = I
@@ -319,10 +321,13 @@ def wp_kcache_group_major(kcache: torch.Tensor, out: torch.Tensor | None = None,
 
 def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens: torch.Tensor, group_cut=None,
               softmax_scale: float = 0.0, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
-              workspace: torch.Tensor | None = None, want_lse: bool = True, stream=None):
+              workspace: torch.Tensor | None = None, want_lse: bool = True, stream=None, mode: int = MODE_GROUPED,
+              layout: int = ROPE_INTERLEAVED):
     """Split-KV decode. q [B,Hq,d] (rotated), V cache [B,Hkv,Lmax,d] bf16, K
     cache the same (rows) or [B,Hkv,d/16,Lmax,16] (group-major, from
-    wp_kcache_group_major), lens int32 [B] (device). Returns (o [B,Hq,d] bf16,
+    wp_kcache_group_major), lens int32 [B] (device). ``group_cut``: group
+    cutoffs [d/16], per-head [Hq, d/16], or (mode=MODE_CHANNEL) channel
+    cutoffs [d/2] with ``layout``; None = dense. Returns (o [B,Hq,d] bf16,
     lse [B,Hq] fp32)."""
     _need(q, "q", torch.bfloat16, 3)
     _need(vcache, "vcache", torch.bfloat16, 4)
@@ -350,10 +355,20 @@ def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if workspace.numel() * workspace.element_size() < ws_bytes:
         raise ValueError("workspace too small")
-    cut_a, cut_p = _host_i32(group_cut, d // 16)
-    _check("wp_decode", load_library().wp_decode_kl(
-        _ptr(q), _ptr(kcache), k_layout, _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p, float(softmax_scale),
-        _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    cut_rows = 1 if group_cut is None or np.asarray(group_cut).ndim == 1 else Hq
+    if mode == MODE_GROUPED and cut_rows == 1:
+        cut_a, cut_p = _host_i32(group_cut, d // 16)
+        _check("wp_decode", load_library().wp_decode_kl(
+            _ptr(q), _ptr(kcache), k_layout, _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, cut_p,
+            float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream(stream)))
+        return out, lse
+    n = (d // 16 if mode == MODE_GROUPED else d // 2) * cut_rows
+    cut_a, cut_p = _host_i32(None if group_cut is None else np.asarray(group_cut).reshape(-1), n)
+    _check("wp_decode", load_library().wp_decode_ex(
+        _ptr(q), _ptr(kcache), k_layout, _ptr(vcache), _ptr(lens), Lmax, B, Hq, Hkv, d, int(mode), cut_p, cut_rows,
+        int(layout), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
     return out, lse
 
 

@@ -326,10 +326,13 @@ size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {
 
 // Shared argument checks and launch of the split-KV decode; block_table null
 // = contiguous caches of Lmax keys, else pages of page_size keys.
+// mask / tables: DECODE_MASK_GROUP_SHARED with group_cut (NULL: dense), or a
+// masked mode with its tables, group_cut then holding the loads' cutoffs.
 static int decode_launch(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens,
                          int Lmax, int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale,
                          void *o, float *lse, void *workspace, size_t ws_bytes, const int32_t *block_table,
-                         int max_pages, int page_size, int n_pages, void *stream) {
+                         int max_pages, int page_size, int n_pages, void *stream, int mask = DECODE_MASK_GROUP_SHARED,
+                         int layout = WP_ROPE_INTERLEAVED, const DecodeTables *tables = nullptr) {
   if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr ||
       workspace == nullptr)
     return WP_ERR_ARG;
@@ -373,7 +376,9 @@ static int decode_launch(const void *q, const void *kcache, int k_layout, const 
     if (a.cut[g] < 0) return WP_ERR_ARG;
   }
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
-  return from_cuda(launch_decode(a, d_h, static_cast<cudaStream_t>(stream)));
+  a.mask = mask;
+  a.layout = layout;
+  return from_cuda(launch_decode(a, tables, d_h, static_cast<cudaStream_t>(stream)));
 }
 
 int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
@@ -381,6 +386,50 @@ int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vc
                  void *workspace, size_t ws_bytes, void *stream) {
   return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, group_cut, softmax_scale, o, lse,
                        workspace, ws_bytes, nullptr, 0, 0, 0, stream);
+}
+
+int wp_decode_ex(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
+                 int B, int H_q, int H_kv, int d_h, int mode, const int32_t *cut, int cut_rows, int layout,
+                 float softmax_scale, void *o, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+  if (mode != WP_MODE_GROUPED && mode != WP_MODE_CHANNEL) return WP_ERR_ARG;
+  if (layout != WP_ROPE_INTERLEAVED && layout != WP_ROPE_HALF_SPLIT) return WP_ERR_ARG;
+  if (H_q <= 0 || (cut_rows != 1 && cut_rows != H_q)) return WP_ERR_ARG;
+  if (cut_rows != 1 && cut == nullptr) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  const int G = d_h / 16, C = d_h / 2;
+  if (mode == WP_MODE_GROUPED && cut_rows == 1)
+    return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, cut, softmax_scale, o, lse,
+                         workspace, ws_bytes, nullptr, 0, 0, 0, stream);
+  if (mode == WP_MODE_CHANNEL && cut_rows != 1) return WP_ERR_UNSUPPORTED;  // per-head exact tables: not built
+  DecodeTables tables;
+  int32_t load_cut[8];
+  if (mode == WP_MODE_GROUPED) {
+    if (static_cast<int64_t>(H_q) * G > 1024) return WP_ERR_UNSUPPORTED;
+    // the K loads cover the union of the heads' windows
+    for (int g = 0; g < G; ++g) load_cut[g] = 0;
+    for (int e = 0; e < H_q * G; ++e) {
+      if (cut[e] < 0) return WP_ERR_ARG;
+      tables.head_cut[e] = cut[e];
+      load_cut[e % G] = cut[e] > load_cut[e % G] ? cut[e] : load_cut[e % G];
+    }
+  } else {
+    // exact rule: a group's K loads follow its largest channel cutoff
+    for (int c = 0; c < C; ++c) {
+      tables.chan_cut[c] = cut == nullptr ? WP_CUTOFF_INF : cut[c];
+      if (tables.chan_cut[c] < 0) return WP_ERR_ARG;
+    }
+    for (int g = 0; g < G; ++g) {
+      int32_t m = 0;
+      for (int k = 16 * g; k < 16 * g + 16; ++k) {
+        const int c = layout == WP_ROPE_INTERLEAVED ? k / 2 : k % C;
+        m = tables.chan_cut[c] > m ? tables.chan_cut[c] : m;
+      }
+      load_cut[g] = m;
+    }
+  }
+  return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, load_cut, softmax_scale, o, lse,
+                       workspace, ws_bytes, nullptr, 0, 0, 0, stream,
+                       mode == WP_MODE_GROUPED ? DECODE_MASK_GROUP_PER_HEAD : DECODE_MASK_CHANNEL, layout, &tables);
 }
 
 int wp_decode_paged(const void *q, const void *k_pages, int k_layout, const void *v_pages, int n_pages, int page_size,

@@ -27,6 +27,7 @@
 // Combine kernel: per (sequence, query head) merge the splits by LSE.
 #include <cuda_bf16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "wp_decode.h"
 #include "wp_device.cuh"
@@ -90,8 +91,26 @@ __device__ __forceinline__ uint32_t piece_off(int r, int p) {
   return static_cast<uint32_t>(r) * DecLayout<D>::ROWB + static_cast<uint32_t>((p ^ (r & 7)) * 16);
 }
 
-template <int D, int R, bool KGM, bool PAGED>
-__global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeArgs a) {
+struct NoDecodeTables {
+  int32_t unused;
+};
+template <int MASK>
+using DecodeTablesArg = typename std::conditional<MASK == DECODE_MASK_GROUP_SHARED, NoDecodeTables, DecodeTables>::type;
+
+// Zeroes the bf16 halves of r (dims k and k+1 of one key) whose channel is out
+// of window at distance dist: the exact per-channel rule on the K operand.
+template <int D>
+__device__ __forceinline__ uint32_t mask_channels(uint32_t r, int k, int64_t dist, const int32_t *ccut, int layout) {
+  constexpr int C = D / 2;
+  const int c0 = layout == WP_ROPE_INTERLEAVED ? k >> 1 : k % C;
+  const int c1 = layout == WP_ROPE_INTERLEAVED ? k >> 1 : (k + 1) % C;
+  const uint32_t keep = (dist <= ccut[c0] ? 0x0000ffffu : 0u) | (dist <= ccut[c1] ? 0xffff0000u : 0u);
+  return r & keep;
+}
+
+template <int D, int R, bool KGM, bool PAGED, int MASK>
+__global__ void __launch_bounds__(DEC_THREADS)
+    decode_split_kernel(const DecodeArgs a, const __grid_constant__ DecodeTablesArg<MASK> tabs) {
   using L = DecLayout<D>;
   constexpr int PIECES = L::PIECES;
   constexpr int KSTEPS = D / 16;
@@ -125,6 +144,15 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
   }
   const int g = lane >> 2, t = lane & 3;
   const int64_t qpos = len - 1;
+  // masked modes: the R heads' group rows or the channel cutoffs in shared memory
+  int32_t *mcut = reinterpret_cast<int32_t *>(dsmem + L::BYTES);
+  if constexpr (MASK == DECODE_MASK_GROUP_PER_HEAD) {
+    for (int e = threadIdx.x; e < R * 8; e += DEC_THREADS)
+      mcut[e] = (e % 8) < D / 16 ? tabs.head_cut[(hq0 + e / 8) * (D / 16) + e % 8] : WP_CUTOFF_INF;
+  } else if constexpr (MASK == DECODE_MASK_CHANNEL) {
+    for (int e = threadIdx.x; e < D / 2; e += DEC_THREADS) mcut[e] = tabs.chan_cut[e];
+  }
+  if constexpr (MASK != DECODE_MASK_GROUP_SHARED) __syncthreads();
 
   // Q as the A operand (rows = query heads; rows >= R and 8..15 are zero).
   uint32_t qa[KSTEPS][2];
@@ -231,8 +259,29 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_split_kernel(const DecodeA
       const int mi = lane >> 3, rr = (mi >> 1) * 8 + (lane & 7), pp = 2 * c + (mi & 1);
       uint32_t b00, b01, b10, b11;
       ldsm_x4(ks + piece_off<D>(rr, pp), b00, b01, b10, b11);
-      mma_16816(s0, qa[c][0], 0u, qa[c][1], 0u, b00, b01);
-      mma_16816(s1, qa[c][0], 0u, qa[c][1], 0u, b10, b11);
+      if constexpr (MASK == DECODE_MASK_CHANNEL) {
+        // b00/b01: key g, dims 16c + 2t (+1) and 16c + 8 + 2t (+1); b10/b11: key 8 + g
+        const int64_t d0 = qpos - (kb0 + g), d1 = d0 - 8;
+        b00 = mask_channels<D>(b00, 16 * c + 2 * t, d0, mcut, a.layout);
+        b01 = mask_channels<D>(b01, 16 * c + 8 + 2 * t, d0, mcut, a.layout);
+        b10 = mask_channels<D>(b10, 16 * c + 2 * t, d1, mcut, a.layout);
+        b11 = mask_channels<D>(b11, 16 * c + 8 + 2 * t, d1, mcut, a.layout);
+      }
+      if constexpr (MASK == DECODE_MASK_GROUP_PER_HEAD) {
+        // this group's products apart, then kept per head (row g) and key
+        float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_16816(t0, qa[c][0], 0u, qa[c][1], 0u, b00, b01);
+        mma_16816(t1, qa[c][0], 0u, qa[c][1], 0u, b10, b11);
+        const int64_t W = mcut[(g < R ? g : 0) * 8 + c];
+        const int64_t d0 = qpos - (kb0 + 2 * t), d2 = d0 - 8;
+        s0[0] += d0 <= W ? t0[0] : 0.f;
+        s0[1] += d0 - 1 <= W ? t0[1] : 0.f;
+        s1[0] += d2 <= W ? t1[0] : 0.f;
+        s1[1] += d2 - 1 <= W ? t1[1] : 0.f;
+      } else {
+        mma_16816(s0, qa[c][0], 0u, qa[c][1], 0u, b00, b01);
+        mma_16816(s1, qa[c][0], 0u, qa[c][1], 0u, b10, b11);
+      }
     }
     // lane holds head g, keys 2t, 2t+1 (s0[0..1]) and 8+2t, 9+2t (s1[0..1])
     float sc[4] = {s0[0], s0[1], s1[0], s1[1]};
@@ -337,22 +386,35 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
   if (d == 0 && a.lse != nullptr) a.lse[bh] = (M + log2f(Lsum)) * 0.69314718055994531f;
 }
 
-template <int D, int R, bool KGM, bool PAGED>
-cudaError_t launch_split_l(const DecodeArgs &a, cudaStream_t stream) {
-  const uint32_t smem = DecLayout<D>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, R, KGM, PAGED>,
+template <int D, int R, bool KGM, bool PAGED, int MASK>
+cudaError_t launch_split_l(const DecodeArgs &a, const DecodeTables *tables, cudaStream_t stream) {
+  const uint32_t smem = DecLayout<D>::BYTES + (MASK == DECODE_MASK_GROUP_SHARED ? 0u : 256u);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, R, KGM, PAGED, MASK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.nsplit, a.Hkv, a.B);
-  decode_split_kernel<D, R, KGM, PAGED><<<grid, DEC_THREADS, smem, stream>>>(a);
+  DecodeTablesArg<MASK> tabs;
+  if constexpr (MASK == DECODE_MASK_GROUP_SHARED)
+    tabs.unused = 0;
+  else
+    tabs = *tables;
+  decode_split_kernel<D, R, KGM, PAGED, MASK><<<grid, DEC_THREADS, smem, stream>>>(a, tabs);
   return cudaGetLastError();
 }
 
 template <int D, int R>
-cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+cudaError_t launch_split(const DecodeArgs &a, const DecodeTables *tables, cudaStream_t stream) {
+  if (a.mask == DECODE_MASK_GROUP_PER_HEAD)  // contiguous caches only (checked on the host)
+    return a.k_group_major ? launch_split_l<D, R, true, false, DECODE_MASK_GROUP_PER_HEAD>(a, tables, stream)
+                           : launch_split_l<D, R, false, false, DECODE_MASK_GROUP_PER_HEAD>(a, tables, stream);
+  if (a.mask == DECODE_MASK_CHANNEL)
+    return a.k_group_major ? launch_split_l<D, R, true, false, DECODE_MASK_CHANNEL>(a, tables, stream)
+                           : launch_split_l<D, R, false, false, DECODE_MASK_CHANNEL>(a, tables, stream);
   if (a.block_table != nullptr)
-    return a.k_group_major ? launch_split_l<D, R, true, true>(a, stream) : launch_split_l<D, R, false, true>(a, stream);
-  return a.k_group_major ? launch_split_l<D, R, true, false>(a, stream) : launch_split_l<D, R, false, false>(a, stream);
+    return a.k_group_major ? launch_split_l<D, R, true, true, 0>(a, tables, stream)
+                           : launch_split_l<D, R, false, true, 0>(a, tables, stream);
+  return a.k_group_major ? launch_split_l<D, R, true, false, 0>(a, tables, stream)
+                         : launch_split_l<D, R, false, false, 0>(a, tables, stream);
 }
 
 // One thread per 16-byte piece of the group-major output, in output order:
@@ -374,12 +436,12 @@ __global__ void kcache_group_major_kernel(const uint4 *__restrict__ src, uint4 *
 }
 
 template <int D>
-cudaError_t launch_split_r(const DecodeArgs &a, int R, cudaStream_t stream) {
+cudaError_t launch_split_r(const DecodeArgs &a, const DecodeTables *tables, int R, cudaStream_t stream) {
   switch (R) {
-    case 1: return launch_split<D, 1>(a, stream);
-    case 2: return launch_split<D, 2>(a, stream);
-    case 4: return launch_split<D, 4>(a, stream);
-    default: return launch_split<D, 8>(a, stream);
+    case 1: return launch_split<D, 1>(a, tables, stream);
+    case 2: return launch_split<D, 2>(a, tables, stream);
+    case 4: return launch_split<D, 4>(a, tables, stream);
+    default: return launch_split<D, 8>(a, tables, stream);
   }
 }
 
@@ -398,9 +460,10 @@ cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *d
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeArgs &a, const DecodeTables *tables, int d_h, cudaStream_t stream) {
   const int R = a.Hq / a.Hkv;
-  cudaError_t e = d_h == 128 ? launch_split_r<128>(a, R, stream) : launch_split_r<64>(a, R, stream);
+  cudaError_t e =
+      d_h == 128 ? launch_split_r<128>(a, tables, R, stream) : launch_split_r<64>(a, tables, R, stream);
   if (e != cudaSuccess) return e;
   if (d_h == 128)
     decode_combine_kernel<128><<<a.B * a.Hq, 128, 0, stream>>>(a);

@@ -23,8 +23,24 @@ struct DecodeArgs {
   int k_group_major;                 // K cache layout: 0 rows, 1 group-major
   const int32_t *block_table;        // paged cache: [B, max_pages] page of each page_size-key block, or null
   int max_pages, page_size, n_pages;
-  int32_t cut[8];                    // group cutoffs
+  int32_t cut[8];                    // group cutoffs (of the K loads: the union over heads / channels)
   float scale_log2;
+  int mask;                          // DECODE_MASK_*: how scores are masked beyond the K loads
+  int layout;                        // rotation layout (channel mode: which channel owns a dim)
+};
+
+// Score masking of the decode kernel. GROUP_SHARED: every head takes `cut`
+// (the K loads already leave out-of-window groups as zeros). GROUP_PER_HEAD:
+// query head h takes row h of a per-head table (the loads cover the union of
+// the heads' windows and each head's scores are masked group by group).
+// CHANNEL: the exact per-channel rule (one query position per sequence, so a
+// channel's K dims are zeroed per key before the product).
+enum : int { DECODE_MASK_GROUP_SHARED = 0, DECODE_MASK_GROUP_PER_HEAD = 1, DECODE_MASK_CHANNEL = 2 };
+
+// Cutoff tables of the masked decode modes, a kernel parameter of their own.
+struct DecodeTables {
+  int32_t head_cut[1024];  // [Hq][D/16] (GROUP_PER_HEAD)
+  int32_t chan_cut[64];    // [D/2] (CHANNEL)
 };
 
 // Scratch layout: o_part first, then lse_part at a 256-byte boundary.
@@ -36,7 +52,7 @@ inline size_t decode_workspace_bytes(int B, int Hq, int nsplit, int D) {
          ((static_cast<size_t>(B) * Hq * nsplit * sizeof(float) + 255) & ~static_cast<size_t>(255));
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, int d_h, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs &a, const DecodeTables *tables, int d_h, cudaStream_t stream);
 
 // K cache rows [BH, Lmax, D] -> group-major [BH, D/16, Lmax, 16] (BH = B * H_kv).
 cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int64_t BH, int Lmax, int D,

@@ -213,3 +213,64 @@ def test_decode_paged_bad_page_gives_nan_rows():
     assert torch.isnan(o[1]).all()
     ro, rl = oracle.decode(widen(q[:1]), widen(kc[:1]), widen(vc[:1]), lens[:1].numpy(), np.full(d // 16, 2 ** 31 - 1))
     assert_attention_close(o[:1].to(torch.bfloat16), lse[:1], ro, rl, "paged, sequence with valid pages")
+
+
+def _decode_inputs(seed, B, Hq, Hkv, d, Lmax):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    return q, kc, vc
+
+
+@pytest.mark.parametrize("group_major", [False, True])
+@pytest.mark.parametrize("Hq,Hkv,d", [(8, 2, 128), (4, 4, 64), (16, 2, 128)])
+def test_decode_per_head_tables(Hq, Hkv, d, group_major):
+    """One cutoff row per query head (wp_decode_ex, grouped): the K loads
+    cover the union of the heads' windows and each head keeps a group's
+    product only inside its own window. Oracle: one head at a time."""
+    B, Lmax = 4, 3000
+    lens = torch.tensor([1, 2999, 1500, 1025], dtype=torch.int32)
+    q, kc, vc = _decode_inputs(61 + Hq + d, B, Hq, Hkv, d, Lmax)
+    rng = np.random.default_rng(Hq * 7 + d)
+    G = d // 16
+    cut = rng.integers(0, 2500, size=(Hq, G)).astype(np.int32)
+    cut[0] = 2 ** 31 - 1  # a dense head next to pruned ones
+    kcd = wp.wp_kcache_group_major(kc.cuda()) if group_major else kc.cuda()
+    o, lse = wp.wp_decode(q.cuda(), kcd, vc.cuda(), lens.cuda(), cut)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    ro = np.zeros((B, Hq, d))
+    rl = np.zeros((B, Hq))
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        a, b_ = oracle.decode(widen(q[:, h:h + 1]), widen(kc[:, hk:hk + 1]), widen(vc[:, hk:hk + 1]), lens.numpy(),
+                              cut[h])
+        ro[:, h], rl[:, h] = a[:, 0], b_[:, 0]
+    assert_attention_close(o, lse, ro, rl, f"per-head decode Hq={Hq} d={d} gm={group_major}")
+
+
+@pytest.mark.parametrize("layout", [wp.ROPE_INTERLEAVED, wp.ROPE_HALF_SPLIT])
+@pytest.mark.parametrize("group_major", [False, True])
+@pytest.mark.parametrize("table", ["wave", "small"])
+def test_decode_exact_channel_mode(layout, group_major, table):
+    """Exact per-channel rule in decode (wp_decode_ex, channel mode) against
+    the oracle's channel-mode row len-1 over the cached keys."""
+    B, Hq, Hkv, d, Lmax = 3, 8, 2, 128, 2600
+    lens = torch.tensor([2600, 700, 1], dtype=torch.int32)
+    q, kc, vc = _decode_inputs(71 + layout, B, Hq, Hkv, d, Lmax)
+    if table == "wave":
+        wc, _ = oracle.cutoffs(d, 1e4, layout)
+    else:
+        wc = np.random.default_rng(5).integers(0, 600, size=d // 2).astype(np.int32)
+    kcd = wp.wp_kcache_group_major(kc.cuda()) if group_major else kc.cuda()
+    o, lse = wp.wp_decode(q.cuda(), kcd, vc.cuda(), lens.cuda(), wc, mode=wp.MODE_CHANNEL, layout=layout)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    # oracle: row len-1 of channel-mode prefill over the cached keys ([B, L, Hkv, d] order)
+    rb = np.repeat(np.arange(B), Hq)
+    rh = np.tile(np.arange(Hq), B)
+    ri = (lens.numpy().astype(np.int64) - 1)[rb]
+    ro, rl = oracle.attention_rows(widen(q).reshape(B * Hq, d), (rb, rh, ri), widen(kc).transpose(0, 2, 1, 3),
+                                   widen(vc).transpose(0, 2, 1, 3), Hq, wc, oracle.MODE_CHANNEL, layout)
+    assert_attention_close(o, lse, ro.reshape(B, Hq, d), rl.reshape(B, Hq), f"exact decode layout={layout}")
