@@ -43,11 +43,17 @@ struct ChannelPrefillArgs {
   int64_t T;
   int cut_rows;
   float scale_log2;
+  long long wait_limit;          // bound of every mbarrier wait (tensor-core kernel)
   int32_t cut[PREFILL_CUT_CAP];  // [cut_rows][d/2] channel cutoffs
 };
 
 cudaError_t launch_prefill_grouped(int d_h, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                    const PrefillArgs &a, const HeadCuts *head_cuts, cudaStream_t stream);
 cudaError_t launch_prefill_channel(int d_h, const ChannelPrefillArgs &a, cudaStream_t stream);
+
+// Exact per-channel rule on the tensor cores (uniform batches).
+constexpr uint32_t PREFILL_SMEM_CAP = 232448;  // dynamic shared memory of one CTA
+cudaError_t launch_prefill_exact(int d_h, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const ChannelPrefillArgs &a, cudaStream_t stream);
 
 }  // namespace wp

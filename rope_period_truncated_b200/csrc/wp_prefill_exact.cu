@@ -1,0 +1,640 @@
+// WavePrune exact per-channel causal prefill on sm_100a: TMA + tcgen05 + TMEM.
+//
+// What it computes (WavePrune reading notes "WavePrune：RoPE 通常只需一个旋转
+// 周期", §2.1 Eq. (6)): for j <= i,
+//   L_ij = scale * sum_c 1[i - j <= W_c] * (q_a k_a + q_b k_b)   (channel c = dims a, b),
+// then the causal softmax and O = A V. A dropped channel adds 0; the pair
+// stays in the softmax.
+//
+// How. The grouped kernel's pipeline: one CTA takes one 128-row query tile
+// of two query heads that share a KV head; a TMA producer warp, one MMA-issuing
+// warp per head, S of each head double-buffered in two 64-key TMEM halves,
+// four softmax warps per head with one thread per query row. What changes is
+// the logit tile: a tensor-core product covers 16 dims (one group), while the
+// rule keeps or drops single channels. For a 64-key sub-tile with distances
+// [dmin, dmax], every channel is skip (W_c < dmin), full (W_c >= dmax) or
+// boundary; then
+//   - a group whose channels are all full is one plain product;
+//   - a group with some full channels is one product against a copy of the
+//     sub-tile's K slice in which the dims of every other channel are zero
+//     (the producer writes the copy once the tile lands, in the TMA layout,
+//     fenced for the tensor core's async proxy; with one cutoff table both
+//     heads use it);
+//   - a boundary channel's product is rank 2, q_a k_a^T + q_b k_b^T: the
+//     softmax threads add it to their row of S with CUDA-core FMAs, only at
+//     the keys within W_c of the row, reading Q and K from the tiles the TMA
+//     loads already hold (so a K stage is free again once the MMAs and the
+//     softmax warps of both heads are done with it).
+// The producer also works out each key tile's channel plan (per head when
+// the heads have their own cutoffs) into a two-entry ring beside the K stages.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "wp_device.cuh"
+#include "wp_prefill.h"
+#include "wp_prefill_common.cuh"
+#include "wp_tile.h"
+
+namespace wp {
+
+namespace {
+
+constexpr int XBM = 128;
+constexpr int XBN = 128;  // key tile of the K/V loads
+constexpr int XSUB = 64;  // key sub-tile of one S buffer
+constexpr int XKST = 2;
+constexpr int XVST = 2;
+constexpr int XTHREADS = 352;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9/10 MMA issuer of head 0/1
+constexpr int XPRODUCER = 8;
+constexpr int XMMA = 9;
+constexpr uint32_t XTMEM_COLS = 512;
+constexpr uint32_t XGROUP_BYTES = 128 * 32;  // 128 rows x 16 bf16
+constexpr uint32_t XHALF_BYTES = 64 * 32;    // the 64 keys of one sub-tile
+constexpr uint32_t XV_CHUNK = 128 * 128;     // 128 keys x 64 bf16
+constexpr int NVAR = 2;  // masked K copies per (plan, sub-tile): partially kept groups
+
+__host__ __device__ constexpr uint32_t xcol_s(int slot) { return 256u * slot; }
+__host__ __device__ constexpr uint32_t xcol_o(int slot) { return 256u * slot + 128u; }
+
+template <int D>
+struct XLayout {
+  static constexpr int G = D / 16;
+  static constexpr uint32_t Q_SLOT = G * XGROUP_BYTES;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t K_OFF = Q_OFF + 2 * Q_SLOT;
+  static constexpr uint32_t K_STAGE = G * XGROUP_BYTES;
+  static constexpr uint32_t V_OFF = K_OFF + XKST * K_STAGE;
+  static constexpr uint32_t V_STAGE = (D / 64) * XV_CHUNK;
+  // masked K copies [stage][plan][half][NVAR], 2 KB each
+  static constexpr uint32_t KV_OFF = V_OFF + XVST * V_STAGE;
+  static constexpr uint32_t BAR_OFF = KV_OFF + XKST * 2 * 2 * NVAR * XHALF_BYTES;
+  // q_full, k_full/empty/ready, v_full/empty, per head x half s_ready/p_ready,
+  // per head o_ready/o_final/drain
+  static constexpr uint32_t NUM_BARS = 1 + 3 * XKST + 2 * XVST + 2 * 4 + 2 * 3;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;    // channel cutoffs [plan][64] int32
+  static constexpr uint32_t GMAX_OFF = CUT_OFF + 512;   // largest cutoff of each group [plan][8] int32
+  static constexpr uint32_t RING_OFF = GMAX_OFF + 64;   // plans [stage][plan][half] x {full, bnd}
+  static constexpr uint32_t END = RING_OFF + XKST * 2 * 2 * 16;
+  static constexpr uint32_t BYTES = END + 1024;  // + alignment of the dynamic base
+};
+static_assert(XLayout<128>::BYTES <= PREFILL_SMEM_CAP, "exact prefill layout exceeds shared memory");
+
+// Dims of group g (bit k = dim 16g + k) that belong to the channels in `chans`.
+// Interleaved: channel c owns dims 2c, 2c+1, so group g holds channels
+// 8g..8g+7, each twice. Half-split: channel c owns dims c and c + D/2, so
+// group g holds channels 16 (g mod D/32) .. +15, once each.
+template <int D>
+__device__ __forceinline__ uint32_t group_keep(uint64_t chans, int g, bool inter) {
+  if (inter) {
+    uint32_t x = static_cast<uint32_t>(chans >> (8 * g)) & 0xffu;
+    x = (x | (x << 4)) & 0x0f0fu;
+    x = (x | (x << 2)) & 0x3333u;
+    x = (x | (x << 1)) & 0x5555u;
+    return x | (x << 1);
+  }
+  return static_cast<uint32_t>(chans >> (16 * (g % (D / 32)))) & 0xffffu;
+}
+
+// Channels owning dims of group g.
+template <int D>
+__device__ __forceinline__ uint64_t group_chans(int g, bool inter) {
+  return inter ? 0xffull << (8 * g) : 0xffffull << (16 * (g % (D / 32)));
+}
+
+// Channel plan of the 128-query x 64-key block (qb, kb64): `full` channels go
+// to plain or partial-group products on the tensor cores, `bnd` channels to
+// masked rank-2 updates. At most NVAR groups get a masked K copy; the full
+// channels of further partial groups move to `bnd`, where their mask keeps
+// every key (W_c >= dmax).
+template <int D>
+__device__ void make_plan(const int32_t *cut, bool inter, int64_t N, int64_t qb, int64_t kb64, uint64_t &full,
+                          uint64_t &bnd) {
+  constexpr int C = D / 2, G = D / 16;
+  full = bnd = 0;
+  int64_t dmin = 0, dmax = -1;
+  if (!tile_distance_range(N, XBM, XSUB, qb, kb64, &dmin, &dmax)) return;
+  for (int c = 0; c < C; ++c) {
+    const int cls = classify_cutoff(dmin, dmax, cut[c]);
+    if (cls == TILE_FULL) full |= 1ull << c;
+    if (cls == TILE_BOUNDARY) bnd |= 1ull << c;
+  }
+  int nvar = 0;
+  for (int g = 0; g < G; ++g) {
+    const uint32_t keep = group_keep<D>(full, g, inter);
+    if (keep == 0u || keep == 0xffffu) continue;
+    if (++nvar <= NVAR) continue;
+    // demoting removes every full channel of g, which can turn a group
+    // counted before (half-split: g - D/32) from plain into partial, so the
+    // count restarts; every restart removes a full channel, so it ends
+    const uint64_t moved = full & group_chans<D>(g, inter);
+    full &= ~moved;
+    bnd |= moved;
+    nvar = 0;
+    g = -1;
+  }
+}
+
+// Warp-wide: copy the 64-key K half tile at `src` to `dst` (both 256-byte
+// aligned, so the TMA 32-byte swizzle is the same), keeping the dims whose bit
+// in `keep` is set and zeroing the rest. Row r's logical 16-byte chunk q sits
+// at position q ^ ((r >> 2) & 1); lane l always moves chunks of logical index
+// (l & 1) ^ ((l >> 3) & 1).
+__device__ __forceinline__ void masked_k_copy(uint8_t *dst, const uint8_t *src, uint32_t keep, int lane) {
+  const int q = (lane & 1) ^ ((lane >> 3) & 1);
+  const uint32_t m8 = (keep >> (8 * q)) & 0xffu;
+  uint32_t wm[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    wm[e] = ((m8 >> (2 * e)) & 1u ? 0x0000ffffu : 0u) | ((m8 >> (2 * e + 1)) & 1u ? 0xffff0000u : 0u);
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int x = it * 32 + lane;  // 16-byte chunk index
+    uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * x);
+    v.x &= wm[0];
+    v.y &= wm[1];
+    v.z &= wm[2];
+    v.w &= wm[3];
+    *reinterpret_cast<uint4 *>(dst + 16 * x) = v;
+  }
+}
+
+// Byte offset of (row, dim) in a 128-row x 16-dim bf16 tile stored with the
+// TMA 32-byte swizzle (address bit 4 ^= bit 7).
+__device__ __forceinline__ uint32_t sw32_offset(int row, int dim) {
+  return 32u * row + 16u * (((dim >> 3) & 1) ^ ((row >> 2) & 1)) + 2u * (dim & 7);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Adds channel c's logits to this row's 64 S columns at the keys k >= cmin:
+// S[k] += q_a k_a[k] + q_b k_b[k]. q_tile: the head's Q tile of group 0;
+// k_tile: the K stage's group-0 tile advanced to the sub-tile's first key.
+// Column chunks of 16 keys that every lane masks are skipped.
+template <int D>
+__device__ __forceinline__ void add_channel(uint32_t (&su)[64], const uint8_t *q_tile, const uint8_t *k_tile, int r,
+                                            int c, bool inter, int cmin) {
+  constexpr int C = D / 2;
+  const int da = inter ? 2 * c : c, db = inter ? 2 * c + 1 : c + C;
+  const int e = da & 15;
+  const float qa = bf16_lo(*reinterpret_cast<const uint16_t *>(q_tile + (da >> 4) * XGROUP_BYTES + sw32_offset(r, e)));
+  const float qb =
+      bf16_lo(*reinterpret_cast<const uint16_t *>(q_tile + (db >> 4) * XGROUP_BYTES + sw32_offset(r, db & 15)));
+  // key k of the sub-tile at 32k + (chunk position) + 2 (e & 7); the chunk
+  // position flips with bit 2 of k
+  const uint8_t *ka0 = k_tile + (da >> 4) * XGROUP_BYTES + 2 * (e & 7) + 16 * (e >> 3);
+  const uint8_t *ka1 = k_tile + (da >> 4) * XGROUP_BYTES + 2 * (e & 7) + 16 * ((e >> 3) ^ 1);
+  const uint32_t gap = static_cast<uint32_t>((db >> 4) - (da >> 4)) * XGROUP_BYTES;  // half-split: dim b's group
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (__all_sync(FULL, cmin >= 16 * j + 16)) continue;
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      const int k = 16 * j + kk;
+      const uint8_t *pa = ((k >> 2) & 1 ? ka1 : ka0) + 32 * k;
+      float kav, kbv;
+      if (inter) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(pa);
+        kav = bf16_lo(w);
+        kbv = bf16_hi(w);
+      } else {
+        kav = bf16_lo(*reinterpret_cast<const uint16_t *>(pa));
+        kbv = bf16_lo(*reinterpret_cast<const uint16_t *>(pa + gap));
+      }
+      if (k >= cmin) su[k] = __float_as_uint(fmaf(qb, kbv, fmaf(qa, kav, __uint_as_float(su[k]))));
+    }
+  }
+}
+
+struct XBarriers {
+  uint64_t *q_full, *k_full, *k_empty, *k_ready, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *o_final, *drain;
+};
+
+template <int D>
+__global__ void __launch_bounds__(XTHREADS, 1)
+    prefill_exact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ ChannelPrefillArgs a) {
+  using L = XLayout<D>;
+  constexpr int G = L::G, C = D / 2;
+  constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, XSUB, false, false);
+  constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+  const bool inter = a.layout == WP_ROPE_INTERLEAVED;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+  XBarriers B;
+  B.q_full = bars;
+  B.k_full = bars + 1;
+  B.k_empty = B.k_full + XKST;
+  B.k_ready = B.k_empty + XKST;  // tile's plans and masked copies written
+  B.v_full = B.k_ready + XKST;
+  B.v_empty = B.v_full + XVST;
+  B.s_ready = B.v_empty + XVST;  // [2 heads][2 halves]
+  B.p_ready = B.s_ready + 4;     // [2 heads][2 halves]
+  B.o_ready = B.p_ready + 4;
+  B.o_final = B.o_ready + 2;
+  B.drain = B.o_final + 2;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
+  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
+  int32_t *cuts = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);    // [plan][64]
+  int32_t *gmax = reinterpret_cast<int32_t *>(smem + L::GMAX_OFF);   // [plan][8]
+  uint64_t *ring = reinterpret_cast<uint64_t *>(smem + L::RING_OFF);  // [stage][plan][half][2]
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  // Grid (head pair within its KV group, query block, KV head x batch), as in
+  // the grouped kernel.
+  const int rep = a.Hq / a.Hkv;
+  const int nslot = (rep % 2 == 0) ? 2 : 1;
+  const int hk = static_cast<int>(blockIdx.z) % a.Hkv;
+  const int b = static_cast<int>(blockIdx.z) / a.Hkv;
+  const int h0 = hk * rep + static_cast<int>(blockIdx.x) * nslot;  // head of slot s = h0 + s
+  const int nqb = (a.N + XBM - 1) / XBM;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.y);
+  const int64_t N = a.N;
+  // one plan (cutoff row, masked copies) for both slots, or one per slot
+  const int nplan = a.cut_rows == 1 ? 1 : nslot;
+  const long long lim = a.wait_limit;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = *reinterpret_cast<volatile int *>(&g_status) != 0 ? 1 : 0;
+    mbar_init(B.q_full, 1);
+    for (int s = 0; s < XKST; ++s) {
+      mbar_init(&B.k_full[s], 1);
+      mbar_init(&B.k_empty[s], 5 * nslot);  // per head: the MMA warp's commit and 4 softmax warps
+      mbar_init(&B.k_ready[s], 1);
+    }
+    for (int s = 0; s < XVST; ++s) {
+      mbar_init(&B.v_full[s], 1);
+      mbar_init(&B.v_empty[s], nslot);
+    }
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(&B.s_ready[s], 1);
+      mbar_init(&B.p_ready[s], 4);  // one arrival per softmax warp
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&B.o_ready[s], 1);
+      mbar_init(&B.o_final[s], 1);
+      mbar_init(&B.drain[s], 1);
+    }
+    fence_barrier_init();
+  }
+  for (int x = threadIdx.x; x < 2 * 64; x += XTHREADS) {
+    const int p = x / 64, c = x % 64;
+    cuts[x] = (c < C && p < nplan) ? a.cut[(a.cut_rows == 1 ? 0 : h0 + p) * C + c] : 0;
+  }
+  __syncthreads();
+  if (threadIdx.x < 2 * 8) {
+    const int p = threadIdx.x / 8, g = threadIdx.x % 8;
+    int32_t m = -1;
+    if (g < G && p < nplan)
+      for (uint64_t cm = group_chans<D>(g, inter); cm; cm &= cm - 1) m = max(m, cuts[64 * p + __ffsll(cm) - 1]);
+    gmax[threadIdx.x] = m;
+  }
+  if (warp == XMMA) {
+    tmem_alloc(tmem_base_slot, XTMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+  const int nkb = *abort_flag ? 0 : qb + 1;  // key tiles qb, qb-1, ..., 0
+  const int nsub = 2 * nkb;
+
+  if (warp == XPRODUCER) {
+    // ------------------------------------------------------------ producer
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(B.q_full, nslot * G * XGROUP_BYTES);
+      for (int s = 0; s < nslot; ++s)
+        for (int g = 0; g < G; ++g)
+          tma_load_4d(smem + L::Q_OFF + s * L::Q_SLOT + g * XGROUP_BYTES, &tm_q, B.q_full, 16 * g, h0 + s,
+                      qb * XBM, b);
+    }
+    __syncwarp();
+    int k_issued = 0, v_issued = 0;
+    bool ok = true;
+    auto load_v = [&](int t) -> bool {
+      const int st = t % XVST;
+      if (t >= XVST && !warp_wait(&B.v_empty[st], ((t / XVST) - 1) & 1, lim, abort_flag)) return false;
+      if (leader) {
+        mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * XV_CHUNK);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_4d(smem + L::V_OFF + st * L::V_STAGE + c * XV_CHUNK, &tm_v, &B.v_full[st], 64 * c, hk,
+                      (qb - t) * XBN, b);
+      }
+      __syncwarp();
+      ++v_issued;
+      return true;
+    };
+    for (int t = 0; ok && t < nkb; ++t) {
+      const int st = t % XKST;
+      if (t >= XKST && !warp_wait(&B.k_empty[st], ((t / XKST) - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      // groups holding a channel that either half does not skip, for either plan
+      uint32_t need = 0;
+      for (int hh = 0; hh < 2; ++hh) {
+        int64_t dmin, dmax;
+        if (!tile_distance_range(N, XBM, XSUB, qb, 2 * (qb - t) + hh, &dmin, &dmax)) continue;
+        for (int x = 0; x < 8 * nplan; ++x)
+          if (static_cast<int64_t>(gmax[x]) >= dmin) need |= 1u << (x % 8);
+      }
+      need &= (1u << G) - 1u;
+      if (leader) {
+        mbar_arrive_expect_tx(&B.k_full[st], __popc(need) * XGROUP_BYTES);
+        for (uint32_t m = need; m; m &= m - 1) {
+          const int g = __ffs(m) - 1;
+          tma_load_4d(smem + L::K_OFF + st * L::K_STAGE + g * XGROUP_BYTES, &tm_k, &B.k_full[st], 16 * g, hk,
+                      (qb - t) * XBN, b);
+        }
+      }
+      __syncwarp();
+      ++k_issued;
+      if (t >= 1) {
+        ok = load_v(t - 1);
+        if (!ok) break;
+      }
+      // the tile's plans, one lane per (plan, half), while K is in flight
+      uint64_t *rs = ring + st * 8;  // [plan][half][full, bnd]
+      if (lane < 2 * nplan) {
+        const int p = lane / 2, hh = lane % 2;
+        uint64_t f, bd;
+        make_plan<D>(cuts + 64 * p, inter, N, qb, 2 * (qb - t) + hh, f, bd);
+        rs[4 * p + 2 * hh] = f;
+        rs[4 * p + 2 * hh + 1] = bd;
+      }
+      __syncwarp();
+      if (!warp_wait(&B.k_full[st], (t / XKST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      // masked K copies of the partially kept groups, in ascending group order
+      for (int p = 0; p < nplan; ++p) {
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint64_t full = rs[4 * p + 2 * hh];
+          int nv = 0;
+          for (int g = 0; g < G && nv < NVAR; ++g) {
+            const uint32_t keep = group_keep<D>(full, g, inter);
+            if (keep == 0u || keep == 0xffffu) continue;
+            masked_k_copy(smem + L::KV_OFF + (((st * 2 + p) * 2 + hh) * NVAR + nv) * XHALF_BYTES,
+                          smem + L::K_OFF + st * L::K_STAGE + g * XGROUP_BYTES + hh * XHALF_BYTES, keep, lane);
+            ++nv;
+          }
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.k_ready[st]);
+    }
+    if (ok && nkb >= 1) ok = load_v(nkb - 1);
+    // Never leave a bulk copy in flight into shared memory this CTA is about
+    // to release: wait for Q and the last issued load of every stage.
+    warp_wait(B.q_full, 0, lim, nullptr);
+    for (int s = 0; s < XKST && s < k_issued; ++s) {
+      const int last = s + ((k_issued - 1 - s) / XKST) * XKST;
+      warp_wait(&B.k_full[s], (last / XKST) & 1, lim, nullptr);
+    }
+    for (int s = 0; s < XVST && s < v_issued; ++s) {
+      const int last = s + ((v_issued - 1 - s) / XVST) * XVST;
+      warp_wait(&B.v_full[s], (last / XVST) & 1, lim, nullptr);
+    }
+  } else if (warp >= XMMA && warp < XMMA + nslot) {
+    // ------------------------------------------------------- MMA issuers
+    const int s = warp - XMMA;
+    const int p = nplan == 1 ? 0 : s;
+    const bool leader = elect_one();
+    const uint64_t q_desc = smem_desc(smem_u32(smem + L::Q_OFF + s * L::Q_SLOT), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t k_desc = smem_desc(smem_u32(smem + L::K_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t kv_desc = smem_desc(smem_u32(smem + L::KV_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), XV_CHUNK, 1024, SMEM_SWIZZLE_128B);
+    bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
+    constexpr uint32_t GD = XGROUP_BYTES >> 4;  // one group tile in descriptor units
+
+    // QK of this head's sub-tile u into S half u & 1 (the tile's plans and
+    // copies are ready): plain groups against the K stage, partially kept
+    // groups against their masked copies, in ascending group order.
+    auto issue_qk = [&](int u) {
+      const int t = u >> 1, hh = u & 1, st = t % XKST;
+      const uint64_t full = ring[st * 8 + 4 * p + 2 * hh];
+      const uint32_t s_col = tmem + xcol_s(s) + XSUB * hh;
+      const uint64_t kst = k_desc + ((st * L::K_STAGE + hh * XHALF_BYTES) >> 4);
+      const uint64_t kvs = kv_desc + (((((st * 2 + p) * 2 + hh) * NVAR) * XHALF_BYTES) >> 4);
+      if (leader) {
+        uint32_t acc = 0;
+        int nv = 0;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const uint32_t keep = group_keep<D>(full, g, inter);
+          if (keep == 0xffffu) {
+            umma_ss(s_col, q_desc + g * GD, kst + g * GD, IDESC_QK, acc);
+            acc = 1;
+          } else if (keep != 0u && nv < NVAR) {
+            umma_ss(s_col, q_desc + g * GD, kvs + nv * (XHALF_BYTES >> 4), IDESC_QK, acc);
+            acc = 1;
+            ++nv;
+          }
+        }
+        umma_commit(&B.s_ready[2 * s + hh]);
+      }
+      __syncwarp();
+    };
+
+    if (ok && nkb > 0) {
+      ok = warp_wait(&B.k_ready[0], 0, lim, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+        issue_qk(1);
+        if (leader) umma_commit(&B.k_empty[0]);
+        __syncwarp();
+      }
+    }
+    for (int u = 0; ok && u < nsub; ++u) {
+      const int t = u >> 1, hh = u & 1;
+      const int vst = t % XVST;
+      if (hh == 0 && !warp_wait(&B.v_full[vst], (t / XVST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint64_t vst_desc = v_desc + ((vst * L::V_STAGE) >> 4);
+      if (!warp_wait(&B.p_ready[2 * s + hh], t & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t p_col = tmem + xcol_s(s) + XSUB * hh;
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < XSUB / 16; ++kk)
+          umma_ts(tmem + xcol_o(s), p_col + kk * 8, vst_desc + (hh * (XSUB / 16) + kk) * (2048 >> 4), IDESC_PV,
+                  (u > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&B.o_ready[s]);
+        if (u == nsub - 1) umma_commit(&B.o_final[s]);
+        if (hh == 1) umma_commit(&B.v_empty[vst]);
+      }
+      __syncwarp();
+      if (u + 2 < nsub) {
+        if (hh == 0) {
+          if (!warp_wait(&B.k_ready[(t + 1) % XKST], ((t + 1) / XKST) & 1, lim, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        issue_qk(u + 2);
+        if (hh == 1) {
+          if (leader) umma_commit(&B.k_empty[(t + 1) % XKST]);
+          __syncwarp();
+        }
+      }
+    }
+    if (leader) umma_commit(&B.drain[s]);
+    __syncwarp();
+    warp_wait(&B.drain[s], 0, lim, nullptr);
+  } else if (warp / 4 < nslot) {
+    // ------------------------------------------------------- softmax warps
+    const int slot = warp / 4;
+    const int q4 = warp % 4;
+    const int p = nplan == 1 ? 0 : slot;
+    const int r = q4 * 32 + lane;  // row of the query tile == TMEM lane
+    const int h = h0 + slot;
+    const int32_t *cut = cuts + 64 * p;
+    const uint8_t *q_tile = smem + L::Q_OFF + slot * L::Q_SLOT;
+    const int64_t i = static_cast<int64_t>(qb) * XBM + r;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t o_addr = lane_addr + xcol_o(slot);
+    const float c2 = a.scale_log2;
+    const uint64_t c2x2 = pack_f2(c2, c2);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = nsub == 0 || warp_wait(B.q_full, 0, lim, abort_flag);
+    for (int u = 0; ok && u < nsub; ++u) {
+      const int t = u >> 1, hh = u & 1, st = t % XKST;
+      const int64_t k0 = static_cast<int64_t>(qb - t) * XBN + XSUB * hh;
+      const uint32_t s_addr = lane_addr + xcol_s(slot) + XSUB * hh;
+      // the tile's plans (and, for the rank-2 updates, its K) are ready
+      if (hh == 0 && !warp_wait(&B.k_ready[st], (t / XKST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint64_t full = ring[st * 8 + 4 * p + 2 * hh], bnd = ring[st * 8 + 4 * p + 2 * hh + 1];
+      if (!warp_wait(&B.s_ready[2 * slot + hh], t & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t su[64];
+      load_half(s_addr, full != 0ull, su);
+      const uint8_t *k_tile = smem + L::K_OFF + st * L::K_STAGE + hh * XHALF_BYTES;
+      for (uint64_t m = bnd; m; m &= m - 1) {
+        const int c = __ffsll(static_cast<long long>(m)) - 1;
+        const int64_t cmin64 = i - k0 - cut[c];
+        const int cmin = cmin64 < 0 ? 0 : (cmin64 > XSUB ? XSUB : static_cast<int>(cmin64));
+        add_channel<D>(su, q_tile, k_tile, r, c, inter, cmin);
+      }
+      if (hh == 1) {  // this warp is done with tile t's K and plans
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&B.k_empty[st]);
+      }
+      if (t == 0) causal_mask(su, XSUB * hh, r);
+      const float m_half = half_max(su) * c2;
+      if (u == 0) {
+        m_run = m_half;
+      } else if (__any_sync(FULL, m_half > m_run + RESCALE_THRESHOLD)) {
+        const float m_new = fmaxf(m_run, m_half);
+        const float alpha = fast_exp2(m_run - m_new);
+        if (!warp_wait(&B.o_ready[slot], (u - 1) & 1, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        scale_cols_f32(o_addr, D / 32, alpha);
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      exp_half<true>(su, c2x2, m_run, acc, s_addr);
+      float s0, s1, s2, s3, s4, s5, s6, s7;
+      unpack_f2(acc[0], s0, s1);
+      unpack_f2(acc[1], s2, s3);
+      unpack_f2(acc[2], s4, s5);
+      unpack_f2(acc[3], s6, s7);
+      l_run += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.p_ready[2 * slot + hh]);
+    }
+    __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+    float *lse_at = a.lse == nullptr ? nullptr : a.lse + (static_cast<int64_t>(b) * a.Hq + h) * a.N + i;
+    if (ok && nsub > 0 && warp_wait(&B.o_final[slot], 0, lim, abort_flag)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t u32[32];
+        tmem_ld32(o_addr + 32 * c4, u32);
+        tmem_wait_ld(u32);
+        uint4 pk4[4];
+        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * inv_l, __uint_as_float(u32[2 * k + 1]) * inv_l);
+        if (i < N) {
+          uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
+        }
+      }
+      if (i < N && lse_at != nullptr) *lse_at = (m_run + log2f(l_run)) * 0.69314718055994531f;
+    } else {
+      *abort_flag = 1;
+      if (i < N) {
+        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) reinterpret_cast<uint4 *>(orow)[k] = nan4;
+        if (lse_at != nullptr) *lse_at = __int_as_float(0x7FC00000);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == XMMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, XTMEM_COLS);
+  }
+}
+
+template <int D>
+cudaError_t launch_exact(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const ChannelPrefillArgs &a, cudaStream_t stream) {
+  const int nqb = (a.N + XBM - 1) / XBM;
+  const int rep = a.Hq / a.Hkv;
+  const int nslot = rep % 2 == 0 ? 2 : 1;
+  const uint32_t smem = XLayout<D>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(prefill_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid(rep / nslot, nqb, a.Hkv * a.B);
+  prefill_exact_kernel<D><<<grid, XTHREADS, smem, stream>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_exact(int d_h, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                                 const ChannelPrefillArgs &a, cudaStream_t stream) {
+  return d_h == 128 ? launch_exact<128>(tq, tk, tv, a, stream) : launch_exact<64>(tq, tk, tv, a, stream);
+}
+
+}  // namespace wp

@@ -61,6 +61,10 @@ def _cut_table(kind, d, theta, layout, mode):
     if kind == "mixed":  # several distinct cutoffs inside one 128x128 tile
         base = np.array([0, 3, 130, 129, 50, 200, 255, 1000], dtype=np.int32)
         return np.resize(base, n)
+    if kind == "alternate":  # every group holds dropped and kept channels at every distance
+        return np.where(np.arange(n) % 2 == 0, 0, 2 ** 30).astype(np.int32)
+    if kind == "spread":  # a distinct cutoff per entry, many inside one 64-key sub-tile
+        return ((np.arange(n) * 37) % 301).astype(np.int32)
     raise ValueError(kind)
 
 
@@ -78,6 +82,10 @@ SMALL = [
     (190, 128, 6, 2, 1e4, wp.ROPE_HALF_SPLIT, "wave"),    # 3 query heads per KV head: one head per CTA;
                                                           # last tile of 62 rows (< one 64-key half)
     (200, 64, 6, 3, 1e4, wp.ROPE_INTERLEAVED, "mixed"),   # 2 per KV head; last tile of 72 rows
+    (400, 128, 2, 1, 1e4, wp.ROPE_INTERLEAVED, "alternate"),  # 8 partially kept groups per sub-tile
+    (400, 128, 2, 1, 1e4, wp.ROPE_HALF_SPLIT, "alternate"),
+    (333, 128, 2, 2, 1e6, wp.ROPE_HALF_SPLIT, "spread"),
+    (333, 64, 4, 2, 1e4, wp.ROPE_INTERLEAVED, "spread"),
 ]
 
 
@@ -96,41 +104,45 @@ def test_small_full_rows(N, d, Hq, Hkv, theta, layout, kind, mode):
     assert_attention_close(o, lse, ro, rl, f"N={N} d={d} {kind} mode={mode}")
 
 
-def _sampled_check(name, per_head):
+def _sampled_check(name, per_head, mode=wp.MODE_GROUPED):
     w = syn.workload(name)
     q, k, v = syn.prefill_inputs(w)
-    _, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
-    o, lse = _gpu_path(q, k, v, w.theta, w.layout, wg, wp.MODE_GROUPED, scale_all=w.scale_all)
+    wc, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
+    cut = wg if mode == wp.MODE_GROUPED else wc
+    o, lse = _gpu_path(q, k, v, w.theta, w.layout, cut, mode, scale_all=w.scale_all)
     rb, rh, ri = syn.sample_rows(w, per_head)
     # oracle: its own rotation of every key and of the sampled query rows
     kr = _oracle_rotated(k, w.theta, w.layout, w.scale_all)
     qrows = q[rb, ri, rh].unsqueeze(0).unsqueeze(2)            # [1, R, 1, d]
     qrot = oracle.rope(widen(qrows), w.theta, w.layout, pos=ri.numpy().reshape(1, -1), scale_all=w.scale_all)
     qrot = oracle.bf16_bits_to_f64(oracle.round_bf16_bits(qrot))[0, :, 0]
-    ro, rl = oracle.attention_rows(qrot, (rb.numpy(), rh.numpy(), ri.numpy()), kr, widen(v), w.Hq, wg,
-                                   oracle.MODE_GROUPED, w.layout)
+    ro, rl = oracle.attention_rows(qrot, (rb.numpy(), rh.numpy(), ri.numpy()), kr, widen(v), w.Hq, cut,
+                                   mode, w.layout)
     og = o[rb.cuda(), ri.cuda(), rh.cuda()]
     lg = lse[rb.cuda(), rh.cuda(), ri.cuda()]
-    return assert_attention_close(og, lg, ro, rl, name)
+    return assert_attention_close(og, lg, ro, rl, f"{name} mode={mode}")
 
 
-def test_qwen3_shaped_every_row():
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_qwen3_shaped_every_row(mode):
     """B2 H32/8 N4096 d128 theta 1e6 half-split, per-dim Q/K scales: every
     row of every head (262,144 rows) against the oracle, through the same
-    rope + prefill launches the bench times."""
+    rope + prefill launches the bench times; grouped and exact rule."""
     w = syn.workload("qwen3_8b_4k")
     q, k, v = syn.prefill_inputs(w)
-    _, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
-    o, lse = _gpu_path(q, k, v, w.theta, w.layout, wg, wp.MODE_GROUPED, scale_all=w.scale_all)
+    wc, wg = oracle.cutoffs(w.d, w.theta, w.layout, scale_all=w.scale_all)
+    cut = wg if mode == wp.MODE_GROUPED else wc
+    o, lse = _gpu_path(q, k, v, w.theta, w.layout, cut, mode, scale_all=w.scale_all)
     qr = _oracle_rotated(q, w.theta, w.layout, w.scale_all)
     kr = _oracle_rotated(k, w.theta, w.layout, w.scale_all)
-    ro, rl = oracle.attention(qr, kr, widen(v), wg, oracle.MODE_GROUPED, w.layout)
-    assert_attention_close(o, lse, ro, rl, "qwen3_8b_4k every row")
+    ro, rl = oracle.attention(qr, kr, widen(v), cut, mode, w.layout)
+    assert_attention_close(o, lse, ro, rl, f"qwen3_8b_4k every row mode={mode}")
 
 
-def test_long_32k_sampled_rows():
-    """B1 H32/8 N32768: 256 sampled rows per head."""
-    _sampled_check("long_32k", 256)
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_long_32k_sampled_rows(mode):
+    """B1 H32/8 N32768: 256 sampled rows per head; grouped and exact rule."""
+    _sampled_check("long_32k", 256, mode)
 
 
 def test_scaled_128k_sampled_rows():
