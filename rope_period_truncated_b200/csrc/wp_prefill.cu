@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     auto load_v = [&](int t) -> bool {
       const int st = t % VST;
-      if (t >= VST && !warp_wait(&B.v_empty[st], ((t / VST) - 1) & 1, lim, abort_flag)) return false;
+      if (t >= VST && !warp_wait_idle(&B.v_empty[st], ((t / VST) - 1) & 1, lim, abort_flag)) return false;
       const int krow = block_row(qb - t);
       if (leader) {
         mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * V_CHUNK_BYTES);
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     };
     for (int t = 0; ok && t < nkb; ++t) {
       const int st = t % KST;
-      if (t >= KST && !warp_wait(&B.k_empty[st], ((t / KST) - 1) & 1, lim, abort_flag)) {
+      if (t >= KST && !warp_wait_idle(&B.k_empty[st], ((t / KST) - 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
@@ -318,14 +318,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok && nkb >= 1) ok = load_v(nkb - 1);
     // Never leave a bulk copy in flight into shared memory this CTA is about
     // to release: wait for Q and the last issued load of every stage.
-    warp_wait(B.q_full, 0, lim, nullptr);
+    warp_wait_idle(B.q_full, 0, lim, nullptr);
     for (int s = 0; s < KST && s < k_issued; ++s) {
       const int last = s + ((k_issued - 1 - s) / KST) * KST;
-      warp_wait(&B.k_full[s], (last / KST) & 1, lim, nullptr);
+      warp_wait_idle(&B.k_full[s], (last / KST) & 1, lim, nullptr);
     }
     for (int s = 0; s < VST && s < v_issued; ++s) {
       const int last = s + ((v_issued - 1 - s) / VST) * VST;
-      warp_wait(&B.v_full[s], (last / VST) & 1, lim, nullptr);
+      warp_wait_idle(&B.v_full[s], (last / VST) & 1, lim, nullptr);
     }
   } else if (warp >= MMA_WARP && warp < MMA_WARP + nslot) {
     // ------------------------------------------------------- MMA issuers

@@ -56,6 +56,32 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, long l
   return __all_sync(FULL, ok);
 }
 
+// The same wait for a warp off the critical path (the TMA producer, the plan
+// warp): it polls and sleeps between polls, so that it takes no issue slots
+// from the softmax warps sharing its SM sub-partition while it waits.
+template <unsigned SLEEP_NS = 100>
+__device__ __forceinline__ bool warp_wait_idle(uint64_t *bar, uint32_t parity, long long lim,
+                                               volatile int *abort_flag) {
+  bool ok = true;
+  if (!mbar_test_wait(bar, parity)) {
+    const long long t0 = clock64();
+    while (!mbar_test_wait(bar, parity)) {
+      if (abort_flag != nullptr && *abort_flag) {
+        ok = false;
+        break;
+      }
+      if (clock64() - t0 > lim) {
+        record_status(WP_ERR_TIMEOUT);
+        if (abort_flag != nullptr) *abort_flag = 1;
+        ok = false;
+        break;
+      }
+      __nanosleep(SLEEP_NS);
+    }
+  }
+  return __all_sync(FULL, ok);
+}
+
 // 64 TMEM columns of this warp's lanes into r, with one wait for both loads;
 // the registers pass through the wait so no use moves above it.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {

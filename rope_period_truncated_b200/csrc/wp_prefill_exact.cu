@@ -16,17 +16,19 @@
 // boundary; then
 //   - a group whose channels are all full is one plain product;
 //   - a group with some full channels is one product against a copy of the
-//     sub-tile's K slice in which the dims of every other channel are zero
-//     (the producer writes the copy once the tile lands, in the TMA layout,
-//     fenced for the tensor core's async proxy; with one cutoff table both
-//     heads use it);
+//     head's Q slice in which the dims of every other channel are zero. The
+//     kept set of a group only changes when a channel's cutoff crosses the
+//     tile's distance range, so the head's MMA warp keeps a few such copies
+//     in shared memory (TMA layout, fenced for the tensor core's async
+//     proxy) and writes a new one only when a new (group, kept set) appears;
 //   - a boundary channel's product is rank 2, q_a k_a^T + q_b k_b^T: the
 //     softmax threads add it to their row of S with CUDA-core FMAs, only at
 //     the keys within W_c of the row, reading Q and K from the tiles the TMA
-//     loads already hold (so a K stage is free again once the MMAs and the
-//     softmax warps of both heads are done with it).
-// The producer also works out each key tile's channel plan (per head when
-// the heads have their own cutoffs) into a two-entry ring beside the K stages.
+//     loads already hold (so a K stage with boundary work is free again once
+//     the softmax warps are done with it too).
+// A plan warp writes each key tile's channel plan (per head when the heads
+// have their own cutoffs) into a two-entry ring beside the K stages, ahead of
+// the data.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -45,14 +47,16 @@ constexpr int XBN = 128;  // key tile of the K/V loads
 constexpr int XSUB = 64;  // key sub-tile of one S buffer
 constexpr int XKST = 2;
 constexpr int XVST = 2;
-constexpr int XTHREADS = 352;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9/10 MMA issuer of head 0/1
+constexpr int XTHREADS = 384;  // warps 0-7 softmax (2 heads), 8 TMA producer, 9/10 MMA issuer of head 0/1, 11 tile plans
 constexpr int XPRODUCER = 8;
 constexpr int XMMA = 9;
+constexpr int XFINISH = 11;
 constexpr uint32_t XTMEM_COLS = 512;
 constexpr uint32_t XGROUP_BYTES = 128 * 32;  // 128 rows x 16 bf16
 constexpr uint32_t XHALF_BYTES = 64 * 32;    // the 64 keys of one sub-tile
 constexpr uint32_t XV_CHUNK = 128 * 128;     // 128 keys x 64 bf16
-constexpr int NVAR = 2;  // masked K copies per (plan, sub-tile): partially kept groups
+constexpr int NVAR = 2;    // partially kept groups per sub-tile (masked Q products)
+constexpr int QSLOTS = 4;  // masked Q copies kept per head: NVAR for the MMAs in flight, NVAR new
 
 __host__ __device__ constexpr uint32_t xcol_s(int slot) { return 256u * slot; }
 __host__ __device__ constexpr uint32_t xcol_o(int slot) { return 256u * slot + 128u; }
@@ -66,10 +70,10 @@ struct XLayout {
   static constexpr uint32_t K_STAGE = G * XGROUP_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + XKST * K_STAGE;
   static constexpr uint32_t V_STAGE = (D / 64) * XV_CHUNK;
-  // masked K copies [stage][plan][half][NVAR], 2 KB each
-  static constexpr uint32_t KV_OFF = V_OFF + XVST * V_STAGE;
-  static constexpr uint32_t BAR_OFF = KV_OFF + XKST * 2 * 2 * NVAR * XHALF_BYTES;
-  // q_full, k_full/empty/ready, v_full/empty, per head x half s_ready/p_ready,
+  // masked Q copies [head][QSLOTS], one group tile each
+  static constexpr uint32_t QV_OFF = V_OFF + XVST * V_STAGE;
+  static constexpr uint32_t BAR_OFF = QV_OFF + 2 * QSLOTS * XGROUP_BYTES;
+  // q_full, k_full/empty/plan, v_full/empty, per head x half s_ready/p_ready,
   // per head o_ready/o_final/drain
   static constexpr uint32_t NUM_BARS = 1 + 3 * XKST + 2 * XVST + 2 * 4 + 2 * 3;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
@@ -103,23 +107,24 @@ __device__ __forceinline__ uint64_t group_chans(int g, bool inter) {
   return inter ? 0xffull << (8 * g) : 0xffffull << (16 * (g % (D / 32)));
 }
 
-// Channel plan of the 128-query x 64-key block (qb, kb64): `full` channels go
-// to plain or partial-group products on the tensor cores, `bnd` channels to
-// masked rank-2 updates. At most NVAR groups get a masked K copy; the full
-// channels of further partial groups move to `bnd`, where their mask keeps
-// every key (W_c >= dmax).
+// Channel plan of the 128-query x 64-key block (qb, kb64), warp-wide: lane l
+// classifies channels l and l + 32, and two ballots per class gather the
+// masks. `full` channels go to plain or partial-group products on the tensor
+// cores, `bnd` channels to masked rank-2 updates. At most NVAR groups get a
+// masked K copy; the full channels of further partial groups move to `bnd`,
+// where their mask keeps every key (W_c >= dmax).
 template <int D>
-__device__ void make_plan(const int32_t *cut, bool inter, int64_t N, int64_t qb, int64_t kb64, uint64_t &full,
-                          uint64_t &bnd) {
+__device__ __forceinline__ void make_plan(const int32_t *cut, bool inter, int64_t N, int64_t qb, int64_t kb64,
+                                          int lane, uint64_t &full, uint64_t &bnd) {
   constexpr int C = D / 2, G = D / 16;
   full = bnd = 0;
   int64_t dmin = 0, dmax = -1;
-  if (!tile_distance_range(N, XBM, XSUB, qb, kb64, &dmin, &dmax)) return;
-  for (int c = 0; c < C; ++c) {
-    const int cls = classify_cutoff(dmin, dmax, cut[c]);
-    if (cls == TILE_FULL) full |= 1ull << c;
-    if (cls == TILE_BOUNDARY) bnd |= 1ull << c;
-  }
+  if (!tile_distance_range(N, XBM, XSUB, qb, kb64, &dmin, &dmax)) return;  // the same in every lane
+  const int k0 = classify_cutoff(dmin, dmax, cut[lane]);
+  const int k1 = lane + 32 < C ? classify_cutoff(dmin, dmax, cut[lane + 32]) : TILE_SKIP;
+  full = __ballot_sync(FULL, k0 == TILE_FULL) | (static_cast<uint64_t>(__ballot_sync(FULL, k1 == TILE_FULL)) << 32);
+  bnd = __ballot_sync(FULL, k0 == TILE_BOUNDARY) |
+        (static_cast<uint64_t>(__ballot_sync(FULL, k1 == TILE_BOUNDARY)) << 32);
   int nvar = 0;
   for (int g = 0; g < G; ++g) {
     const uint32_t keep = group_keep<D>(full, g, inter);
@@ -136,12 +141,13 @@ __device__ void make_plan(const int32_t *cut, bool inter, int64_t N, int64_t qb,
   }
 }
 
-// Warp-wide: copy the 64-key K half tile at `src` to `dst` (both 256-byte
+// Warp-wide: copy the 128-row Q group tile at `src` to `dst` (both 256-byte
 // aligned, so the TMA 32-byte swizzle is the same), keeping the dims whose bit
-// in `keep` is set and zeroing the rest. Row r's logical 16-byte chunk q sits
-// at position q ^ ((r >> 2) & 1); lane l always moves chunks of logical index
+// in `keep` is set and zeroing the rest; then fence the copy for the tensor
+// core's async proxy. Row r's logical 16-byte chunk q sits at position
+// q ^ ((r >> 2) & 1); lane l always moves chunks of logical index
 // (l & 1) ^ ((l >> 3) & 1).
-__device__ __forceinline__ void masked_k_copy(uint8_t *dst, const uint8_t *src, uint32_t keep, int lane) {
+__device__ __forceinline__ void masked_q_copy(uint8_t *dst, const uint8_t *src, uint32_t keep, int lane) {
   const int q = (lane & 1) ^ ((lane >> 3) & 1);
   const uint32_t m8 = (keep >> (8 * q)) & 0xffu;
   uint32_t wm[4];
@@ -149,7 +155,7 @@ __device__ __forceinline__ void masked_k_copy(uint8_t *dst, const uint8_t *src, 
   for (int e = 0; e < 4; ++e)
     wm[e] = ((m8 >> (2 * e)) & 1u ? 0x0000ffffu : 0u) | ((m8 >> (2 * e + 1)) & 1u ? 0xffff0000u : 0u);
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
+  for (int it = 0; it < 8; ++it) {
     const int x = it * 32 + lane;  // 16-byte chunk index
     uint4 v = *reinterpret_cast<const uint4 *>(src + 16 * x);
     v.x &= wm[0];
@@ -158,6 +164,8 @@ __device__ __forceinline__ void masked_k_copy(uint8_t *dst, const uint8_t *src, 
     v.w &= wm[3];
     *reinterpret_cast<uint4 *>(dst + 16 * x) = v;
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
 }
 
 // Byte offset of (row, dim) in a 128-row x 16-dim bf16 tile stored with the
@@ -172,10 +180,11 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // Adds channel c's logits to this row's 64 S columns at the keys k >= cmin:
 // S[k] += q_a k_a[k] + q_b k_b[k]. q_tile: the head's Q tile of group 0;
 // k_tile: the K stage's group-0 tile advanced to the sub-tile's first key.
-// Column chunks of 16 keys that every lane masks are skipped.
+// Column chunks of 16 keys that every lane masks (k < cmin) or that lie
+// past every lane's causal limit (k > kmax) are skipped.
 template <int D>
 __device__ __forceinline__ void add_channel(uint32_t (&su)[64], const uint8_t *q_tile, const uint8_t *k_tile, int r,
-                                            int c, bool inter, int cmin) {
+                                            int c, bool inter, int cmin, int kmax) {
   constexpr int C = D / 2;
   const int da = inter ? 2 * c : c, db = inter ? 2 * c + 1 : c + C;
   const int e = da & 15;
@@ -189,7 +198,7 @@ __device__ __forceinline__ void add_channel(uint32_t (&su)[64], const uint8_t *q
   const uint32_t gap = static_cast<uint32_t>((db >> 4) - (da >> 4)) * XGROUP_BYTES;  // half-split: dim b's group
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    if (__all_sync(FULL, cmin >= 16 * j + 16)) continue;
+    if (__all_sync(FULL, cmin >= 16 * j + 16 || kmax < 16 * j)) continue;
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
       const int k = 16 * j + kk;
@@ -209,7 +218,7 @@ __device__ __forceinline__ void add_channel(uint32_t (&su)[64], const uint8_t *q
 }
 
 struct XBarriers {
-  uint64_t *q_full, *k_full, *k_empty, *k_ready, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *o_final, *drain;
+  uint64_t *q_full, *k_full, *k_empty, *k_plan, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *o_final, *drain;
 };
 
 template <int D>
@@ -229,8 +238,8 @@ __global__ void __launch_bounds__(XTHREADS, 1)
   B.q_full = bars;
   B.k_full = bars + 1;
   B.k_empty = B.k_full + XKST;
-  B.k_ready = B.k_empty + XKST;  // tile's plans and masked copies written
-  B.v_full = B.k_ready + XKST;
+  B.k_plan = B.k_empty + XKST;  // the tile's plans are in the ring
+  B.v_full = B.k_plan + XKST;
   B.v_empty = B.v_full + XVST;
   B.s_ready = B.v_empty + XVST;  // [2 heads][2 halves]
   B.p_ready = B.s_ready + 4;     // [2 heads][2 halves]
@@ -265,7 +274,7 @@ __global__ void __launch_bounds__(XTHREADS, 1)
     for (int s = 0; s < XKST; ++s) {
       mbar_init(&B.k_full[s], 1);
       mbar_init(&B.k_empty[s], 5 * nslot);  // per head: the MMA warp's commit and 4 softmax warps
-      mbar_init(&B.k_ready[s], 1);
+      mbar_init(&B.k_plan[s], 1);
     }
     for (int s = 0; s < XVST; ++s) {
       mbar_init(&B.v_full[s], 1);
@@ -307,6 +316,9 @@ __global__ void __launch_bounds__(XTHREADS, 1)
 
   if (warp == XPRODUCER) {
     // ------------------------------------------------------------ producer
+    // Q of both heads once; per key tile the K slices of the groups some
+    // channel of either half (either plan) does not skip, then V one tile
+    // behind. It never waits for a load to land, so two stay in flight.
     const bool leader = elect_one();
     if (leader) {
       tma_prefetch_desc(&tm_q);
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(XTHREADS, 1)
     bool ok = true;
     auto load_v = [&](int t) -> bool {
       const int st = t % XVST;
-      if (t >= XVST && !warp_wait(&B.v_empty[st], ((t / XVST) - 1) & 1, lim, abort_flag)) return false;
+      if (t >= XVST && !warp_wait_idle(&B.v_empty[st], ((t / XVST) - 1) & 1, lim, abort_flag)) return false;
       if (leader) {
         mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * XV_CHUNK);
         for (int c = 0; c < D / 64; ++c)
@@ -336,11 +348,10 @@ __global__ void __launch_bounds__(XTHREADS, 1)
     };
     for (int t = 0; ok && t < nkb; ++t) {
       const int st = t % XKST;
-      if (t >= XKST && !warp_wait(&B.k_empty[st], ((t / XKST) - 1) & 1, lim, abort_flag)) {
+      if (t >= XKST && !warp_wait_idle(&B.k_empty[st], ((t / XKST) - 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
-      // groups holding a channel that either half does not skip, for either plan
       uint32_t need = 0;
       for (int hh = 0; hh < 2; ++hh) {
         int64_t dmin, dmax;
@@ -359,53 +370,39 @@ __global__ void __launch_bounds__(XTHREADS, 1)
       }
       __syncwarp();
       ++k_issued;
-      if (t >= 1) {
-        ok = load_v(t - 1);
-        if (!ok) break;
-      }
-      // the tile's plans, one lane per (plan, half), while K is in flight
-      uint64_t *rs = ring + st * 8;  // [plan][half][full, bnd]
-      if (lane < 2 * nplan) {
-        const int p = lane / 2, hh = lane % 2;
-        uint64_t f, bd;
-        make_plan<D>(cuts + 64 * p, inter, N, qb, 2 * (qb - t) + hh, f, bd);
-        rs[4 * p + 2 * hh] = f;
-        rs[4 * p + 2 * hh + 1] = bd;
-      }
-      __syncwarp();
-      if (!warp_wait(&B.k_full[st], (t / XKST) & 1, lim, abort_flag)) {
-        ok = false;
-        break;
-      }
-      // masked K copies of the partially kept groups, in ascending group order
-      for (int p = 0; p < nplan; ++p) {
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint64_t full = rs[4 * p + 2 * hh];
-          int nv = 0;
-          for (int g = 0; g < G && nv < NVAR; ++g) {
-            const uint32_t keep = group_keep<D>(full, g, inter);
-            if (keep == 0u || keep == 0xffffu) continue;
-            masked_k_copy(smem + L::KV_OFF + (((st * 2 + p) * 2 + hh) * NVAR + nv) * XHALF_BYTES,
-                          smem + L::K_OFF + st * L::K_STAGE + g * XGROUP_BYTES + hh * XHALF_BYTES, keep, lane);
-            ++nv;
-          }
-        }
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&B.k_ready[st]);
+      if (t >= 1) ok = load_v(t - 1);
     }
     if (ok && nkb >= 1) ok = load_v(nkb - 1);
     // Never leave a bulk copy in flight into shared memory this CTA is about
     // to release: wait for Q and the last issued load of every stage.
-    warp_wait(B.q_full, 0, lim, nullptr);
+    warp_wait_idle(B.q_full, 0, lim, nullptr);
     for (int s = 0; s < XKST && s < k_issued; ++s) {
       const int last = s + ((k_issued - 1 - s) / XKST) * XKST;
-      warp_wait(&B.k_full[s], (last / XKST) & 1, lim, nullptr);
+      warp_wait_idle(&B.k_full[s], (last / XKST) & 1, lim, nullptr);
     }
     for (int s = 0; s < XVST && s < v_issued; ++s) {
       const int last = s + ((v_issued - 1 - s) / XVST) * XVST;
-      warp_wait(&B.v_full[s], (last / XVST) & 1, lim, nullptr);
+      warp_wait_idle(&B.v_full[s], (last / XVST) & 1, lim, nullptr);
+    }
+  } else if (warp == XFINISH) {
+    // ------------------------------------------------------------ plan warp
+    // Per key tile the channel plan of each (plan, half), once the tile two
+    // back has released the ring entry (the stage's k_empty).
+    for (int t = 0; t < nkb; ++t) {
+      const int st = t % XKST;
+      if (t >= XKST && !warp_wait_idle(&B.k_empty[st], ((t / XKST) - 1) & 1, lim, abort_flag)) break;
+      uint64_t *rs = ring + st * 8;  // [plan][half][full, bnd]
+      for (int p = 0; p < nplan; ++p)
+        for (int hh = 0; hh < 2; ++hh) {
+          uint64_t f, bd;
+          make_plan<D>(cuts + 64 * p, inter, N, qb, 2 * (qb - t) + hh, lane, f, bd);
+          if (lane == 0) {
+            rs[4 * p + 2 * hh] = f;
+            rs[4 * p + 2 * hh + 1] = bd;
+          }
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&B.k_plan[st]);
     }
   } else if (warp >= XMMA && warp < XMMA + nslot) {
     // ------------------------------------------------------- MMA issuers
@@ -414,44 +411,121 @@ __global__ void __launch_bounds__(XTHREADS, 1)
     const bool leader = elect_one();
     const uint64_t q_desc = smem_desc(smem_u32(smem + L::Q_OFF + s * L::Q_SLOT), 16, 256, SMEM_SWIZZLE_32B);
     const uint64_t k_desc = smem_desc(smem_u32(smem + L::K_OFF), 16, 256, SMEM_SWIZZLE_32B);
-    const uint64_t kv_desc = smem_desc(smem_u32(smem + L::KV_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    uint8_t *qv = smem + L::QV_OFF + s * QSLOTS * XGROUP_BYTES;
+    const uint64_t qv_desc = smem_desc(smem_u32(qv), 16, 256, SMEM_SWIZZLE_32B);
     const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), XV_CHUNK, 1024, SMEM_SWIZZLE_128B);
     bool ok = warp_wait(B.q_full, 0, lim, abort_flag);
     constexpr uint32_t GD = XGROUP_BYTES >> 4;  // one group tile in descriptor units
+    // The masked Q copies: slot j holds group (skey[j] >> 16) with kept dims
+    // (skey[j] & 0xffff) and was last read by QK(suse[j]). QK(u) may
+    // overwrite a slot unless QK(u - 1) reads it (QK(u - 2) and earlier have
+    // completed: the softmax consumed their S before P(u - 2) freed the half
+    // for u).
+    uint32_t skey[QSLOTS];
+    int suse[QSLOTS];
+#pragma unroll
+    for (int j = 0; j < QSLOTS; ++j) {
+      skey[j] = 0xffffffffu;
+      suse[j] = -4;
+    }
+    // copy slot of a partially kept group's key for QK(u), writing the copy
+    // on a miss
+    auto slot_for = [&](uint32_t key, int u) -> int {
+      int found = -1;
+#pragma unroll
+      for (int j = 0; j < QSLOTS; ++j)
+        if (skey[j] == key) found = j;
+      if (found < 0) {
+#pragma unroll
+        for (int j = QSLOTS - 1; j >= 0; --j)
+          if (suse[j] < u - 1) found = j;
+        found = found < 0 ? 0 : found;  // never: at most NVAR slots are in use by QK(u - 1)
+        masked_q_copy(qv + found * XGROUP_BYTES, smem + L::Q_OFF + s * L::Q_SLOT + (key >> 16) * XGROUP_BYTES,
+                      key & 0xffffu, lane);
+#pragma unroll
+        for (int j = 0; j < QSLOTS; ++j)
+          if (j == found) skey[j] = key;
+      }
+#pragma unroll
+      for (int j = 0; j < QSLOTS; ++j)
+        if (j == found) suse[j] = u;
+      return found;
+    };
 
-    // QK of this head's sub-tile u into S half u & 1 (the tile's plans and
-    // copies are ready): plain groups against the K stage, partially kept
-    // groups against their masked copies, in ascending group order.
+    // QK of this head's sub-tile u into S half u & 1 (the tile's K and plans
+    // are in): plain groups from Q, partially kept groups from masked copies.
     auto issue_qk = [&](int u) {
       const int t = u >> 1, hh = u & 1, st = t % XKST;
       const uint64_t full = ring[st * 8 + 4 * p + 2 * hh];
       const uint32_t s_col = tmem + xcol_s(s) + XSUB * hh;
       const uint64_t kst = k_desc + ((st * L::K_STAGE + hh * XHALF_BYTES) >> 4);
-      const uint64_t kvs = kv_desc + (((((st * 2 + p) * 2 + hh) * NVAR) * XHALF_BYTES) >> 4);
+      // plain groups, and the partially kept ones (at most NVAR, as the
+      // plan allows) with their kept dims: key = group << 16 | kept
+      uint32_t plain = 0;
+      uint32_t pkey0 = 0, pkey1 = 0;
+      int npart = 0;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const uint32_t keep = group_keep<D>(full, g, inter);
+        if (keep == 0xffffu) {
+          plain |= 1u << g;
+        } else if (keep != 0u && npart < NVAR) {
+          const uint32_t key = (static_cast<uint32_t>(g) << 16) | keep;
+          if (npart == 0) pkey0 = key;
+          else pkey1 = key;
+          ++npart;
+        }
+      }
+      // descriptors of the partially kept groups' products, broadcast from
+      // lane 0 so that they are warp-uniform values
+      uint64_t pa0 = 0, pb0 = 0, pa1 = 0, pb1 = 0;
+      if (npart > 0) {
+        pa0 = qv_desc + slot_for(pkey0, u) * GD;
+        pb0 = kst + (pkey0 >> 16) * GD;
+      }
+      if (npart > 1) {
+        pa1 = qv_desc + slot_for(pkey1, u) * GD;
+        pb1 = kst + (pkey1 >> 16) * GD;
+      }
+      if (npart > 0) {
+        pa0 = __shfl_sync(FULL, pa0, 0);
+        pb0 = __shfl_sync(FULL, pb0, 0);
+        pa1 = __shfl_sync(FULL, pa1, 0);
+        pb1 = __shfl_sync(FULL, pb1, 0);
+      }
       if (leader) {
+        // The plain groups first, with descriptors at fixed offsets from
+        // loop-invariant bases (this issue loop is the MMA warp's hot path),
+        // then the few partially kept ones from their copy slots.
         uint32_t acc = 0;
-        int nv = 0;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          const uint32_t keep = group_keep<D>(full, g, inter);
-          if (keep == 0xffffu) {
+          if ((plain >> g) & 1u) {
             umma_ss(s_col, q_desc + g * GD, kst + g * GD, IDESC_QK, acc);
             acc = 1;
-          } else if (keep != 0u && nv < NVAR) {
-            umma_ss(s_col, q_desc + g * GD, kvs + nv * (XHALF_BYTES >> 4), IDESC_QK, acc);
-            acc = 1;
-            ++nv;
           }
         }
+        if (npart > 0) {
+          umma_ss(s_col, pa0, pb0, IDESC_QK, acc);
+          acc = 1;
+        }
+        if (npart > 1) umma_ss(s_col, pa1, pb1, IDESC_QK, acc);
         umma_commit(&B.s_ready[2 * s + hh]);
       }
       __syncwarp();
     };
+    // a key tile's K and plans
+    auto tile_in = [&](int t) -> bool {
+      const int st = t % XKST;
+      if (!warp_wait(&B.k_full[st], (t / XKST) & 1, lim, abort_flag)) return false;
+      if (!warp_wait(&B.k_plan[st], (t / XKST) & 1, lim, abort_flag)) return false;
+      tc_fence_after();
+      return true;
+    };
 
     if (ok && nkb > 0) {
-      ok = warp_wait(&B.k_ready[0], 0, lim, abort_flag);
+      ok = tile_in(0);
       if (ok) {
-        tc_fence_after();
         issue_qk(0);
         issue_qk(1);
         if (leader) umma_commit(&B.k_empty[0]);
@@ -483,12 +557,9 @@ __global__ void __launch_bounds__(XTHREADS, 1)
       }
       __syncwarp();
       if (u + 2 < nsub) {
-        if (hh == 0) {
-          if (!warp_wait(&B.k_ready[(t + 1) % XKST], ((t + 1) / XKST) & 1, lim, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        if (hh == 0 && !tile_in(t + 1)) {
+          ok = false;
+          break;
         }
         issue_qk(u + 2);
         if (hh == 1) {
@@ -516,16 +587,36 @@ __global__ void __launch_bounds__(XTHREADS, 1)
     const uint64_t c2x2 = pack_f2(c2, c2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = nsub == 0 || warp_wait(B.q_full, 0, lim, abort_flag);
+    uint64_t full1 = 0, bnd1 = 0;  // the plan of the tile's second half
+    bool hold = false;             // this warp still reads the tile's K stage
     for (int u = 0; ok && u < nsub; ++u) {
       const int t = u >> 1, hh = u & 1, st = t % XKST;
       const int64_t k0 = static_cast<int64_t>(qb - t) * XBN + XSUB * hh;
       const uint32_t s_addr = lane_addr + xcol_s(slot) + XSUB * hh;
-      // the tile's plans (and, for the rank-2 updates, its K) are ready
-      if (hh == 0 && !warp_wait(&B.k_ready[st], (t / XKST) & 1, lim, abort_flag)) {
-        ok = false;
-        break;
+      uint64_t full, bnd;
+      if (hh == 0) {
+        // both halves' plans; without boundary work the tile's stage and ring
+        // entry are released right away
+        if (!warp_wait(&B.k_plan[st], (t / XKST) & 1, lim, abort_flag)) {
+          ok = false;
+          break;
+        }
+        full = ring[st * 8 + 4 * p];
+        bnd = ring[st * 8 + 4 * p + 1];
+        full1 = ring[st * 8 + 4 * p + 2];
+        bnd1 = ring[st * 8 + 4 * p + 3];
+        hold = (bnd | bnd1) != 0ull;
+        if (!hold) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&B.k_empty[st]);
+        } else if (!warp_wait(&B.k_full[st], (t / XKST) & 1, lim, abort_flag)) {  // K read below
+          ok = false;
+          break;
+        }
+      } else {
+        full = full1;
+        bnd = bnd1;
       }
-      const uint64_t full = ring[st * 8 + 4 * p + 2 * hh], bnd = ring[st * 8 + 4 * p + 2 * hh + 1];
       if (!warp_wait(&B.s_ready[2 * slot + hh], t & 1, lim, abort_flag)) {
         ok = false;
         break;
@@ -534,13 +625,14 @@ __global__ void __launch_bounds__(XTHREADS, 1)
       uint32_t su[64];
       load_half(s_addr, full != 0ull, su);
       const uint8_t *k_tile = smem + L::K_OFF + st * L::K_STAGE + hh * XHALF_BYTES;
+      const int kmax = t == 0 ? r - XSUB * hh : XSUB - 1;  // last causal key column of this row
       for (uint64_t m = bnd; m; m &= m - 1) {
         const int c = __ffsll(static_cast<long long>(m)) - 1;
         const int64_t cmin64 = i - k0 - cut[c];
         const int cmin = cmin64 < 0 ? 0 : (cmin64 > XSUB ? XSUB : static_cast<int>(cmin64));
-        add_channel<D>(su, q_tile, k_tile, r, c, inter, cmin);
+        add_channel<D>(su, q_tile, k_tile, r, c, inter, cmin, kmax);
       }
-      if (hh == 1) {  // this warp is done with tile t's K and plans
+      if (hh == 1 && hold) {  // this warp is done with tile t's K
         __syncwarp();
         if (lane == 0) mbar_arrive(&B.k_empty[st]);
       }
