@@ -56,6 +56,7 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--no-exact", action="store_true", help="skip the exact per-channel prefill entry")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--kcache", choices=["group-major", "rows"], default="group-major",
                    help="layout of the decode K cache in HBM")
@@ -66,6 +67,8 @@ def parse_args():
                         "whole channels (the pages' grouping, Table 12 cutoffs)")
     p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                    help="restrict the step (profiling a single kernel)")
+    p.add_argument("--prefill-mode", choices=["grouped", "exact"], default="grouped",
+                   help="rule of the timed prefill in a restricted profiling case (--only prefill)")
     p.add_argument("--prefill-n", type=int, default=0,
                    help="override the prefill sequence length (smaller profiling case; not a bench line)")
     return p.parse_args()
@@ -172,6 +175,15 @@ def backward_flops(N, d, Hq, B, wg):
     return useful, dense
 
 
+def exact_flops(N, d, Hq, B, wc):
+    """Useful FLOPs of one exact-rule prefill, pair exact: per pair j <= i,
+    2*2 per channel with i-j <= W_c (its two dims) plus 2*d for PV."""
+    delta = np.arange(N, dtype=np.int64)
+    pairs = (N - delta).astype(np.float64)
+    active = (delta[:, None] <= np.asarray(wc, dtype=np.int64)[None, :]).sum(1)
+    return float((pairs * (2 * 2 * active + 2 * d)).sum()) * B * Hq
+
+
 def decode_required_bytes(lens, wg, B, Hq, Hkv, d):
     """K bytes of in-window groups (32 B per group per key) plus all of V,
     plus the query, output and LSE."""
@@ -252,10 +264,12 @@ class ClockSampler:
 class Path:
     """Device buffers and launches of one hot-path step."""
 
-    def __init__(self, device, prefill_n=0, kcache_layout="group-major", grouping="half-split", page_size=0):
+    def __init__(self, device, prefill_n=0, kcache_layout="group-major", grouping="half-split", page_size=0,
+                 prefill_mode="grouped"):
         import dataclasses
         import rope_period_truncated_b200 as wp
         self.wp = wp
+        self.prefill_mode = prefill_mode
         self.pw = syn.workload("long_32k")
         if prefill_n:
             self.pw = dataclasses.replace(self.pw, N=prefill_n)
@@ -272,7 +286,7 @@ class Path:
         paired = grouping == "paired" and pw.layout == wp.ROPE_HALF_SPLIT
         self.rope_layout = wp.ROPE_HALF_SPLIT_PAIRED if paired else pw.layout
         self.cut_layout = wp.ROPE_INTERLEAVED if paired else pw.layout
-        _, self.wg = wp.wp_cutoffs(pw.d, pw.theta, self.cut_layout, scale_all=pw.scale_all)
+        self.wc, self.wg = wp.wp_cutoffs(pw.d, pw.theta, self.cut_layout, scale_all=pw.scale_all)
         dq, kc, vc, lens = syn.decode_inputs(dw)
         self.host_decode = (dq, lens)
         self.dq = dq.to(device).reshape(dw.B, 1, dw.Hq, dw.d)
@@ -321,8 +335,15 @@ class Path:
         return self.prefill_only(cut)
 
     def prefill_only(self, cut="wave"):
+        if self.prefill_mode == "exact" and cut == "wave":
+            return self.prefill_exact_only()
         return self.wp.wp_prefill(self.qr, self.kr, self.v, self.wg if cut == "wave" else None,
                                   self.wp.MODE_GROUPED, self.cut_layout, out=self.o, lse=self.lse)
+
+    def prefill_exact_only(self):
+        """The same prefill under the exact per-channel rule."""
+        return self.wp.wp_prefill(self.qr, self.kr, self.v, self.wc, self.wp.MODE_CHANNEL, self.cut_layout,
+                                  out=self.o, lse=self.lse)
 
     def decode(self, cut="wave"):
         wp, dw = self.wp, self.dw
@@ -488,7 +509,9 @@ def run_ours(args, rank, world, local):
     wpbuild.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    path = Path(dev, args.prefill_n, args.kcache, args.grouping, args.page_size)
+    if args.prefill_mode != "grouped" and args.only != "prefill":
+        raise SystemExit("--prefill-mode exact is a profiling case of --only prefill")
+    path = Path(dev, args.prefill_n, args.kcache, args.grouping, args.page_size, args.prefill_mode)
     peaks, peak_kind = load_peaks()
     do_prefill = args.only in ("all", "prefill")
     do_decode = args.only in ("all", "decode")
@@ -615,6 +638,22 @@ def run_ours(args, rank, world, local):
         del dout, dq, dk, dv
         path.prefill()  # the wave forward's outputs again
 
+    # the same 32K prefill under the exact per-channel rule (wp_prefill, MODE_CHANNEL)
+    exact = None
+    if args.only == "all" and not args.no_exact:
+        path.rope_prefill()
+        ex_flops = exact_flops(pw.N, pw.d, pw.Hq, pw.B, path.wc)
+        ex_ms = statistics.median(time_kernel(path.prefill_exact_only, 3, 1) for _ in range(3))
+        ex_ms = max_over_ranks([ex_ms], dev)[0]
+        exact = {"kernel": "wp_prefill, exact per-channel rule (tcgen05 products of full and partially kept "
+                           "groups, rank-2 updates of boundary channels)",
+                 "ms": round(ex_ms, 3), "grouped_ms": round(prefill_ms, 3),
+                 "useful_tflops": round(ex_flops / (ex_ms * 1e-3) / 1e12, 2), "useful_flops": ex_flops,
+                 "peak": peaks["bf16_tflops"],
+                 "frac": round(ex_flops / (ex_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                 "note": "useful FLOPs pair exact: 4 per kept channel per pair (its two dims) + 2*d for PV"}
+        path.prefill()  # the grouped forward's outputs again
+
     # end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e and args.only == "all":
@@ -677,6 +716,7 @@ def run_ours(args, rank, world, local):
                   "kernel_ms": round(rope_ms, 5), "bytes_per_step": rope_bytes} if do_prefill else None),
         "dense_comparison": dense,
         "backward": backward,
+        "exact": exact,
         "e2e": e2e,
         "gpu_launches": {"all": 6, "prefill": 3, "decode": 3}[args.only] * K,
         "clocks": clk,

@@ -66,6 +66,21 @@ def test_backward_flops_match_enumeration(N):
     assert dense == tot_dense * 2 * 3
 
 
+@pytest.mark.parametrize("N", [1, 130, 400])
+def test_exact_flops_match_enumeration(N):
+    """Per causal pair: 2*2 per channel with i-j <= W_c (its two dims) and
+    2*d for PV; every channel kept gives the dense causal count."""
+    d = 64
+    wc = [0, 3, 7, 130, 131, 1000] + [2 ** 31 - 1] * (d // 2 - 6)
+    tot = 0
+    for i in range(N):
+        for j in range(i + 1):
+            tot += 2 * 2 * sum(1 for w in wc if i - j <= w) + 2 * d
+    assert bench.exact_flops(N, d, 2, 3, wc) == tot * 2 * 3
+    dense = sum(4 * d for i in range(N) for j in range(i + 1)) * 2 * 3
+    assert bench.exact_flops(N, d, 2, 3, [2 ** 31 - 1] * (d // 2)) == dense
+
+
 def test_decode_required_bytes_match_enumeration():
     rng = np.random.default_rng(3)
     lens = rng.integers(1, 400, size=5)
