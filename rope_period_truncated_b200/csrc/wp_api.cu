@@ -64,15 +64,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 4-D bf16 view (d, H, N, B) of a [B, N, H, d] tensor; box (box_d, 1, 128, 1).
-bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int d, int box_d, CUtensorMapSwizzle sw) {
+// 4-D bf16 view (d, H, N, B) of a [B, N, H, d] tensor; box (box_d, 1, box_rows, 1).
+bool make_map(CUtensorMap *m, const void *base, int B, int N, int H, int d, int box_d, CUtensorMapSwizzle sw,
+              int box_rows = 128) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(N),
                         static_cast<cuuint64_t>(B)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(H) * d * 2,
                            static_cast<cuuint64_t>(N) * H * d * 2};
-  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, 128, 1};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -325,7 +326,16 @@ int wp_prefill_backward(const void *q, const void *k, const void *v, const void 
   }
   a.scale = scale;
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
-  return from_cuda(launch_backward(d_h, a, static_cast<cudaStream_t>(stream)));
+  a.wait_limit = g_wait_limit;
+  if ((N + 127) / 128 > 65535) return WP_ERR_UNSUPPORTED;
+  BackwardMaps m;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_map(&m.q128, q, B, N, H_q, d_h, 16, sw, 128) || !make_map(&m.do128, dout, B, N, H_q, d_h, 16, sw, 128) ||
+      !make_map(&m.k64, k, B, N, H_kv, d_h, 16, sw, 64) || !make_map(&m.v64, v, B, N, H_kv, d_h, 16, sw, 64) ||
+      !make_map(&m.k128, k, B, N, H_kv, d_h, 16, sw, 128) || !make_map(&m.v128, v, B, N, H_kv, d_h, 16, sw, 128) ||
+      !make_map(&m.q64, q, B, N, H_q, d_h, 16, sw, 64) || !make_map(&m.do64, dout, B, N, H_q, d_h, 16, sw, 64))
+    return WP_ERR_CUDA;
+  return from_cuda(launch_backward(d_h, a, m, static_cast<cudaStream_t>(stream)));
 }
 
 size_t wp_decode_workspace_bytes(int B, int H_q, int d_h, int Lmax) {

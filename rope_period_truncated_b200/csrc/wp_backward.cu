@@ -522,27 +522,20 @@ __global__ void __launch_bounds__(BWD_THREADS) dkdv_kernel(const __grid_constant
 }
 
 template <int D>
-cudaError_t launch(const BackwardArgs &a, cudaStream_t stream) {
+cudaError_t launch(const BackwardArgs &a, const BackwardMaps &maps, cudaStream_t stream) {
   const int64_t rows = static_cast<int64_t>(a.B) * a.N * a.Hq;
   delta_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), BWD_THREADS, 0, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, DqSmem<D>::BYTES);
+  e = launch_backward_dq_tc(D, a, maps, stream);
   if (e != cudaSuccess) return e;
-  dq_kernel<D><<<dim3((a.N + DQ_BQ - 1) / DQ_BQ, a.Hq, a.B), BWD_THREADS, DqSmem<D>::BYTES, stream>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const uint32_t kv_bytes = KvSmem<D>::bytes(a.Hq / a.Hkv);
-  e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kv_bytes));
-  if (e != cudaSuccess) return e;
-  dkdv_kernel<D><<<dim3((a.N + KV_BK - 1) / KV_BK, a.Hkv, a.B), BWD_THREADS, kv_bytes, stream>>>(a);
-  return cudaGetLastError();
+  return launch_backward_dkdv_tc(D, a, maps, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_backward(int d_h, const BackwardArgs &a, cudaStream_t stream) {
-  return d_h == 128 ? launch<128>(a, stream) : launch<64>(a, stream);
+cudaError_t launch_backward(int d_h, const BackwardArgs &a, const BackwardMaps &maps, cudaStream_t stream) {
+  return d_h == 128 ? launch<128>(a, maps, stream) : launch<64>(a, maps, stream);
 }
 
 }  // namespace wp

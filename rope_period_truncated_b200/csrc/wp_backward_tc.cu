@@ -1,0 +1,990 @@
+// WavePrune grouped-cutoff causal prefill backward on sm_100a: TMA + tcgen05 + TMEM.
+//
+// What it computes (WavePrune reading notes "WavePrune：RoPE 通常只需一个旋转
+// 周期", §2.1 Eq. (6), §2.3 Eq. (8) and §2.3's paragraph on the backward
+// kernel): with P_ij = exp(L_ij - LSE_i) from the forward's LSE and
+// D_i = <dO_i, O_i>,
+//   dS_ij   = P_ij (<dO_i, V_j> - D_i),
+//   dQ_i[g] = scale * sum_j 1[i - j <= W_g] dS_ij K_j[g]   (16-dim group g),
+// and (the key-major kernel) dV_j = sum_i P_ij dO_i, dK_j[g] likewise with Q.
+// In the backward the head dimension is the output axis of the dQ and dK
+// products, so the group mask goes on the gradient operand dS before the
+// product: full groups take dS as it is, skipped groups nothing, a boundary
+// group dS masked by its own cutoff.
+//
+// dq_tc_kernel: one CTA per (128-row query block, query head). It walks the
+// 64-key sub-tiles from the diagonal backwards (u = 0, 1, ...; distances
+// grow with u). Warp roles:
+//   warp 4   TMA producer: Q and dO of the block once (16-dim boxes, 32-byte
+//            swizzle); per sub-tile the K group tiles some group needs and V,
+//            three stages.
+//   warp 5   MMA issuer: S(u) = sum_g Q_g K_g^T (M128 N64 K16 per non-skipped
+//            group) and dP(u) = dO V^T into double-buffered TMEM, then, once
+//            the row warps have written dS(u) (bf16, over S's first 32
+//            columns), dQ[g0:g1] += dS K[g0:g1] for each run of consecutive
+//            full groups as M128 N16*(g1-g0) K16 products with dS read from
+//            TMEM and K read MN-major from the same swizzled group tiles.
+//   warps 0-3 one thread per query row: P, dS = P (dP - D), dS to TMEM; the
+//            epilogue scales dQ and writes it as bf16.
+// Boundary groups (cutoff inside the sub-tile's distance range), as in the
+// forward kernel: their S products go first, one cutoff class at a time in
+// ascending order, and the row warps mask S in place after each (nested
+// windows: the exact per-group mask). For dQ the classes go in descending
+// order: before each class's products the row warps overwrite dS in TMEM
+// with dS masked by that class's cutoff. Both are round trips between the
+// MMA warp and the row warps, so the MMA warp issues S(v) of a sub-tile with
+// boundary classes only after it has issued dQ(v - 1) (a sub-tile without
+// them is issued two ahead): the row warps finish sub-tile v - 1 before they
+// mask S(v), and the MMA warp never waits on them for a later sub-tile.
+//
+// dkdv_tc_kernel: one CTA per (128-row key block, KV head), the same roles
+// with keys as rows: K and V of the block once; per 64-query sub-tile (the
+// KV head's query heads one after another, each from the diagonal outwards)
+// Q, dO and their LSE and D. S^T = K Q^T and dP^T = V dO^T on the tensor
+// cores, P^T and dS^T per key row, then dV += P^T dO (N = d) and
+// dK[g0:g1] += dS^T Q[g0:g1] per run of full groups; the query heads of the
+// KV head add into the same TMEM accumulators, so nothing is reduced across
+// CTAs. Boundary classes as above, with the window on the query columns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "wp_backward.h"
+#include "wp_device.cuh"
+#include "wp_prefill_common.cuh"
+#include "wp_tile.h"
+
+namespace wp {
+
+namespace {
+
+constexpr int TBQ = 128;  // rows of a CTA's block
+constexpr int TBS = 64;   // columns of a sub-tile
+constexpr int TNST = 3;   // stages of the streamed operands
+constexpr int TC_THREADS = 192;
+constexpr int T_PROD = 4, T_MMA = 5;
+constexpr uint32_t TILE128 = 128 * 32;  // a 16-dim group tile of 128 rows
+constexpr uint32_t TILE64 = 64 * 32;    // a 16-dim group tile of 64 rows
+constexpr float TLOG2E = 1.4426950408889634f;
+
+// TMEM columns of the dQ kernel
+constexpr uint32_t DQ_S = 0;     // S / dS of buffer b at 64 b
+constexpr uint32_t DQ_DP = 128;  // dP of buffer b at 128 + 64 b
+constexpr uint32_t DQ_ACC = 256;
+
+template <int D>
+struct DqTL {
+  static constexpr int G = D / 16;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t DO_OFF = Q_OFF + G * TILE128;
+  static constexpr uint32_t K_OFF = DO_OFF + G * TILE128;
+  static constexpr uint32_t STAGE = G * TILE64;
+  static constexpr uint32_t V_OFF = K_OFF + TNST * STAGE;
+  static constexpr uint32_t BAR_OFF = V_OFF + TNST * STAGE;
+  // qd_full, kv_full[TNST], kv_empty[TNST], s_ready[2], ds_ready[2],
+  // bnd_ready, bnd_done, dsm_req, dsm_done, dq_final, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // the head's group cutoffs, 8 int32
+  static constexpr uint32_t BYTES = CUT_OFF + 32 + 1024;
+};
+
+// Group classes of a 128-row x 64-column block whose causal pairs span
+// distances [dmin, dmax] (any = it has causal pairs): full and boundary bits.
+struct SubPlan {
+  uint32_t full, bnd;
+  bool any;
+};
+__device__ __forceinline__ SubPlan sub_plan(const int32_t *cut, int G, bool any, int64_t dmin, int64_t dmax) {
+  SubPlan p{0u, 0u, any};
+  if (any) {
+    for (int g = 0; g < G; ++g) {
+      const int c = classify_cutoff(dmin, dmax, cut[g]);
+      if (c == TILE_FULL) p.full |= 1u << g;
+      if (c == TILE_BOUNDARY) p.bnd |= 1u << g;
+    }
+  }
+  return p;
+}
+
+// Largest cutoff among the boundary groups in `bnd` that is < prev (prev =
+// INT64_MAX for the first); false when none. `mask` gets the groups of it.
+__device__ __forceinline__ bool prev_boundary_class(const int32_t *cut, uint32_t bnd, int64_t prev, int32_t *W,
+                                                    uint32_t *mask) {
+  int64_t best = -1;
+  for (uint32_t m = bnd; m; m &= m - 1) {
+    const int64_t w = cut[__ffs(m) - 1];
+    if (w < prev && w > best) best = w;
+  }
+  if (best < 0) return false;
+  uint32_t mk = 0;
+  for (uint32_t m = bnd; m; m &= m - 1) {
+    const int g = __ffs(m) - 1;
+    if (static_cast<int64_t>(cut[g]) == best) mk |= 1u << g;
+  }
+  *W = static_cast<int32_t>(best);
+  *mask = mk;
+  return true;
+}
+
+// dS (fp32, 64 columns) as bf16 pairs into 32 TMEM columns, columns c < cmin zeroed.
+__device__ __forceinline__ void store_ds(uint32_t taddr, const float (&ds)[64], int cmin) {
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    pk[k] = pack_bf16x2(2 * k < cmin ? 0.f : ds[2 * k], 2 * k + 1 < cmin ? 0.f : ds[2 * k + 1]);
+  tmem_st32(taddr, pk);
+}
+
+template <int D>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const __grid_constant__ BackwardArgs a) {
+  using L = DqTL<D>;
+  constexpr int G = L::G;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, TBS, false, false);
+  constexpr uint32_t GD128 = TILE128 >> 4, GD64 = TILE64 >> 4;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+  uint64_t *qd_full = bars;
+  uint64_t *kv_full = bars + 1;
+  uint64_t *kv_empty = kv_full + TNST;
+  uint64_t *s_ready = kv_empty + TNST;  // [2 buffers]
+  uint64_t *ds_ready = s_ready + 2;     // [2 buffers]
+  uint64_t *bnd_ready = ds_ready + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
+  uint64_t *dq_final = dsm_done + 1, *drain = dq_final + 1;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
+  int32_t *cut = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (a.Hq / a.Hkv);
+  const int nqb = (a.N + TBQ - 1) / TBQ;
+  const int qb = nqb - 1 - static_cast<int>(blockIdx.x);  // heaviest blocks first
+  const int64_t N = a.N;
+  const long long lim = a.wait_limit;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = *reinterpret_cast<volatile int *>(&g_status) != 0 ? 1 : 0;
+    mbar_init(qd_full, 1);
+    for (int s = 0; s < TNST; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_ready[s], 1);
+      mbar_init(&ds_ready[s], 4);
+    }
+    mbar_init(bnd_ready, 1);
+    mbar_init(bnd_done, 4);
+    mbar_init(dsm_req, 1);
+    mbar_init(dsm_done, 4);
+    mbar_init(dq_final, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (threadIdx.x < 8) cut[threadIdx.x] = threadIdx.x < G ? a.cut[(a.cut_rows == 1 ? 0 : h) * G + threadIdx.x] : 0;
+  if (warp == T_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nsub = *abort_flag ? 0 : 2 * (qb + 1);  // key sub-tile 2qb + 1 - u
+  // the plan of sub-tile u
+  auto plan_of = [&](int u) -> SubPlan {
+    int64_t dmin = 0, dmax = -1;
+    const bool any = tile_distance_range(N, TBQ, TBS, qb, 2 * qb + 1 - u, &dmin, &dmax);
+    return sub_plan(cut, G, any, dmin, dmax);
+  };
+
+  if (warp == T_PROD) {
+    // ------------------------------------------------------------ producer
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(qd_full, 2 * G * TILE128);
+      for (int g = 0; g < G; ++g) {
+        tma_load_4d(smem + L::Q_OFF + g * TILE128, &tm_q, qd_full, 16 * g, h, qb * TBQ, b);
+        tma_load_4d(smem + L::DO_OFF + g * TILE128, &tm_do, qd_full, 16 * g, h, qb * TBQ, b);
+      }
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int u = 0; u < nsub; ++u) {
+      const int st = u % TNST;
+      if (u >= TNST && !warp_wait_idle(&kv_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
+      // a sub-tile without causal pairs (past the end of a ragged last block)
+      // loads nothing: its dS is 0 whatever the buffers hold
+      const SubPlan pl = plan_of(u);
+      const uint32_t need = pl.full | pl.bnd;
+      const int nv = pl.any ? G : 0;
+      const int krow = (2 * qb + 1 - u) * TBS;
+      if (leader) {
+        mbar_arrive_expect_tx(&kv_full[st], (__popc(need) + nv) * TILE64);
+        for (uint32_t m = need; m; m &= m - 1) {
+          const int g = __ffs(m) - 1;
+          tma_load_4d(smem + L::K_OFF + st * L::STAGE + g * TILE64, &tm_k, &kv_full[st], 16 * g, hk, krow, b);
+        }
+        for (int g = 0; g < nv; ++g)
+          tma_load_4d(smem + L::V_OFF + st * L::STAGE + g * TILE64, &tm_v, &kv_full[st], 16 * g, hk, krow, b);
+      }
+      __syncwarp();
+      ++issued;
+    }
+    warp_wait_idle(qd_full, 0, lim, nullptr);
+    for (int s = 0; s < TNST && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / TNST) * TNST;
+      warp_wait_idle(&kv_full[s], (last / TNST) & 1, lim, nullptr);
+    }
+  } else if (warp == T_MMA) {
+    // -------------------------------------------------------- MMA issuer
+    const bool leader = elect_one();
+    const uint64_t q_desc = smem_desc(smem_u32(smem + L::Q_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t do_desc = smem_desc(smem_u32(smem + L::DO_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t k_desc = smem_desc(smem_u32(smem + L::K_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    // K as the B operand of dQ += dS K: keys along K (8-row groups 256 B
+    // apart), dims along N (16-dim group tiles TILE64 apart)
+    const uint64_t kmn_desc = smem_desc(smem_u32(smem + L::K_OFF), TILE64, 256, SMEM_SWIZZLE_32B);
+    bool ok = warp_wait(qd_full, 0, lim, abort_flag);
+    int bnd_cnt = 0, dsm_cnt = 0;
+
+    // S(u) and dP(u) into buffer u & 1
+    auto issue_sdp = [&](int u) -> bool {
+      const int st = u % TNST, bf = u & 1;
+      if (!warp_wait(&kv_full[st], (u / TNST) & 1, lim, abort_flag)) return false;
+      tc_fence_after();
+      const SubPlan pl = plan_of(u);
+      const uint32_t s_col = tmem + DQ_S + 64 * bf;
+      const uint64_t kst = k_desc + ((st * L::STAGE) >> 4);
+      uint32_t acc = 0;
+      if (pl.bnd) {
+        int64_t prev = -1;
+        int32_t W;
+        uint32_t cls;
+        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+          if (leader) {
+            for (int g = 0; g < G; ++g)
+              if ((cls >> g) & 1u) {
+                umma_ss(s_col, q_desc + g * GD128, kst + g * GD64, IDESC_S, acc);
+                acc = 1;
+              }
+            umma_commit(bnd_ready);
+          }
+          acc = 1;
+          __syncwarp();
+          if (!warp_wait(bnd_done, bnd_cnt & 1, lim, abort_flag)) return false;
+          tc_fence_after();
+          ++bnd_cnt;
+          prev = W;
+        }
+      }
+      if (leader) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          if ((pl.full >> g) & 1u) {
+            umma_ss(s_col, q_desc + g * GD128, kst + g * GD64, IDESC_S, acc);
+            acc = 1;
+          }
+        const uint64_t vst = v_desc + ((st * L::STAGE) >> 4);
+        if (pl.any) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            umma_ss(tmem + DQ_DP + 64 * bf, do_desc + g * GD128, vst + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_ready[bf]);
+      }
+      __syncwarp();
+      return true;
+    };
+    // dQ[groups] += dS(u) K[groups], one product set per run of consecutive groups
+    auto issue_dq_groups = [&](int u, uint32_t groups) {
+      const int st = u % TNST, bf = u & 1;
+      const uint64_t kst = kmn_desc + ((st * L::STAGE) >> 4);
+      while (groups) {
+        const int g0 = __ffs(groups) - 1;
+        int g1 = g0;
+        while (g1 < G && ((groups >> g1) & 1u)) ++g1;
+        groups &= ~(((1u << g1) - 1u) & ~((1u << g0) - 1u));
+        const uint32_t idesc = idesc_bf16_f32(128, 16 * (g1 - g0), false, true);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < TBS / 16; ++kk)
+            umma_ts(tmem + DQ_ACC + 16 * g0, tmem + DQ_S + 64 * bf + kk * 8,
+                    kst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
+        }
+        __syncwarp();
+      }
+    };
+    // dQ(u): full groups on dS as it is, then the boundary classes in
+    // descending cutoff order, each after the row warps masked dS for it
+    auto issue_dq = [&](int u) -> bool {
+      const SubPlan pl = plan_of(u);
+      issue_dq_groups(u, pl.full);
+      int64_t prev = INT64_MAX;
+      int32_t W;
+      uint32_t cls;
+      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        if (leader) umma_commit(dsm_req);
+        __syncwarp();
+        if (!warp_wait(dsm_done, dsm_cnt & 1, lim, abort_flag)) return false;
+        tc_fence_after();
+        ++dsm_cnt;
+        issue_dq_groups(u, cls);
+        prev = W;
+      }
+      if (leader) umma_commit(&kv_empty[u % TNST]);
+      __syncwarp();
+      return true;
+    };
+
+    // S of sub-tile v goes out two ahead, or one ahead when v has boundary
+    // classes (its handshakes must follow the row warps' finish of v - 1).
+    int next = 0;
+    auto advance = [&](int done) -> bool {
+      while (next < nsub && next <= done + 2) {
+        if (plan_of(next).bnd != 0u && next > done + 1) break;
+        if (!issue_sdp(next)) return false;
+        ++next;
+      }
+      return true;
+    };
+    if (ok) ok = advance(-1);
+    for (int u = 0; ok && u < nsub; ++u) {
+      if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      ok = issue_dq(u);
+      if (ok) ok = advance(u);
+    }
+    if (leader) {
+      umma_commit(dq_final);
+      umma_commit(drain);
+    }
+    __syncwarp();
+    warp_wait(drain, 0, lim, nullptr);
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- row warps
+    const int r = warp * 32 + lane;
+    const int64_t i = static_cast<int64_t>(qb) * TBQ + r;
+    const bool row_ok = i < N;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N + (row_ok ? i : 0);
+    const float lse2 = row_ok ? a.lse[lrow] * TLOG2E : 0.f;
+    const float di = row_ok ? a.delta[lrow] : 0.f;
+    const float c2 = a.scale_log2;
+    // zero the dQ accumulator: every dQ product accumulates
+    {
+      uint32_t z[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) z[k] = 0u;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) tmem_st32(lane_addr + DQ_ACC + 32 * c4, z);
+      tmem_wait_st();
+    }
+    int bnd_cnt = 0, dsm_cnt = 0;
+    bool ok = true;
+    for (int u = 0; ok && u < nsub; ++u) {
+      const int bf = u & 1;
+      const int64_t k0 = static_cast<int64_t>(2 * qb + 1 - u) * TBS;  // first key of the sub-tile
+      const uint32_t s_addr = lane_addr + DQ_S + 64 * bf;
+      const SubPlan pl = plan_of(u);
+      if (pl.bnd) {
+        // S masked in place after each boundary class: keep key c iff i - (k0 + c) <= W
+        int64_t prev = -1;
+        int32_t W;
+        uint32_t cls;
+        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+          ok = warp_wait(bnd_ready, bnd_cnt & 1, lim, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const int64_t cm = i - k0 - W;
+          const int cmin = cm < 0 ? 0 : (cm > TBS ? TBS : static_cast<int>(cm));
+          uint32_t su[64];
+          tmem_ld64(s_addr, su);
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c < cmin) su[c] = 0u;
+          tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+          tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bnd_done);
+          ++bnd_cnt;
+          prev = W;
+        }
+        if (!ok) break;
+      }
+      if (!warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t su[64], dp[64];
+      load_half(s_addr, (pl.full | pl.bnd) != 0u, su);
+      tmem_ld64(lane_addr + DQ_DP + 64 * bf, dp);
+      // P = exp2(S c2 - LSE log2 e) on the causal pairs of valid rows, dS = P (dP - D)
+      const int64_t jmax = i - k0;  // last causal key column
+      float ds[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const bool live = row_ok && c <= jmax;
+        const float p = fast_exp2(fmaf(__uint_as_float(su[c]), c2, -lse2));
+        ds[c] = live ? p * (__uint_as_float(dp[c]) - di) : 0.f;
+      }
+      store_ds(s_addr, ds, 0);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_ready[bf]);
+      // boundary classes of dQ, descending cutoffs: dS masked for each
+      int64_t prev = INT64_MAX;
+      int32_t W;
+      uint32_t cls;
+      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        ok = warp_wait(dsm_req, dsm_cnt & 1, lim, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const int64_t cm = i - k0 - W;
+        store_ds(s_addr, ds, cm < 0 ? 0 : (cm > TBS ? TBS : static_cast<int>(cm)));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dsm_done);
+        ++dsm_cnt;
+        prev = W;
+      }
+    }
+    __nv_bfloat16 *dqrow = a.dq + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+    if (ok && nsub > 0 && warp_wait(dq_final, 0, lim, abort_flag)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t u32[32];
+        tmem_ld32(lane_addr + DQ_ACC + 32 * c4, u32);
+        tmem_wait_ld(u32);
+        uint4 pk4[4];
+        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * a.scale, __uint_as_float(u32[2 * k + 1]) * a.scale);
+        if (row_ok) {
+          uint4 *dst = reinterpret_cast<uint4 *>(dqrow + 32 * c4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
+        }
+      }
+    } else {
+      *abort_flag = 1;
+      if (row_ok) {
+        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) reinterpret_cast<uint4 *>(dqrow)[k] = nan4;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == T_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// TMEM columns of the dK/dV kernel
+constexpr uint32_t KV_S = 0;     // S^T / P^T of buffer b at 64 b
+constexpr uint32_t KV_DP = 128;  // dP^T / dS^T of buffer b at 128 + 64 b
+constexpr uint32_t KV_DK = 256;
+template <int D>
+constexpr uint32_t kv_dv() {
+  return KV_DK + D;
+}
+
+template <int D>
+struct KvTL {
+  static constexpr int G = D / 16;
+  static constexpr uint32_t K_OFF = 0;
+  static constexpr uint32_t V_OFF = K_OFF + G * TILE128;
+  static constexpr uint32_t Q_OFF = V_OFF + G * TILE128;
+  static constexpr uint32_t STAGE = G * TILE64;
+  static constexpr uint32_t DO_OFF = Q_OFF + TNST * STAGE;
+  static constexpr uint32_t LD_OFF = DO_OFF + TNST * STAGE;  // per stage: LSE (log2 units) and D, 64 each
+  static constexpr uint32_t BAR_OFF = LD_OFF + TNST * 512;
+  // kv_full, qd_full[TNST], qd_empty[TNST], s_ready[2], ds_ready[2],
+  // bnd_ready, bnd_done, dsm_req, dsm_done, kv_final, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // cutoff rows of the KV head's query heads, [rep][8]
+  static constexpr uint32_t BYTES = CUT_OFF + 64 * 8 * 4 + 1024;
+};
+
+// dS^T (fp32, 64 query columns) as bf16 pairs into 32 TMEM columns, columns c > cmax zeroed.
+__device__ __forceinline__ void store_ds_upto(uint32_t taddr, const float (&ds)[64], int cmax) {
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    pk[k] = pack_bf16x2(2 * k > cmax ? 0.f : ds[2 * k], 2 * k + 1 > cmax ? 0.f : ds[2 * k + 1]);
+  tmem_st32(taddr, pk);
+}
+
+template <int D>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ BackwardArgs a) {
+  using L = KvTL<D>;
+  constexpr int G = L::G;
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, TBS, false, false);
+  constexpr uint32_t GD128 = TILE128 >> 4, GD64 = TILE64 >> 4;
+  constexpr uint32_t KV_DV = kv_dv<D>();
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+  uint64_t *kv_full = bars;
+  uint64_t *qd_full = bars + 1;
+  uint64_t *qd_empty = qd_full + TNST;
+  uint64_t *s_ready = qd_empty + TNST;  // [2 buffers]
+  uint64_t *ds_ready = s_ready + 2;     // [2 buffers]
+  uint64_t *bnd_ready = ds_ready + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
+  uint64_t *kv_final = dsm_done + 1, *drain = kv_final + 1;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
+  int32_t *cuts = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);  // [rep][8]
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int kb = static_cast<int>(blockIdx.x);  // key blocks near the start see the most queries: first
+  const int hk = blockIdx.y, b = blockIdx.z;
+  const int rep = a.Hq / a.Hkv;
+  const int64_t N = a.N;
+  const int nq64 = (a.N + TBS - 1) / TBS;
+  const int per_head = nq64 - 2 * kb;  // query sub-tiles 2kb .. nq64-1 of each head
+  const long long lim = a.wait_limit;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = *reinterpret_cast<volatile int *>(&g_status) != 0 ? 1 : 0;
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < TNST; ++s) {
+      mbar_init(&qd_full[s], 1);
+      mbar_init(&qd_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_ready[s], 1);
+      mbar_init(&ds_ready[s], 4);
+    }
+    mbar_init(bnd_ready, 1);
+    mbar_init(bnd_done, 4);
+    mbar_init(dsm_req, 1);
+    mbar_init(dsm_done, 4);
+    mbar_init(kv_final, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  for (int x = threadIdx.x; x < rep * 8; x += TC_THREADS) {
+    const int hr = x / 8, g = x % 8;
+    cuts[x] = g < G ? a.cut[(a.cut_rows == 1 ? 0 : hk * rep + hr) * G + g] : 0;
+  }
+  if (warp == T_MMA) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nsub = *abort_flag ? 0 : rep * per_head;
+  // sub-tile u: query head hk * rep + u / per_head, query rows 64 * (2kb + u % per_head) ..
+  auto head_of = [&](int u) { return u / per_head; };
+  auto q0_of = [&](int u) { return static_cast<int64_t>(2 * kb + u % per_head) * TBS; };
+  auto plan_of = [&](int u) -> SubPlan {
+    int64_t dmin = 0, dmax = -1;
+    const bool any = tile_distance_range(N, TBS, TBQ, 2 * kb + u % per_head, kb, &dmin, &dmax);
+    return sub_plan(cuts + 8 * head_of(u), G, any, dmin, dmax);
+  };
+
+  if (warp == T_PROD) {
+    // ------------------------------------------------------------ producer
+    const bool leader = elect_one();
+    if (leader) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(kv_full, 2 * G * TILE128);
+      for (int g = 0; g < G; ++g) {
+        tma_load_4d(smem + L::K_OFF + g * TILE128, &tm_k, kv_full, 16 * g, hk, kb * TBQ, b);
+        tma_load_4d(smem + L::V_OFF + g * TILE128, &tm_v, kv_full, 16 * g, hk, kb * TBQ, b);
+      }
+    }
+    __syncwarp();
+    int issued = 0;
+    for (int u = 0; u < nsub; ++u) {
+      const int st = u % TNST;
+      if (u >= TNST && !warp_wait_idle(&qd_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
+      const SubPlan pl = plan_of(u);
+      const uint32_t need = pl.full | pl.bnd;
+      const int h = hk * rep + head_of(u);
+      const int64_t q0 = q0_of(u);
+      // the sub-tile's LSE (log2 units) and D, read by the row warps
+      float *ld = reinterpret_cast<float *>(smem + L::LD_OFF + st * 512);
+      const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N;
+      for (int c = lane; c < TBS; c += 32) {
+        const bool in = q0 + c < N;
+        ld[c] = in ? a.lse[lrow + q0 + c] * TLOG2E : 0.f;
+        ld[TBS + c] = in ? a.delta[lrow + q0 + c] : 0.f;
+      }
+      __syncwarp();
+      if (leader) {
+        mbar_arrive_expect_tx(&qd_full[st], (__popc(need) + G) * TILE64);
+        for (uint32_t m = need; m; m &= m - 1) {
+          const int g = __ffs(m) - 1;
+          tma_load_4d(smem + L::Q_OFF + st * L::STAGE + g * TILE64, &tm_q, &qd_full[st], 16 * g, h,
+                      static_cast<int>(q0), b);
+        }
+        for (int g = 0; g < G; ++g)
+          tma_load_4d(smem + L::DO_OFF + st * L::STAGE + g * TILE64, &tm_do, &qd_full[st], 16 * g, h,
+                      static_cast<int>(q0), b);
+      }
+      __syncwarp();
+      ++issued;
+    }
+    warp_wait_idle(kv_full, 0, lim, nullptr);
+    for (int s = 0; s < TNST && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / TNST) * TNST;
+      warp_wait_idle(&qd_full[s], (last / TNST) & 1, lim, nullptr);
+    }
+  } else if (warp == T_MMA) {
+    // -------------------------------------------------------- MMA issuer
+    const bool leader = elect_one();
+    const uint64_t k_desc = smem_desc(smem_u32(smem + L::K_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t v_desc = smem_desc(smem_u32(smem + L::V_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t q_desc = smem_desc(smem_u32(smem + L::Q_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    const uint64_t do_desc = smem_desc(smem_u32(smem + L::DO_OFF), 16, 256, SMEM_SWIZZLE_32B);
+    // Q and dO as the B operands of the dK and dV products: queries along K,
+    // dims along N (16-dim group tiles TILE64 apart)
+    const uint64_t qmn_desc = smem_desc(smem_u32(smem + L::Q_OFF), TILE64, 256, SMEM_SWIZZLE_32B);
+    const uint64_t domn_desc = smem_desc(smem_u32(smem + L::DO_OFF), TILE64, 256, SMEM_SWIZZLE_32B);
+    bool ok = warp_wait(kv_full, 0, lim, abort_flag);
+    int bnd_cnt = 0, dsm_cnt = 0;
+
+    auto issue_sdp = [&](int u) -> bool {
+      const int st = u % TNST, bf = u & 1;
+      if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag)) return false;
+      tc_fence_after();
+      const SubPlan pl = plan_of(u);
+      const int32_t *cut = cuts + 8 * head_of(u);
+      const uint32_t s_col = tmem + KV_S + 64 * bf;
+      const uint64_t qst = q_desc + ((st * L::STAGE) >> 4);
+      uint32_t acc = 0;
+      if (pl.bnd) {
+        int64_t prev = -1;
+        int32_t W;
+        uint32_t cls;
+        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+          if (leader) {
+            for (int g = 0; g < G; ++g)
+              if ((cls >> g) & 1u) {
+                umma_ss(s_col, k_desc + g * GD128, qst + g * GD64, IDESC_S, acc);
+                acc = 1;
+              }
+            umma_commit(bnd_ready);
+          }
+          acc = 1;
+          __syncwarp();
+          if (!warp_wait(bnd_done, bnd_cnt & 1, lim, abort_flag)) return false;
+          tc_fence_after();
+          ++bnd_cnt;
+          prev = W;
+        }
+      }
+      if (leader) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          if ((pl.full >> g) & 1u) {
+            umma_ss(s_col, k_desc + g * GD128, qst + g * GD64, IDESC_S, acc);
+            acc = 1;
+          }
+        const uint64_t dost = do_desc + ((st * L::STAGE) >> 4);
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          umma_ss(tmem + KV_DP + 64 * bf, v_desc + g * GD128, dost + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
+        umma_commit(&s_ready[bf]);
+      }
+      __syncwarp();
+      return true;
+    };
+    // dK[groups] += dS^T Q[groups], one product set per run of consecutive groups
+    auto issue_dk_groups = [&](int u, uint32_t groups) {
+      const int st = u % TNST, bf = u & 1;
+      const uint64_t qst = qmn_desc + ((st * L::STAGE) >> 4);
+      while (groups) {
+        const int g0 = __ffs(groups) - 1;
+        int g1 = g0;
+        while (g1 < G && ((groups >> g1) & 1u)) ++g1;
+        groups &= ~(((1u << g1) - 1u) & ~((1u << g0) - 1u));
+        const uint32_t idesc = idesc_bf16_f32(128, 16 * (g1 - g0), false, true);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < TBS / 16; ++kk)
+            umma_ts(tmem + KV_DK + 16 * g0, tmem + KV_DP + 64 * bf + kk * 8,
+                    qst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
+        }
+        __syncwarp();
+      }
+    };
+    // dV(u), then dK(u): full groups on dS^T as it is, then the boundary
+    // classes in descending cutoff order, each after the row warps masked dS^T
+    auto issue_dkdv = [&](int u) -> bool {
+      const int st = u % TNST, bf = u & 1;
+      const SubPlan pl = plan_of(u);
+      const int32_t *cut = cuts + 8 * head_of(u);
+      if (leader) {
+        constexpr uint32_t IDESC_DV = idesc_bf16_f32(128, D, false, true);
+        const uint64_t dost = domn_desc + ((st * L::STAGE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < TBS / 16; ++kk)
+          umma_ts(tmem + KV_DV, tmem + KV_S + 64 * bf + kk * 8, dost + ((kk * 16 * 32) >> 4), IDESC_DV, 1u);
+      }
+      __syncwarp();
+      issue_dk_groups(u, pl.full);
+      int64_t prev = INT64_MAX;
+      int32_t W;
+      uint32_t cls;
+      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        if (leader) umma_commit(dsm_req);
+        __syncwarp();
+        if (!warp_wait(dsm_done, dsm_cnt & 1, lim, abort_flag)) return false;
+        tc_fence_after();
+        ++dsm_cnt;
+        issue_dk_groups(u, cls);
+        prev = W;
+      }
+      if (leader) umma_commit(&qd_empty[st]);
+      __syncwarp();
+      return true;
+    };
+
+    int next = 0;
+    auto advance = [&](int done) -> bool {
+      while (next < nsub && next <= done + 2) {
+        if (plan_of(next).bnd != 0u && next > done + 1) break;
+        if (!issue_sdp(next)) return false;
+        ++next;
+      }
+      return true;
+    };
+    if (ok) ok = advance(-1);
+    for (int u = 0; ok && u < nsub; ++u) {
+      if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      ok = issue_dkdv(u);
+      if (ok) ok = advance(u);
+    }
+    if (leader) {
+      umma_commit(kv_final);
+      umma_commit(drain);
+    }
+    __syncwarp();
+    warp_wait(drain, 0, lim, nullptr);
+  } else if (warp < 4) {
+    // ---------------------------------------------------------- row warps
+    const int r = warp * 32 + lane;
+    const int64_t j = static_cast<int64_t>(kb) * TBQ + r;  // this thread's key
+    const bool row_ok = j < N;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c2 = a.scale_log2;
+    {
+      uint32_t z[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) z[k] = 0u;
+#pragma unroll
+      for (int c4 = 0; c4 < 2 * D / 32; ++c4) tmem_st32(lane_addr + KV_DK + 32 * c4, z);
+      tmem_wait_st();
+    }
+    int bnd_cnt = 0, dsm_cnt = 0;
+    bool ok = true;
+    for (int u = 0; ok && u < nsub; ++u) {
+      const int st = u % TNST, bf = u & 1;
+      const int64_t q0 = q0_of(u);
+      const uint32_t s_addr = lane_addr + KV_S + 64 * bf, dp_addr = lane_addr + KV_DP + 64 * bf;
+      const SubPlan pl = plan_of(u);
+      const int32_t *cut = cuts + 8 * head_of(u);
+      if (pl.bnd) {
+        // S^T masked in place after each boundary class: keep query c iff (q0 + c) - j <= W
+        int64_t prev = -1;
+        int32_t W;
+        uint32_t cls;
+        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+          ok = warp_wait(bnd_ready, bnd_cnt & 1, lim, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const int64_t cm = j - q0 + W;
+          const int cmax = cm < -1 ? -1 : (cm > TBS - 1 ? TBS - 1 : static_cast<int>(cm));
+          uint32_t su[64];
+          tmem_ld64(s_addr, su);
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c > cmax) su[c] = 0u;
+          tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
+          tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bnd_done);
+          ++bnd_cnt;
+          prev = W;
+        }
+        if (!ok) break;
+      }
+      // the sub-tile's LSE and D (the producer wrote them before its loads)
+      if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag) ||
+          !warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512);
+      uint32_t su[64], dp[64];
+      load_half(s_addr, (pl.full | pl.bnd) != 0u, su);
+      tmem_ld64(dp_addr, dp);
+      // P^T = exp2(S^T c2 - LSE_i log2 e) on the causal pairs i >= j, dS^T = P^T (dP^T - D_i)
+      const int64_t cmin = j - q0;  // first causal query column
+      const int64_t cval = N - 1 - q0;  // last valid query column
+      float pf[64], ds[64];
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = ld4[c4], d4 = ld4[16 + c4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 4 * c4 + e;
+          const bool live = row_ok && c >= cmin && c <= cval;
+          const float p = fast_exp2(fmaf(__uint_as_float(su[c]), c2, -lv[e]));
+          pf[c] = live ? p : 0.f;
+          ds[c] = live ? p * (__uint_as_float(dp[c]) - dv[e]) : 0.f;
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pk[k] = pack_bf16x2(pf[2 * k], pf[2 * k + 1]);
+        tmem_st32(s_addr, pk);
+      }
+      store_ds_upto(dp_addr, ds, TBS - 1);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ds_ready[bf]);
+      int64_t prev = INT64_MAX;
+      int32_t W;
+      uint32_t cls;
+      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        ok = warp_wait(dsm_req, dsm_cnt & 1, lim, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const int64_t cm = j - q0 + W;
+        store_ds_upto(dp_addr, ds, cm < -1 ? -1 : (cm > TBS - 1 ? TBS - 1 : static_cast<int>(cm)));
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dsm_done);
+        ++dsm_cnt;
+        prev = W;
+      }
+    }
+    __nv_bfloat16 *dkrow = a.dk + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D;
+    __nv_bfloat16 *dvrow = a.dv + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D;
+    if (ok && nsub > 0 && warp_wait(kv_final, 0, lim, abort_flag)) {
+      tc_fence_after();
+#pragma unroll
+      for (int c4 = 0; c4 < 2 * D / 32; ++c4) {
+        uint32_t u32[32];
+        tmem_ld32(lane_addr + KV_DK + 32 * c4, u32);
+        tmem_wait_ld(u32);
+        const float sc = c4 < D / 32 ? a.scale : 1.f;  // dK carries the softmax scale, dV not
+        uint4 pk4[4];
+        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * sc, __uint_as_float(u32[2 * k + 1]) * sc);
+        if (row_ok) {
+          uint4 *dst = reinterpret_cast<uint4 *>(c4 < D / 32 ? dkrow + 32 * c4 : dvrow + 32 * (c4 - D / 32));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
+        }
+      }
+    } else {
+      *abort_flag = 1;
+      if (row_ok) {
+        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+#pragma unroll
+        for (int k = 0; k < D / 8; ++k) {
+          reinterpret_cast<uint4 *>(dkrow)[k] = nan4;
+          reinterpret_cast<uint4 *>(dvrow)[k] = nan4;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == T_MMA) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_dkdv(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t stream) {
+  // one CTA per SM: the kernel holds all 512 TMEM columns
+  const uint32_t smem = KvTL<D>::BYTES > 120u * 1024u ? KvTL<D>::BYTES : 120u * 1024u;
+  cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dkdv_tc_kernel<D><<<dim3((a.N + TBQ - 1) / TBQ, a.Hkv, a.B), TC_THREADS, smem, stream>>>(m.k128, m.v128, m.q64,
+                                                                                         m.do64, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_dq(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t stream) {
+  // one CTA per SM: the kernel holds all 512 TMEM columns
+  const uint32_t smem = DqTL<D>::BYTES > 120u * 1024u ? DqTL<D>::BYTES : 120u * 1024u;
+  cudaError_t e = cudaFuncSetAttribute(dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dq_tc_kernel<D><<<dim3((a.N + TBQ - 1) / TBQ, a.Hq, a.B), TC_THREADS, smem, stream>>>(m.q128, m.do128, m.k64,
+                                                                                       m.v64, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward_dq_tc(int d_h, const BackwardArgs &a, const BackwardMaps &maps, cudaStream_t stream) {
+  return d_h == 128 ? launch_dq<128>(a, maps, stream) : launch_dq<64>(a, maps, stream);
+}
+
+cudaError_t launch_backward_dkdv_tc(int d_h, const BackwardArgs &a, const BackwardMaps &maps, cudaStream_t stream) {
+  return d_h == 128 ? launch_dkdv<128>(a, maps, stream) : launch_dkdv<64>(a, maps, stream);
+}
+
+}  // namespace wp
