@@ -65,7 +65,7 @@ def parse_args():
     p.add_argument("--grouping", choices=["half-split", "paired"], default="half-split",
                    help="paired: Q/K of the half-split model rotated into the interleaved order, groups of 8 "
                         "whole channels (the pages' grouping, Table 12 cutoffs)")
-    p.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    p.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                    help="restrict the step (profiling a single kernel)")
     p.add_argument("--prefill-mode", choices=["grouped", "exact"], default="grouped",
                    help="rule of the timed prefill in a restricted profiling case (--only prefill)")
@@ -609,7 +609,7 @@ def run_ours(args, rank, world, local):
 
     # backward of the 32K prefill (wp_prefill_backward), wave and dense
     backward = None
-    if args.only == "all" and not args.no_backward:
+    if args.only in ("all", "backward") and not args.no_backward:
         dout = torch.randn(path.o.shape, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).to(dev)
         dq, dk, dv = torch.empty_like(path.qr), torch.empty_like(path.kr), torch.empty_like(path.v)
         bw_useful, bw_dense = backward_flops(pw.N, pw.d, pw.Hq, pw.B, path.wg)
@@ -718,7 +718,7 @@ def run_ours(args, rank, world, local):
         "backward": backward,
         "exact": exact,
         "e2e": e2e,
-        "gpu_launches": {"all": 6, "prefill": 3, "decode": 3}[args.only] * K,
+        "gpu_launches": {"all": 6, "prefill": 3, "decode": 3, "backward": 0}[args.only] * K,
         "clocks": clk,
         "paper_context": {"source": "A100 FlashWavePrune vs FlashAttention-2, d128, theta 1e6 (context only)",
                           "prefill_speedup_32k": 1.15, "decode_speedup_32k": 1.24},

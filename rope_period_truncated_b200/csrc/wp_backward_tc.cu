@@ -15,17 +15,23 @@
 // dq_tc_kernel: one CTA per (128-row query block, query head). It walks the
 // 64-key sub-tiles from the diagonal backwards (u = 0, 1, ...; distances
 // grow with u). Warp roles:
-//   warp 4   TMA producer: Q and dO of the block once (16-dim boxes, 32-byte
-//            swizzle); per sub-tile the K group tiles some group needs and V,
+//   warp 8   TMA producer: Q and dO of the block once (16-dim boxes, 32-byte
+//            swizzle); per sub-tile the K group tiles some group needs, V and
+//            the sub-tile's group classes (a plan word beside the stage),
 //            three stages.
-//   warp 5   MMA issuer: S(u) = sum_g Q_g K_g^T (M128 N64 K16 per non-skipped
+//   warp 9   MMA issuer: S(u) = sum_g Q_g K_g^T (M128 N64 K16 per non-skipped
 //            group) and dP(u) = dO V^T into double-buffered TMEM, then, once
 //            the row warps have written dS(u) (bf16, over S's first 32
 //            columns), dQ[g0:g1] += dS K[g0:g1] for each run of consecutive
 //            full groups as M128 N16*(g1-g0) K16 products with dS read from
 //            TMEM and K read MN-major from the same swizzled group tiles.
-//   warps 0-3 one thread per query row: P, dS = P (dP - D), dS to TMEM; the
-//            epilogue scales dQ and writes it as bf16.
+//   warps 0-7 two threads per query row: warp w reads TMEM lanes 32 (w % 4)..
+//            and the sub-tile's columns 32 (w / 4) .. +31, and forms P and
+//            dS = P (dP - D) there in packed f32x2 arithmetic (no row
+//            reduction is needed: P comes from the forward's LSE). Each writes
+//            its dS as bf16 over the first 16 of its own S columns, and the
+//            MMAs address the two halves separately. The epilogue scales dQ
+//            and writes it as bf16.
 // Boundary groups (cutoff inside the sub-tile's distance range), as in the
 // forward kernel: their S products go first, one cutoff class at a time in
 // ascending order, and the row warps mask S in place after each (nested
@@ -61,51 +67,29 @@ namespace {
 constexpr int TBQ = 128;  // rows of a CTA's block
 constexpr int TBS = 64;   // columns of a sub-tile
 constexpr int TNST = 3;   // stages of the streamed operands
-constexpr int TC_THREADS = 192;
-constexpr int T_PROD = 4, T_MMA = 5;
+constexpr int TC_THREADS = 320;  // warps 0-7 row warps, 8 TMA producer, 9 MMA issuer
+constexpr int NROWW = 8;
+constexpr int T_PROD = 8, T_MMA = 9;
 constexpr uint32_t TILE128 = 128 * 32;  // a 16-dim group tile of 128 rows
 constexpr uint32_t TILE64 = 64 * 32;    // a 16-dim group tile of 64 rows
 constexpr float TLOG2E = 1.4426950408889634f;
 
-// TMEM columns of the dQ kernel
-constexpr uint32_t DQ_S = 0;     // S / dS of buffer b at 64 b
-constexpr uint32_t DQ_DP = 128;  // dP of buffer b at 128 + 64 b
-constexpr uint32_t DQ_ACC = 256;
-
-template <int D>
-struct DqTL {
-  static constexpr int G = D / 16;
-  static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t DO_OFF = Q_OFF + G * TILE128;
-  static constexpr uint32_t K_OFF = DO_OFF + G * TILE128;
-  static constexpr uint32_t STAGE = G * TILE64;
-  static constexpr uint32_t V_OFF = K_OFF + TNST * STAGE;
-  static constexpr uint32_t BAR_OFF = V_OFF + TNST * STAGE;
-  // qd_full, kv_full[TNST], kv_empty[TNST], s_ready[2], ds_ready[2],
-  // bnd_ready, bnd_done, dsm_req, dsm_done, dq_final, drain
-  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
-  static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // the head's group cutoffs, 8 int32
-  static constexpr uint32_t BYTES = CUT_OFF + 32 + 1024;
-};
-
-// Group classes of a 128-row x 64-column block whose causal pairs span
-// distances [dmin, dmax] (any = it has causal pairs): full and boundary bits.
-struct SubPlan {
-  uint32_t full, bnd;
-  bool any;
-};
-__device__ __forceinline__ SubPlan sub_plan(const int32_t *cut, int G, bool any, int64_t dmin, int64_t dmax) {
-  SubPlan p{0u, 0u, any};
+// A sub-tile's group classes: bits 0-7 full groups, 8-15 boundary groups,
+// bit 16 set when the sub-tile holds causal pairs at all.
+__device__ __forceinline__ uint32_t plan_word(const int32_t *cut, int G, bool any, int64_t dmin, int64_t dmax) {
+  uint32_t full = 0, bnd = 0;
   if (any) {
     for (int g = 0; g < G; ++g) {
       const int c = classify_cutoff(dmin, dmax, cut[g]);
-      if (c == TILE_FULL) p.full |= 1u << g;
-      if (c == TILE_BOUNDARY) p.bnd |= 1u << g;
+      if (c == TILE_FULL) full |= 1u << g;
+      if (c == TILE_BOUNDARY) bnd |= 1u << g;
     }
   }
-  return p;
+  return full | (bnd << 8) | (any ? 1u << 16 : 0u);
 }
+__device__ __forceinline__ uint32_t pw_full(uint32_t w) { return w & 0xffu; }
+__device__ __forceinline__ uint32_t pw_bnd(uint32_t w) { return (w >> 8) & 0xffu; }
+__device__ __forceinline__ bool pw_any(uint32_t w) { return (w >> 16) & 1u; }
 
 // Largest cutoff among the boundary groups in `bnd` that is < prev (prev =
 // INT64_MAX for the first); false when none. `mask` gets the groups of it.
@@ -127,14 +111,106 @@ __device__ __forceinline__ bool prev_boundary_class(const int32_t *cut, uint32_t
   return true;
 }
 
-// dS (fp32, 64 columns) as bf16 pairs into 32 TMEM columns, columns c < cmin zeroed.
-__device__ __forceinline__ void store_ds(uint32_t taddr, const float (&ds)[64], int cmin) {
-  uint32_t pk[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-    pk[k] = pack_bf16x2(2 * k < cmin ? 0.f : ds[2 * k], 2 * k + 1 < cmin ? 0.f : ds[2 * k + 1]);
-  tmem_st32(taddr, pk);
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
 }
+
+// 32 TMEM columns at each of two addresses, one wait for both.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t (&r0)[32], uint32_t a1, uint32_t (&r1)[32]) {
+  tmem_ld32(a0, r0);
+  tmem_ld32(a1, r1);
+  tmem_wait_ld(r0);
+  tmem_wait_ld(r1);
+}
+
+// 32 fp32 values as bf16 pairs into 16 TMEM columns; columns outside
+// [lo, hi] (0-based within the 32) written as 0.
+__device__ __forceinline__ void store_bf16_32(uint32_t taddr, const float (&x)[32], int lo, int hi) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    pk[k] = pack_bf16x2(2 * k < lo || 2 * k > hi ? 0.f : x[2 * k], 2 * k + 1 < lo || 2 * k + 1 > hi ? 0.f : x[2 * k + 1]);
+  tmem_st16(taddr, pk);
+}
+
+// TMEM address of K16 step kk of a bf16 operand written by the two column
+// halves: keys (or queries) 16 kk .. belong to half kk / 2, which keeps its
+// 16 packed columns at the start of its own 32.
+__device__ __forceinline__ uint32_t half_operand(uint32_t base, int kk) { return base + 32 * (kk >> 1) + 8 * (kk & 1); }
+
+// Zero n32 x 32 TMEM columns of this warp's lanes.
+__device__ __forceinline__ void tmem_zero(uint32_t taddr, int n32) {
+  uint32_t z[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) z[k] = 0u;
+  for (int c = 0; c < n32; ++c) tmem_st32(taddr + 32 * c, z);
+  tmem_wait_st();
+}
+
+// Scale 32 fp32 TMEM columns, write them to global memory as bf16 (16-byte stores).
+__device__ __forceinline__ void store_row32(uint32_t taddr, float scale, __nv_bfloat16 *dst, bool ok) {
+  uint32_t u32[32];
+  tmem_ld32(taddr, u32);
+  tmem_wait_ld(u32);
+  uint4 pk4[4];
+  uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * scale, __uint_as_float(u32[2 * k + 1]) * scale);
+  if (ok) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) reinterpret_cast<uint4 *>(dst)[k] = pk4[k];
+  }
+}
+
+__device__ __forceinline__ void store_nan(__nv_bfloat16 *dst, int n) {
+  const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
+  for (int k = 0; k < n / 8; ++k) reinterpret_cast<uint4 *>(dst)[k] = nan4;
+}
+
+// The MMA warp's issue order, shared by both kernels: S(v) of sub-tile v goes
+// out two ahead of the gradient products, or one ahead when v has boundary
+// classes (its handshakes must follow the row warps' finish of v - 1).
+// `plan(v)` waits for v's stage and returns its plan word; `sdp(v)` issues
+// S(v) and dP(v).
+template <class PlanFn, class SdpFn>
+__device__ __forceinline__ bool advance_sdp(int &next, int done, int nsub, PlanFn plan, SdpFn sdp) {
+  while (next < nsub && next <= done + 2) {
+    uint32_t w;
+    if (!plan(next, w)) return false;
+    if (pw_bnd(w) != 0u && next > done + 1) break;
+    if (!sdp(next, w)) return false;
+    ++next;
+  }
+  return true;
+}
+
+// ============================================================ dQ kernel
+
+// TMEM columns of the dQ kernel
+constexpr uint32_t DQ_S = 0;     // S / dS of buffer b at 64 b
+constexpr uint32_t DQ_DP = 128;  // dP of buffer b at 128 + 64 b
+constexpr uint32_t DQ_ACC = 256;
+
+template <int D>
+struct DqTL {
+  static constexpr int G = D / 16;
+  static constexpr uint32_t Q_OFF = 0;
+  static constexpr uint32_t DO_OFF = Q_OFF + G * TILE128;
+  static constexpr uint32_t K_OFF = DO_OFF + G * TILE128;
+  static constexpr uint32_t STAGE = G * TILE64;
+  static constexpr uint32_t V_OFF = K_OFF + TNST * STAGE;
+  static constexpr uint32_t BAR_OFF = V_OFF + TNST * STAGE;
+  // qd_full, kv_full[TNST], kv_empty[TNST], s_ready[2], ds_ready[2],
+  // bnd_ready, bnd_done, dsm_req, dsm_done, dq_final, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
+  static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // the head's group cutoffs, 8 int32
+  static constexpr uint32_t PLAN_OFF = CUT_OFF + 32;  // plan word per stage
+  static constexpr uint32_t BYTES = PLAN_OFF + 16 + 1024;
+};
 
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -159,6 +235,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
   int32_t *cut = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);
+  volatile uint32_t *plans = reinterpret_cast<volatile uint32_t *>(smem + L::PLAN_OFF);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -177,12 +254,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_ready[s], 1);
-      mbar_init(&ds_ready[s], 4);
+      mbar_init(&ds_ready[s], NROWW);
     }
     mbar_init(bnd_ready, 1);
-    mbar_init(bnd_done, 4);
+    mbar_init(bnd_done, NROWW);
     mbar_init(dsm_req, 1);
-    mbar_init(dsm_done, 4);
+    mbar_init(dsm_done, NROWW);
     mbar_init(dq_final, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -197,12 +274,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nsub = *abort_flag ? 0 : 2 * (qb + 1);  // key sub-tile 2qb + 1 - u
-  // the plan of sub-tile u
-  auto plan_of = [&](int u) -> SubPlan {
-    int64_t dmin = 0, dmax = -1;
-    const bool any = tile_distance_range(N, TBQ, TBS, qb, 2 * qb + 1 - u, &dmin, &dmax);
-    return sub_plan(cut, G, any, dmin, dmax);
-  };
 
   if (warp == T_PROD) {
     // ------------------------------------------------------------ producer
@@ -223,11 +294,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int u = 0; u < nsub; ++u) {
       const int st = u % TNST;
       if (u >= TNST && !warp_wait_idle(&kv_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
+      int64_t dmin = 0, dmax = -1;
+      const bool any = tile_distance_range(N, TBQ, TBS, qb, 2 * qb + 1 - u, &dmin, &dmax);
+      const uint32_t w = plan_word(cut, G, any, dmin, dmax);
+      if (lane == 0) plans[st] = w;
+      __syncwarp();
       // a sub-tile without causal pairs (past the end of a ragged last block)
       // loads nothing: its dS is 0 whatever the buffers hold
-      const SubPlan pl = plan_of(u);
-      const uint32_t need = pl.full | pl.bnd;
-      const int nv = pl.any ? G : 0;
+      const uint32_t need = pw_full(w) | pw_bnd(w);
+      const int nv = any ? G : 0;
       const int krow = (2 * qb + 1 - u) * TBS;
       if (leader) {
         mbar_arrive_expect_tx(&kv_full[st], (__popc(need) + nv) * TILE64);
@@ -259,20 +334,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool ok = warp_wait(qd_full, 0, lim, abort_flag);
     int bnd_cnt = 0, dsm_cnt = 0;
 
-    // S(u) and dP(u) into buffer u & 1
-    auto issue_sdp = [&](int u) -> bool {
+    auto plan = [&](int u, uint32_t &w) -> bool {
+      if (!warp_wait(&kv_full[u % TNST], (u / TNST) & 1, lim, abort_flag)) return false;
+      w = plans[u % TNST];
+      return true;
+    };
+    // S(u) and dP(u) into buffer u & 1 (its stage loaded)
+    auto issue_sdp = [&](int u, uint32_t w) -> bool {
       const int st = u % TNST, bf = u & 1;
-      if (!warp_wait(&kv_full[st], (u / TNST) & 1, lim, abort_flag)) return false;
       tc_fence_after();
-      const SubPlan pl = plan_of(u);
       const uint32_t s_col = tmem + DQ_S + 64 * bf;
       const uint64_t kst = k_desc + ((st * L::STAGE) >> 4);
       uint32_t acc = 0;
-      if (pl.bnd) {
+      if (pw_bnd(w)) {
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
           if (leader) {
             for (int g = 0; g < G; ++g)
               if ((cls >> g) & 1u) {
@@ -290,14 +368,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       if (leader) {
+        const uint32_t full = pw_full(w);
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          if ((pl.full >> g) & 1u) {
+          if ((full >> g) & 1u) {
             umma_ss(s_col, q_desc + g * GD128, kst + g * GD64, IDESC_S, acc);
             acc = 1;
           }
         const uint64_t vst = v_desc + ((st * L::STAGE) >> 4);
-        if (pl.any) {
+        if (pw_any(w)) {
 #pragma unroll
           for (int g = 0; g < G; ++g)
             umma_ss(tmem + DQ_DP + 64 * bf, do_desc + g * GD128, vst + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
@@ -320,7 +399,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + DQ_ACC + 16 * g0, tmem + DQ_S + 64 * bf + kk * 8,
+            umma_ts(tmem + DQ_ACC + 16 * g0, half_operand(tmem + DQ_S + 64 * bf, kk),
                     kst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
@@ -329,12 +408,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // dQ(u): full groups on dS as it is, then the boundary classes in
     // descending cutoff order, each after the row warps masked dS for it
     auto issue_dq = [&](int u) -> bool {
-      const SubPlan pl = plan_of(u);
-      issue_dq_groups(u, pl.full);
+      const uint32_t w = plans[u % TNST];
+      issue_dq_groups(u, pw_full(w));
       int64_t prev = INT64_MAX;
       int32_t W;
       uint32_t cls;
-      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+      while (prev_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
         if (leader) umma_commit(dsm_req);
         __syncwarp();
         if (!warp_wait(dsm_done, dsm_cnt & 1, lim, abort_flag)) return false;
@@ -348,18 +427,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       return true;
     };
 
-    // S of sub-tile v goes out two ahead, or one ahead when v has boundary
-    // classes (its handshakes must follow the row warps' finish of v - 1).
     int next = 0;
-    auto advance = [&](int done) -> bool {
-      while (next < nsub && next <= done + 2) {
-        if (plan_of(next).bnd != 0u && next > done + 1) break;
-        if (!issue_sdp(next)) return false;
-        ++next;
-      }
-      return true;
-    };
-    if (ok) ok = advance(-1);
+    if (ok) ok = advance_sdp(next, -1, nsub, plan, issue_sdp);
     for (int u = 0; ok && u < nsub; ++u) {
       if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
         ok = false;
@@ -367,7 +436,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       tc_fence_after();
       ok = issue_dq(u);
-      if (ok) ok = advance(u);
+      if (ok) ok = advance_sdp(next, u, nsub, plan, issue_sdp);
     }
     if (leader) {
       umma_commit(dq_final);
@@ -375,50 +444,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     __syncwarp();
     warp_wait(drain, 0, lim, nullptr);
-  } else if (warp < 4) {
+  } else if (warp < NROWW) {
     // ---------------------------------------------------------- row warps
-    const int r = warp * 32 + lane;
+    const int q4 = warp & 3, hf = warp >> 2, cb = 32 * hf;  // lane quarter, first column
+    const int r = q4 * 32 + lane;
     const int64_t i = static_cast<int64_t>(qb) * TBQ + r;
     const bool row_ok = i < N;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N + (row_ok ? i : 0);
     const float lse2 = row_ok ? a.lse[lrow] * TLOG2E : 0.f;
     const float di = row_ok ? a.delta[lrow] : 0.f;
-    const float c2 = a.scale_log2;
-    // zero the dQ accumulator: every dQ product accumulates
-    {
-      uint32_t z[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = 0u;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) tmem_st32(lane_addr + DQ_ACC + 32 * c4, z);
-      tmem_wait_st();
-    }
+    const uint64_t c2x2 = pack_f2(a.scale_log2, a.scale_log2), nl2 = pack_f2(-lse2, -lse2), nd2 = pack_f2(-di, -di);
+    tmem_zero(lane_addr + DQ_ACC + hf * (D / 2), D / 64);  // every dQ product accumulates
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
-      const int bf = u & 1;
-      const int64_t k0 = static_cast<int64_t>(2 * qb + 1 - u) * TBS;  // first key of the sub-tile
-      const uint32_t s_addr = lane_addr + DQ_S + 64 * bf;
-      const SubPlan pl = plan_of(u);
-      if (pl.bnd) {
+      const int st = u % TNST, bf = u & 1;
+      const int64_t k0 = static_cast<int64_t>(2 * qb + 1 - u) * TBS + cb;  // first key of my columns
+      const uint32_t s_addr = lane_addr + DQ_S + 64 * bf + cb;
+      if (!warp_wait(&kv_full[st], (u / TNST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t w = plans[st];
+      if (pw_bnd(w)) {
         // S masked in place after each boundary class: keep key c iff i - (k0 + c) <= W
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
           ok = warp_wait(bnd_ready, bnd_cnt & 1, lim, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const int64_t cm = i - k0 - W;
-          const int cmin = cm < 0 ? 0 : (cm > TBS ? TBS : static_cast<int>(cm));
-          uint32_t su[64];
-          tmem_ld64(s_addr, su);
+          const int cmin = cm < 0 ? 0 : (cm > 32 ? 32 : static_cast<int>(cm));
+          uint32_t su[32];
+          tmem_ld32(s_addr, su);
+          tmem_wait_ld(su);
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c < cmin) su[c] = 0u;
-          tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
-          tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+          tmem_st32(s_addr, su);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -433,19 +499,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      uint32_t su[64], dp[64];
-      load_half(s_addr, (pl.full | pl.bnd) != 0u, su);
-      tmem_ld64(lane_addr + DQ_DP + 64 * bf, dp);
-      // P = exp2(S c2 - LSE log2 e) on the causal pairs of valid rows, dS = P (dP - D)
-      const int64_t jmax = i - k0;  // last causal key column
-      float ds[64];
+      uint32_t su[32], dp[32];
+      if (pw_full(w) | pw_bnd(w)) {
+        tmem_ld32x2(s_addr, su, lane_addr + DQ_DP + 64 * bf + cb, dp);
+      } else {
+        tmem_ld32(lane_addr + DQ_DP + 64 * bf + cb, dp);
+        tmem_wait_ld(dp);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const bool live = row_ok && c <= jmax;
-        const float p = fast_exp2(fmaf(__uint_as_float(su[c]), c2, -lse2));
-        ds[c] = live ? p * (__uint_as_float(dp[c]) - di) : 0.f;
+        for (int c = 0; c < 32; ++c) su[c] = 0u;
       }
-      store_ds(s_addr, ds, 0);
+      // P = exp2(S c2 - LSE log2 e) and dS = P (dP - D) on the causal pairs of a valid row
+      const int64_t jm = i - k0;  // my last causal column
+      const int jmax = !row_ok ? -1 : (jm > 31 ? 31 : (jm < -1 ? -1 : static_cast<int>(jm)));
+      float ds[32];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[2 * k]), __uint_as_float(su[2 * k + 1])), c2x2, nl2);
+        float x0, x1;
+        unpack_f2(x2, x0, x1);
+        const uint64_t g2 = fadd2(pack_f2(__uint_as_float(dp[2 * k]), __uint_as_float(dp[2 * k + 1])), nd2);
+        float d0, d1;
+        unpack_f2(fmul2(pack_f2(fast_exp2(x0), fast_exp2(x1)), g2), d0, d1);
+        ds[2 * k] = d0;
+        ds[2 * k + 1] = d1;
+      }
+      store_bf16_32(s_addr, ds, 0, jmax);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -454,12 +532,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int64_t prev = INT64_MAX;
       int32_t W;
       uint32_t cls;
-      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+      while (prev_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
         ok = warp_wait(dsm_req, dsm_cnt & 1, lim, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const int64_t cm = i - k0 - W;
-        store_ds(s_addr, ds, cm < 0 ? 0 : (cm > TBS ? TBS : static_cast<int>(cm)));
+        store_bf16_32(s_addr, ds, cm < 0 ? 0 : (cm > 32 ? 32 : static_cast<int>(cm)), jmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -468,32 +546,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prev = W;
       }
     }
-    __nv_bfloat16 *dqrow = a.dq + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
+    __nv_bfloat16 *dqrow = a.dq + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D + hf * (D / 2);
     if (ok && nsub > 0 && warp_wait(dq_final, 0, lim, abort_flag)) {
       tc_fence_after();
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t u32[32];
-        tmem_ld32(lane_addr + DQ_ACC + 32 * c4, u32);
-        tmem_wait_ld(u32);
-        uint4 pk4[4];
-        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * a.scale, __uint_as_float(u32[2 * k + 1]) * a.scale);
-        if (row_ok) {
-          uint4 *dst = reinterpret_cast<uint4 *>(dqrow + 32 * c4);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
-        }
-      }
+      for (int c = 0; c < D / 64; ++c)
+        store_row32(lane_addr + DQ_ACC + hf * (D / 2) + 32 * c, a.scale, dqrow + 32 * c, row_ok);
     } else {
       *abort_flag = 1;
-      if (row_ok) {
-        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) reinterpret_cast<uint4 *>(dqrow)[k] = nan4;
-      }
+      if (row_ok) store_nan(dqrow, D / 2);
     }
   }
 
@@ -506,18 +566,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
+// ========================================================= dK/dV kernel
+
 // TMEM columns of the dK/dV kernel
 constexpr uint32_t KV_S = 0;     // S^T / P^T of buffer b at 64 b
 constexpr uint32_t KV_DP = 128;  // dP^T / dS^T of buffer b at 128 + 64 b
 constexpr uint32_t KV_DK = 256;
-template <int D>
-constexpr uint32_t kv_dv() {
-  return KV_DK + D;
-}
 
 template <int D>
 struct KvTL {
   static constexpr int G = D / 16;
+  static constexpr uint32_t DV_COL = KV_DK + D;
   static constexpr uint32_t K_OFF = 0;
   static constexpr uint32_t V_OFF = K_OFF + G * TILE128;
   static constexpr uint32_t Q_OFF = V_OFF + G * TILE128;
@@ -529,18 +588,10 @@ struct KvTL {
   // bnd_ready, bnd_done, dsm_req, dsm_done, kv_final, drain
   static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // cutoff rows of the KV head's query heads, [rep][8]
+  static constexpr uint32_t PLAN_OFF = MISC_OFF + 16;  // plan word and head of each stage
+  static constexpr uint32_t CUT_OFF = PLAN_OFF + 32;   // cutoff rows of the KV head's query heads, [rep][8]
   static constexpr uint32_t BYTES = CUT_OFF + 64 * 8 * 4 + 1024;
 };
-
-// dS^T (fp32, 64 query columns) as bf16 pairs into 32 TMEM columns, columns c > cmax zeroed.
-__device__ __forceinline__ void store_ds_upto(uint32_t taddr, const float (&ds)[64], int cmax) {
-  uint32_t pk[32];
-#pragma unroll
-  for (int k = 0; k < 32; ++k)
-    pk[k] = pack_bf16x2(2 * k > cmax ? 0.f : ds[2 * k], 2 * k + 1 > cmax ? 0.f : ds[2 * k + 1]);
-  tmem_st32(taddr, pk);
-}
 
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -551,7 +602,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   constexpr int G = L::G;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, TBS, false, false);
   constexpr uint32_t GD128 = TILE128 >> 4, GD64 = TILE64 >> 4;
-  constexpr uint32_t KV_DV = kv_dv<D>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -565,7 +615,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t *kv_final = dsm_done + 1, *drain = kv_final + 1;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
-  int32_t *cuts = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);  // [rep][8]
+  volatile uint32_t *plans = reinterpret_cast<volatile uint32_t *>(smem + L::PLAN_OFF);  // [stage]
+  int32_t *cuts = reinterpret_cast<int32_t *>(smem + L::CUT_OFF);                        // [rep][8]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int kb = static_cast<int>(blockIdx.x);  // key blocks near the start see the most queries: first
@@ -585,12 +636,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_ready[s], 1);
-      mbar_init(&ds_ready[s], 4);
+      mbar_init(&ds_ready[s], NROWW);
     }
     mbar_init(bnd_ready, 1);
-    mbar_init(bnd_done, 4);
+    mbar_init(bnd_done, NROWW);
     mbar_init(dsm_req, 1);
-    mbar_init(dsm_done, 4);
+    mbar_init(dsm_done, NROWW);
     mbar_init(kv_final, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -609,13 +660,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   const int nsub = *abort_flag ? 0 : rep * per_head;
   // sub-tile u: query head hk * rep + u / per_head, query rows 64 * (2kb + u % per_head) ..
-  auto head_of = [&](int u) { return u / per_head; };
   auto q0_of = [&](int u) { return static_cast<int64_t>(2 * kb + u % per_head) * TBS; };
-  auto plan_of = [&](int u) -> SubPlan {
-    int64_t dmin = 0, dmax = -1;
-    const bool any = tile_distance_range(N, TBS, TBQ, 2 * kb + u % per_head, kb, &dmin, &dmax);
-    return sub_plan(cuts + 8 * head_of(u), G, any, dmin, dmax);
-  };
 
   if (warp == T_PROD) {
     // ------------------------------------------------------------ producer
@@ -636,11 +681,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int u = 0; u < nsub; ++u) {
       const int st = u % TNST;
       if (u >= TNST && !warp_wait_idle(&qd_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
-      const SubPlan pl = plan_of(u);
-      const uint32_t need = pl.full | pl.bnd;
-      const int h = hk * rep + head_of(u);
+      const int hr = u / per_head;
+      const int h = hk * rep + hr;
       const int64_t q0 = q0_of(u);
-      // the sub-tile's LSE (log2 units) and D, read by the row warps
+      int64_t dmin = 0, dmax = -1;
+      const bool any = tile_distance_range(N, TBS, TBQ, 2 * kb + u % per_head, kb, &dmin, &dmax);
+      const uint32_t w = plan_word(cuts + 8 * hr, G, any, dmin, dmax);
+      // the plan, and the sub-tile's LSE (log2 units) and D, read by the row warps
       float *ld = reinterpret_cast<float *>(smem + L::LD_OFF + st * 512);
       const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N;
       for (int c = lane; c < TBS; c += 32) {
@@ -648,7 +695,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ld[c] = in ? a.lse[lrow + q0 + c] * TLOG2E : 0.f;
         ld[TBS + c] = in ? a.delta[lrow + q0 + c] : 0.f;
       }
+      if (lane == 0) {
+        plans[2 * st] = w;
+        plans[2 * st + 1] = static_cast<uint32_t>(hr);
+      }
       __syncwarp();
+      const uint32_t need = pw_full(w) | pw_bnd(w);
       if (leader) {
         mbar_arrive_expect_tx(&qd_full[st], (__popc(need) + G) * TILE64);
         for (uint32_t m = need; m; m &= m - 1) {
@@ -682,20 +734,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool ok = warp_wait(kv_full, 0, lim, abort_flag);
     int bnd_cnt = 0, dsm_cnt = 0;
 
-    auto issue_sdp = [&](int u) -> bool {
+    auto plan = [&](int u, uint32_t &w) -> bool {
+      if (!warp_wait(&qd_full[u % TNST], (u / TNST) & 1, lim, abort_flag)) return false;
+      w = plans[2 * (u % TNST)];
+      return true;
+    };
+    auto issue_sdp = [&](int u, uint32_t w) -> bool {
       const int st = u % TNST, bf = u & 1;
-      if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag)) return false;
       tc_fence_after();
-      const SubPlan pl = plan_of(u);
-      const int32_t *cut = cuts + 8 * head_of(u);
+      const int32_t *cut = cuts + 8 * static_cast<int>(plans[2 * st + 1]);
       const uint32_t s_col = tmem + KV_S + 64 * bf;
       const uint64_t qst = q_desc + ((st * L::STAGE) >> 4);
       uint32_t acc = 0;
-      if (pl.bnd) {
+      if (pw_bnd(w)) {
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
           if (leader) {
             for (int g = 0; g < G; ++g)
               if ((cls >> g) & 1u) {
@@ -713,9 +768,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
       if (leader) {
+        const uint32_t full = pw_full(w);
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          if ((pl.full >> g) & 1u) {
+          if ((full >> g) & 1u) {
             umma_ss(s_col, k_desc + g * GD128, qst + g * GD64, IDESC_S, acc);
             acc = 1;
           }
@@ -741,7 +797,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + KV_DK + 16 * g0, tmem + KV_DP + 64 * bf + kk * 8,
+            umma_ts(tmem + KV_DK + 16 * g0, half_operand(tmem + KV_DP + 64 * bf, kk),
                     qst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
@@ -751,21 +807,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // classes in descending cutoff order, each after the row warps masked dS^T
     auto issue_dkdv = [&](int u) -> bool {
       const int st = u % TNST, bf = u & 1;
-      const SubPlan pl = plan_of(u);
-      const int32_t *cut = cuts + 8 * head_of(u);
+      const uint32_t w = plans[2 * st];
+      const int32_t *cut = cuts + 8 * static_cast<int>(plans[2 * st + 1]);
       if (leader) {
         constexpr uint32_t IDESC_DV = idesc_bf16_f32(128, D, false, true);
         const uint64_t dost = domn_desc + ((st * L::STAGE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < TBS / 16; ++kk)
-          umma_ts(tmem + KV_DV, tmem + KV_S + 64 * bf + kk * 8, dost + ((kk * 16 * 32) >> 4), IDESC_DV, 1u);
+          umma_ts(tmem + L::DV_COL, half_operand(tmem + KV_S + 64 * bf, kk), dost + ((kk * 16 * 32) >> 4), IDESC_DV,
+                  1u);
       }
       __syncwarp();
-      issue_dk_groups(u, pl.full);
+      issue_dk_groups(u, pw_full(w));
       int64_t prev = INT64_MAX;
       int32_t W;
       uint32_t cls;
-      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+      while (prev_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
         if (leader) umma_commit(dsm_req);
         __syncwarp();
         if (!warp_wait(dsm_done, dsm_cnt & 1, lim, abort_flag)) return false;
@@ -780,15 +837,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     };
 
     int next = 0;
-    auto advance = [&](int done) -> bool {
-      while (next < nsub && next <= done + 2) {
-        if (plan_of(next).bnd != 0u && next > done + 1) break;
-        if (!issue_sdp(next)) return false;
-        ++next;
-      }
-      return true;
-    };
-    if (ok) ok = advance(-1);
+    if (ok) ok = advance_sdp(next, -1, nsub, plan, issue_sdp);
     for (int u = 0; ok && u < nsub; ++u) {
       if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
         ok = false;
@@ -796,7 +845,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       tc_fence_after();
       ok = issue_dkdv(u);
-      if (ok) ok = advance(u);
+      if (ok) ok = advance_sdp(next, u, nsub, plan, issue_sdp);
     }
     if (leader) {
       umma_commit(kv_final);
@@ -804,47 +853,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     __syncwarp();
     warp_wait(drain, 0, lim, nullptr);
-  } else if (warp < 4) {
+  } else if (warp < NROWW) {
     // ---------------------------------------------------------- row warps
-    const int r = warp * 32 + lane;
+    const int q4 = warp & 3, hf = warp >> 2, cb = 32 * hf;  // lane quarter, first column
+    const int r = q4 * 32 + lane;
     const int64_t j = static_cast<int64_t>(kb) * TBQ + r;  // this thread's key
     const bool row_ok = j < N;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const float c2 = a.scale_log2;
-    {
-      uint32_t z[32];
-#pragma unroll
-      for (int k = 0; k < 32; ++k) z[k] = 0u;
-#pragma unroll
-      for (int c4 = 0; c4 < 2 * D / 32; ++c4) tmem_st32(lane_addr + KV_DK + 32 * c4, z);
-      tmem_wait_st();
-    }
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint64_t c2x2 = pack_f2(a.scale_log2, a.scale_log2);
+    tmem_zero(lane_addr + KV_DK + hf * (D / 2), D / 64);
+    tmem_zero(lane_addr + L::DV_COL + hf * (D / 2), D / 64);
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
       const int st = u % TNST, bf = u & 1;
-      const int64_t q0 = q0_of(u);
-      const uint32_t s_addr = lane_addr + KV_S + 64 * bf, dp_addr = lane_addr + KV_DP + 64 * bf;
-      const SubPlan pl = plan_of(u);
-      const int32_t *cut = cuts + 8 * head_of(u);
-      if (pl.bnd) {
+      const int64_t q0 = q0_of(u) + cb;  // query of my first column
+      const uint32_t s_addr = lane_addr + KV_S + 64 * bf + cb, dp_addr = lane_addr + KV_DP + 64 * bf + cb;
+      if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const uint32_t w = plans[2 * st];
+      const int32_t *cut = cuts + 8 * static_cast<int>(plans[2 * st + 1]);
+      if (pw_bnd(w)) {
         // S^T masked in place after each boundary class: keep query c iff (q0 + c) - j <= W
         int64_t prev = -1;
         int32_t W;
         uint32_t cls;
-        while (next_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+        while (next_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
           ok = warp_wait(bnd_ready, bnd_cnt & 1, lim, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const int64_t cm = j - q0 + W;
-          const int cmax = cm < -1 ? -1 : (cm > TBS - 1 ? TBS - 1 : static_cast<int>(cm));
-          uint32_t su[64];
-          tmem_ld64(s_addr, su);
+          const int cmax = cm < -1 ? -1 : (cm > 31 ? 31 : static_cast<int>(cm));
+          uint32_t su[32];
+          tmem_ld32(s_addr, su);
+          tmem_wait_ld(su);
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c > cmax) su[c] = 0u;
-          tmem_st32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&su[0]));
-          tmem_st32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&su[32]));
+          tmem_st32(s_addr, su);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -854,41 +902,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
       }
-      // the sub-tile's LSE and D (the producer wrote them before its loads)
-      if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag) ||
-          !warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
+      if (!warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512);
-      uint32_t su[64], dp[64];
-      load_half(s_addr, (pl.full | pl.bnd) != 0u, su);
-      tmem_ld64(dp_addr, dp);
-      // P^T = exp2(S^T c2 - LSE_i log2 e) on the causal pairs i >= j, dS^T = P^T (dP^T - D_i)
-      const int64_t cmin = j - q0;  // first causal query column
-      const int64_t cval = N - 1 - q0;  // last valid query column
-      float pf[64], ds[64];
+      uint32_t su[32], dp[32];
+      if (pw_full(w) | pw_bnd(w)) {
+        tmem_ld32x2(s_addr, su, dp_addr, dp);
+      } else {
+        tmem_ld32(dp_addr, dp);
+        tmem_wait_ld(dp);
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c = 0; c < 32; ++c) su[c] = 0u;
+      }
+      // P^T = exp2(S^T c2 - LSE_i log2 e) on the causal pairs i >= j of valid
+      // queries, dS^T = P^T (dP^T - D_i)
+      const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512) + hf * 8;
+      const int64_t cm0 = j - q0, cv = N - 1 - q0;  // my first causal and last valid column
+      const int lo = !row_ok ? 32 : (cm0 < 0 ? 0 : (cm0 > 32 ? 32 : static_cast<int>(cm0)));
+      const int hi = cv > 31 ? 31 : static_cast<int>(cv);
+      float pf[32], ds[32];
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 l4 = ld4[c4], d4 = ld4[16 + c4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = 4 * c4 + e;
-          const bool live = row_ok && c >= cmin && c <= cval;
-          const float p = fast_exp2(fmaf(__uint_as_float(su[c]), c2, -lv[e]));
-          pf[c] = live ? p : 0.f;
-          ds[c] = live ? p * (__uint_as_float(dp[c]) - dv[e]) : 0.f;
+        for (int e = 0; e < 2; ++e) {
+          const int c = 4 * c4 + 2 * e;
+          const float la = e == 0 ? l4.x : l4.z, lb = e == 0 ? l4.y : l4.w;
+          const float da = e == 0 ? d4.x : d4.z, db = e == 0 ? d4.y : d4.w;
+          const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[c]), __uint_as_float(su[c + 1])), c2x2,
+                                    pack_f2(-la, -lb));
+          float x0, x1;
+          unpack_f2(x2, x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          const uint64_t g2 = fsub2(pack_f2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), pack_f2(da, db));
+          float d0, d1;
+          unpack_f2(fmul2(pack_f2(p0, p1), g2), d0, d1);
+          pf[c] = p0;
+          pf[c + 1] = p1;
+          ds[c] = d0;
+          ds[c + 1] = d1;
         }
       }
-      {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) pk[k] = pack_bf16x2(pf[2 * k], pf[2 * k + 1]);
-        tmem_st32(s_addr, pk);
-      }
-      store_ds_upto(dp_addr, ds, TBS - 1);
+      store_bf16_32(s_addr, pf, lo, hi);
+      store_bf16_32(dp_addr, ds, lo, hi);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -896,12 +954,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int64_t prev = INT64_MAX;
       int32_t W;
       uint32_t cls;
-      while (prev_boundary_class(cut, pl.bnd, prev, &W, &cls)) {
+      while (prev_boundary_class(cut, pw_bnd(w), prev, &W, &cls)) {
         ok = warp_wait(dsm_req, dsm_cnt & 1, lim, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const int64_t cm = j - q0 + W;
-        store_ds_upto(dp_addr, ds, cm < -1 ? -1 : (cm > TBS - 1 ? TBS - 1 : static_cast<int>(cm)));
+        const int cmax = cm < -1 ? -1 : (cm > 31 ? 31 : static_cast<int>(cm));
+        store_bf16_32(dp_addr, ds, lo, hi < cmax ? hi : cmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -910,36 +969,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prev = W;
       }
     }
-    __nv_bfloat16 *dkrow = a.dk + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D;
-    __nv_bfloat16 *dvrow = a.dv + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D;
+    __nv_bfloat16 *dkrow = a.dk + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + hf * (D / 2);
+    __nv_bfloat16 *dvrow = a.dv + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + hf * (D / 2);
     if (ok && nsub > 0 && warp_wait(kv_final, 0, lim, abort_flag)) {
       tc_fence_after();
-#pragma unroll
-      for (int c4 = 0; c4 < 2 * D / 32; ++c4) {
-        uint32_t u32[32];
-        tmem_ld32(lane_addr + KV_DK + 32 * c4, u32);
-        tmem_wait_ld(u32);
-        const float sc = c4 < D / 32 ? a.scale : 1.f;  // dK carries the softmax scale, dV not
-        uint4 pk4[4];
-        uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
-#pragma unroll
-        for (int k = 0; k < 16; ++k)
-          pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * sc, __uint_as_float(u32[2 * k + 1]) * sc);
-        if (row_ok) {
-          uint4 *dst = reinterpret_cast<uint4 *>(c4 < D / 32 ? dkrow + 32 * c4 : dvrow + 32 * (c4 - D / 32));
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = pk4[k];
-        }
+      for (int c = 0; c < D / 64; ++c) {
+        store_row32(lane_addr + KV_DK + hf * (D / 2) + 32 * c, a.scale, dkrow + 32 * c, row_ok);
+        store_row32(lane_addr + L::DV_COL + hf * (D / 2) + 32 * c, 1.f, dvrow + 32 * c, row_ok);
       }
     } else {
       *abort_flag = 1;
       if (row_ok) {
-        const uint4 nan4 = make_uint4(0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u, 0x7FC07FC0u);
-#pragma unroll
-        for (int k = 0; k < D / 8; ++k) {
-          reinterpret_cast<uint4 *>(dkrow)[k] = nan4;
-          reinterpret_cast<uint4 *>(dvrow)[k] = nan4;
-        }
+        store_nan(dkrow, D / 2);
+        store_nan(dvrow, D / 2);
       }
     }
   }
@@ -954,18 +996,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 template <int D>
-cudaError_t launch_dkdv(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t stream) {
-  // one CTA per SM: the kernel holds all 512 TMEM columns
-  const uint32_t smem = KvTL<D>::BYTES > 120u * 1024u ? KvTL<D>::BYTES : 120u * 1024u;
-  cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dkdv_tc_kernel<D><<<dim3((a.N + TBQ - 1) / TBQ, a.Hkv, a.B), TC_THREADS, smem, stream>>>(m.k128, m.v128, m.q64,
-                                                                                         m.do64, a);
-  return cudaGetLastError();
-}
-
-template <int D>
 cudaError_t launch_dq(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t stream) {
   // one CTA per SM: the kernel holds all 512 TMEM columns
   const uint32_t smem = DqTL<D>::BYTES > 120u * 1024u ? DqTL<D>::BYTES : 120u * 1024u;
@@ -974,6 +1004,17 @@ cudaError_t launch_dq(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t
   if (e != cudaSuccess) return e;
   dq_tc_kernel<D><<<dim3((a.N + TBQ - 1) / TBQ, a.Hq, a.B), TC_THREADS, smem, stream>>>(m.q128, m.do128, m.k64,
                                                                                        m.v64, a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_dkdv(const BackwardArgs &a, const BackwardMaps &m, cudaStream_t stream) {
+  const uint32_t smem = KvTL<D>::BYTES > 120u * 1024u ? KvTL<D>::BYTES : 120u * 1024u;
+  cudaError_t e = cudaFuncSetAttribute(dkdv_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dkdv_tc_kernel<D><<<dim3((a.N + TBQ - 1) / TBQ, a.Hkv, a.B), TC_THREADS, smem, stream>>>(m.k128, m.v128, m.q64,
+                                                                                         m.do64, a);
   return cudaGetLastError();
 }
 
