@@ -626,7 +626,7 @@ def run_ours(args, rank, world, local):
             times.setdefault(cut, []).append(t)
         wave_ms, dense_ms = min(times["wave"]), min(times["dense"])
         wave_ms, dense_ms = max_over_ranks([wave_ms, dense_ms], dev)
-        backward = {"kernel": "wp_prefill_backward (delta + dQ + dK/dV, warp-level mma.sync)",
+        backward = {"kernel": "wp_prefill_backward (delta + dQ + dK/dV on tcgen05)",
                     "ms": round(wave_ms, 3), "dense_ms": round(dense_ms, 3),
                     "useful_tflops": round(bw_useful / (wave_ms * 1e-3) / 1e12, 2),
                     "dense_tflops": round(bw_dense / (dense_ms * 1e-3) / 1e12, 2),

@@ -221,10 +221,13 @@ size_t wp_prefill_backward_workspace_bytes(int B, int N, int H_q);
  *   cut, cut_rows  group cutoffs as in wp_prefill_ex: cut_rows = 1 (cut
  *               [d_h/16], or NULL: dense) or H_q ([H_q][d_h/16]).
  *   softmax_scale  the forward's scale (<= 0: 1/sqrt(d_h)).
- * Grouped mode only. The products run on warp-level tensor cores with bf16
- * operands (P and dS rounded to bf16) and fp32 accumulation. d_h in
- * {64, 128}. Errors: WP_ERR_ARG, WP_ERR_UNSUPPORTED (also: more than 2048
- * table entries; more than 64 query heads per KV head), WP_ERR_CUDA.
+ * Grouped mode only. The products run on the tcgen05 tensor cores with bf16
+ * operands (P and dS rounded to bf16) and fp32 accumulation in TMEM. The
+ * status word (wp_device_status) works as for wp_prefill: a wait that gives
+ * up records WP_ERR_TIMEOUT and the affected rows of dq, dk, dv are NaN.
+ * d_h in {64, 128}. Errors: WP_ERR_ARG, WP_ERR_UNSUPPORTED (also: more than
+ * 2048 table entries; more than 64 query heads per KV head; N above
+ * 128 * 65535), WP_ERR_CUDA.
  */
 int wp_prefill_backward(const void *q, const void *k, const void *v, const void *o, const void *dout, const float *lse,
                         void *dq, void *dk, void *dv, void *workspace, size_t ws_bytes, int B, int N, int H_q,

@@ -18,7 +18,7 @@
 //   warp 8   TMA producer: Q and dO of the block once (16-dim boxes, 32-byte
 //            swizzle); per sub-tile the K group tiles some group needs, V and
 //            the sub-tile's group classes (a plan word beside the stage),
-//            three stages.
+//            four stages.
 //   warp 9   MMA issuer: S(u) = sum_g Q_g K_g^T (M128 N64 K16 per non-skipped
 //            group) and dP(u) = dO V^T into double-buffered TMEM, then, once
 //            the row warps have written dS(u) (bf16, over S's first 32
@@ -66,10 +66,13 @@ namespace {
 
 constexpr int TBQ = 128;  // rows of a CTA's block
 constexpr int TBS = 64;   // columns of a sub-tile
-constexpr int TNST = 3;   // stages of the streamed operands
-constexpr int TC_THREADS = 320;  // warps 0-7 row warps, 8 TMA producer, 9 MMA issuer
-constexpr int NROWW = 8;
-constexpr int T_PROD = 8, T_MMA = 9;
+constexpr int TNST = 4;   // stages of the streamed operands
+constexpr int CSPLIT = 2;               // row warps per TMEM lane quarter: the sub-tile's columns split
+constexpr int COLS = TBS / CSPLIT;      // columns of one row warp
+constexpr int NROWW = 4 * CSPLIT;       // row warps
+constexpr int TC_THREADS = 32 * (NROWW + 2);  // + TMA producer, MMA issuer
+constexpr int T_PROD = NROWW, T_MMA = NROWW + 1;
+static_assert(COLS == 16 || COLS == 32, "row warps take 16 or 32 columns");
 constexpr uint32_t TILE128 = 128 * 32;  // a 16-dim group tile of 128 rows
 constexpr uint32_t TILE64 = 64 * 32;    // a 16-dim group tile of 64 rows
 constexpr float TLOG2E = 1.4426950408889634f;
@@ -117,51 +120,106 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 32 TMEM columns at each of two addresses, one wait for both.
-__device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t (&r0)[32], uint32_t a1, uint32_t (&r1)[32]) {
-  tmem_ld32(a0, r0);
-  tmem_ld32(a1, r1);
-  tmem_wait_ld(r0);
-  tmem_wait_ld(r1);
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
+[[maybe_unused]] __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
-// 32 fp32 values as bf16 pairs into 16 TMEM columns; columns outside
-// [lo, hi] (0-based within the 32) written as 0.
-__device__ __forceinline__ void store_bf16_32(uint32_t taddr, const float (&x)[32], int lo, int hi) {
-  uint32_t pk[16];
+// COLS TMEM columns of this warp's lanes into r (and waited for).
+template <int NC>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
+  if constexpr (NC == 32) {
+    tmem_ld32(taddr, r);
+    tmem_wait_ld(r);
+  } else {
+    tmem_ld16(taddr, r);
+    tmem_wait_ld16(r);
+  }
+}
+// COLS columns at each of two addresses, one wait for both.
+template <int NC>
+__device__ __forceinline__ void ld_cols2(uint32_t a0, uint32_t (&r0)[NC], uint32_t a1, uint32_t (&r1)[NC]) {
+  if constexpr (NC == 32) {
+    tmem_ld32(a0, r0);
+    tmem_ld32(a1, r1);
+    tmem_wait_ld(r0);
+    tmem_wait_ld(r1);
+  } else {
+    tmem_ld16(a0, r0);
+    tmem_ld16(a1, r1);
+    tmem_wait_ld16(r0);
+    tmem_wait_ld16(r1);
+  }
+}
+template <int NC>
+__device__ __forceinline__ void st_cols(uint32_t taddr, const uint32_t (&r)[NC]) {
+  if constexpr (NC == 32)
+    tmem_st32(taddr, r);
+  else
+    tmem_st16(taddr, r);
+}
+
+// COLS fp32 values as bf16 pairs into COLS / 2 TMEM columns; columns outside
+// [lo, hi] (0-based within the COLS) written as 0.
+template <int NC>
+__device__ __forceinline__ void store_bf16_cols(uint32_t taddr, const float (&x)[NC], int lo, int hi) {
+  uint32_t pk[NC / 2];
 #pragma unroll
-  for (int k = 0; k < 16; ++k)
+  for (int k = 0; k < NC / 2; ++k)
     pk[k] = pack_bf16x2(2 * k < lo || 2 * k > hi ? 0.f : x[2 * k], 2 * k + 1 < lo || 2 * k + 1 > hi ? 0.f : x[2 * k + 1]);
-  tmem_st16(taddr, pk);
+  if constexpr (NC == 32)
+    tmem_st16(taddr, pk);
+  else
+    tmem_st8(taddr, pk);
 }
 
-// TMEM address of K16 step kk of a bf16 operand written by the two column
-// halves: keys (or queries) 16 kk .. belong to half kk / 2, which keeps its
-// 16 packed columns at the start of its own 32.
-__device__ __forceinline__ uint32_t half_operand(uint32_t base, int kk) { return base + 32 * (kk >> 1) + 8 * (kk & 1); }
+// TMEM address of K16 step kk of a bf16 operand written by the column
+// splits: keys (or queries) 16 kk .. belong to split 16 kk / COLS, which
+// keeps its COLS / 2 packed columns at the start of its own COLS.
+__device__ __forceinline__ uint32_t split_operand(uint32_t base, int kk) {
+  return base + COLS * (16 * kk / COLS) + (16 * kk % COLS) / 2;
+}
 
-// Zero n32 x 32 TMEM columns of this warp's lanes.
-__device__ __forceinline__ void tmem_zero(uint32_t taddr, int n32) {
-  uint32_t z[32];
+// Zero n16 x 16 TMEM columns of this warp's lanes.
+__device__ __forceinline__ void tmem_zero16(uint32_t taddr, int n16) {
+  uint32_t z[16];
 #pragma unroll
-  for (int k = 0; k < 32; ++k) z[k] = 0u;
-  for (int c = 0; c < n32; ++c) tmem_st32(taddr + 32 * c, z);
+  for (int k = 0; k < 16; ++k) z[k] = 0u;
+  for (int c = 0; c < n16; ++c) tmem_st16(taddr + 16 * c, z);
   tmem_wait_st();
 }
 
-// Scale 32 fp32 TMEM columns, write them to global memory as bf16 (16-byte stores).
-__device__ __forceinline__ void store_row32(uint32_t taddr, float scale, __nv_bfloat16 *dst, bool ok) {
-  uint32_t u32[32];
-  tmem_ld32(taddr, u32);
-  tmem_wait_ld(u32);
-  uint4 pk4[4];
+// Scale 16 fp32 TMEM columns, write them to global memory as bf16 (16-byte stores).
+__device__ __forceinline__ void store_row16(uint32_t taddr, float scale, __nv_bfloat16 *dst, bool ok) {
+  uint32_t u16[16];
+  tmem_ld16(taddr, u16);
+  tmem_wait_ld16(u16);
+  uint4 pk4[2];
   uint32_t *pw = reinterpret_cast<uint32_t *>(pk4);
 #pragma unroll
-  for (int k = 0; k < 16; ++k)
-    pw[k] = pack_bf16x2(__uint_as_float(u32[2 * k]) * scale, __uint_as_float(u32[2 * k + 1]) * scale);
+  for (int k = 0; k < 8; ++k)
+    pw[k] = pack_bf16x2(__uint_as_float(u16[2 * k]) * scale, __uint_as_float(u16[2 * k + 1]) * scale);
   if (ok) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) reinterpret_cast<uint4 *>(dst)[k] = pk4[k];
+    reinterpret_cast<uint4 *>(dst)[0] = pk4[0];
+    reinterpret_cast<uint4 *>(dst)[1] = pk4[1];
   }
 }
 
@@ -209,7 +267,7 @@ struct DqTL {
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // the head's group cutoffs, 8 int32
   static constexpr uint32_t PLAN_OFF = CUT_OFF + 32;  // plan word per stage
-  static constexpr uint32_t BYTES = PLAN_OFF + 16 + 1024;
+  static constexpr uint32_t BYTES = PLAN_OFF + 4 * TNST + 1024;
 };
 
 template <int D>
@@ -293,7 +351,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int issued = 0;
     for (int u = 0; u < nsub; ++u) {
       const int st = u % TNST;
-      if (u >= TNST && !warp_wait_idle(&kv_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
+      if (u >= TNST && !warp_wait_idle<32>(&kv_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
       int64_t dmin = 0, dmax = -1;
       const bool any = tile_distance_range(N, TBQ, TBS, qb, 2 * qb + 1 - u, &dmin, &dmax);
       const uint32_t w = plan_word(cut, G, any, dmin, dmax);
@@ -399,7 +457,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + DQ_ACC + 16 * g0, half_operand(tmem + DQ_S + 64 * bf, kk),
+            umma_ts(tmem + DQ_ACC + 16 * g0, split_operand(tmem + DQ_S + 64 * bf, kk),
                     kst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
@@ -446,7 +504,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     warp_wait(drain, 0, lim, nullptr);
   } else if (warp < NROWW) {
     // ---------------------------------------------------------- row warps
-    const int q4 = warp & 3, hf = warp >> 2, cb = 32 * hf;  // lane quarter, first column
+    const int q4 = warp & 3, cq = warp >> 2, cb = COLS * cq;  // lane quarter, first column
     const int r = q4 * 32 + lane;
     const int64_t i = static_cast<int64_t>(qb) * TBQ + r;
     const bool row_ok = i < N;
@@ -455,7 +513,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const float lse2 = row_ok ? a.lse[lrow] * TLOG2E : 0.f;
     const float di = row_ok ? a.delta[lrow] : 0.f;
     const uint64_t c2x2 = pack_f2(a.scale_log2, a.scale_log2), nl2 = pack_f2(-lse2, -lse2), nd2 = pack_f2(-di, -di);
-    tmem_zero(lane_addr + DQ_ACC + hf * (D / 2), D / 64);  // every dQ product accumulates
+    constexpr int DPW = D / CSPLIT;  // accumulator columns of this warp in the epilogue
+    tmem_zero16(lane_addr + DQ_ACC + cq * DPW, DPW / 16);  // every dQ product accumulates
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
@@ -477,14 +536,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const int64_t cm = i - k0 - W;
-          const int cmin = cm < 0 ? 0 : (cm > 32 ? 32 : static_cast<int>(cm));
-          uint32_t su[32];
-          tmem_ld32(s_addr, su);
-          tmem_wait_ld(su);
+          const int cmin = cm < 0 ? 0 : (cm > COLS ? COLS : static_cast<int>(cm));
+          uint32_t su[COLS];
+          ld_cols(s_addr, su);
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < COLS; ++c)
             if (c < cmin) su[c] = 0u;
-          tmem_st32(s_addr, su);
+          st_cols(s_addr, su);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -499,21 +557,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      uint32_t su[32], dp[32];
+      uint32_t su[COLS], dp[COLS];
       if (pw_full(w) | pw_bnd(w)) {
-        tmem_ld32x2(s_addr, su, lane_addr + DQ_DP + 64 * bf + cb, dp);
+        ld_cols2(s_addr, su, lane_addr + DQ_DP + 64 * bf + cb, dp);
       } else {
-        tmem_ld32(lane_addr + DQ_DP + 64 * bf + cb, dp);
-        tmem_wait_ld(dp);
+        ld_cols(lane_addr + DQ_DP + 64 * bf + cb, dp);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) su[c] = 0u;
+        for (int c = 0; c < COLS; ++c) su[c] = 0u;
       }
       // P = exp2(S c2 - LSE log2 e) and dS = P (dP - D) on the causal pairs of a valid row
       const int64_t jm = i - k0;  // my last causal column
-      const int jmax = !row_ok ? -1 : (jm > 31 ? 31 : (jm < -1 ? -1 : static_cast<int>(jm)));
-      float ds[32];
+      const int jmax = !row_ok ? -1 : (jm > COLS - 1 ? COLS - 1 : (jm < -1 ? -1 : static_cast<int>(jm)));
+      float ds[COLS];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
+      for (int k = 0; k < COLS / 2; ++k) {
         const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[2 * k]), __uint_as_float(su[2 * k + 1])), c2x2, nl2);
         float x0, x1;
         unpack_f2(x2, x0, x1);
@@ -523,7 +580,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ds[2 * k] = d0;
         ds[2 * k + 1] = d1;
       }
-      store_bf16_32(s_addr, ds, 0, jmax);
+      store_bf16_cols(s_addr, ds, 0, jmax);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -537,7 +594,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int64_t cm = i - k0 - W;
-        store_bf16_32(s_addr, ds, cm < 0 ? 0 : (cm > 32 ? 32 : static_cast<int>(cm)), jmax);
+        store_bf16_cols(s_addr, ds, cm < 0 ? 0 : (cm > COLS ? COLS : static_cast<int>(cm)), jmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -546,14 +603,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prev = W;
       }
     }
-    __nv_bfloat16 *dqrow = a.dq + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D + hf * (D / 2);
+    __nv_bfloat16 *dqrow = a.dq + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D + cq * DPW;
     if (ok && nsub > 0 && warp_wait(dq_final, 0, lim, abort_flag)) {
       tc_fence_after();
-      for (int c = 0; c < D / 64; ++c)
-        store_row32(lane_addr + DQ_ACC + hf * (D / 2) + 32 * c, a.scale, dqrow + 32 * c, row_ok);
+      for (int c = 0; c < DPW / 16; ++c)
+        store_row16(lane_addr + DQ_ACC + cq * DPW + 16 * c, a.scale, dqrow + 16 * c, row_ok);
     } else {
       *abort_flag = 1;
-      if (row_ok) store_nan(dqrow, D / 2);
+      if (row_ok) store_nan(dqrow, DPW);
     }
   }
 
@@ -589,7 +646,7 @@ struct KvTL {
   static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr uint32_t PLAN_OFF = MISC_OFF + 16;  // plan word and head of each stage
-  static constexpr uint32_t CUT_OFF = PLAN_OFF + 32;   // cutoff rows of the KV head's query heads, [rep][8]
+  static constexpr uint32_t CUT_OFF = PLAN_OFF + 8 * TNST;  // cutoff rows of the KV head's query heads, [rep][8]
   static constexpr uint32_t BYTES = CUT_OFF + 64 * 8 * 4 + 1024;
 };
 
@@ -680,14 +737,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int issued = 0;
     for (int u = 0; u < nsub; ++u) {
       const int st = u % TNST;
-      if (u >= TNST && !warp_wait_idle(&qd_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
+      if (u >= TNST && !warp_wait_idle<32>(&qd_empty[st], ((u / TNST) - 1) & 1, lim, abort_flag)) break;
       const int hr = u / per_head;
       const int h = hk * rep + hr;
       const int64_t q0 = q0_of(u);
       int64_t dmin = 0, dmax = -1;
       const bool any = tile_distance_range(N, TBS, TBQ, 2 * kb + u % per_head, kb, &dmin, &dmax);
       const uint32_t w = plan_word(cuts + 8 * hr, G, any, dmin, dmax);
-      // the plan, and the sub-tile's LSE (log2 units) and D, read by the row warps
+      // The bulk copies go out first; the plan and the sub-tile's LSE (log2
+      // units) and D, which the row warps read, are written while they fly,
+      // and the arrival that carries the expected bytes comes last (the
+      // copies' completions may precede it: the phase waits for both).
+      const uint32_t need = pw_full(w) | pw_bnd(w);
+      if (leader) {
+        for (uint32_t m = need; m; m &= m - 1) {
+          const int g = __ffs(m) - 1;
+          tma_load_4d(smem + L::Q_OFF + st * L::STAGE + g * TILE64, &tm_q, &qd_full[st], 16 * g, h,
+                      static_cast<int>(q0), b);
+        }
+        for (int g = 0; g < G; ++g)
+          tma_load_4d(smem + L::DO_OFF + st * L::STAGE + g * TILE64, &tm_do, &qd_full[st], 16 * g, h,
+                      static_cast<int>(q0), b);
+      }
       float *ld = reinterpret_cast<float *>(smem + L::LD_OFF + st * 512);
       const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N;
       for (int c = lane; c < TBS; c += 32) {
@@ -700,18 +771,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         plans[2 * st + 1] = static_cast<uint32_t>(hr);
       }
       __syncwarp();
-      const uint32_t need = pw_full(w) | pw_bnd(w);
-      if (leader) {
-        mbar_arrive_expect_tx(&qd_full[st], (__popc(need) + G) * TILE64);
-        for (uint32_t m = need; m; m &= m - 1) {
-          const int g = __ffs(m) - 1;
-          tma_load_4d(smem + L::Q_OFF + st * L::STAGE + g * TILE64, &tm_q, &qd_full[st], 16 * g, h,
-                      static_cast<int>(q0), b);
-        }
-        for (int g = 0; g < G; ++g)
-          tma_load_4d(smem + L::DO_OFF + st * L::STAGE + g * TILE64, &tm_do, &qd_full[st], 16 * g, h,
-                      static_cast<int>(q0), b);
-      }
+      if (leader) mbar_arrive_expect_tx(&qd_full[st], (__popc(need) + G) * TILE64);
       __syncwarp();
       ++issued;
     }
@@ -797,7 +857,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + KV_DK + 16 * g0, half_operand(tmem + KV_DP + 64 * bf, kk),
+            umma_ts(tmem + KV_DK + 16 * g0, split_operand(tmem + KV_DP + 64 * bf, kk),
                     qst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
@@ -814,7 +874,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t dost = domn_desc + ((st * L::STAGE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < TBS / 16; ++kk)
-          umma_ts(tmem + L::DV_COL, half_operand(tmem + KV_S + 64 * bf, kk), dost + ((kk * 16 * 32) >> 4), IDESC_DV,
+          umma_ts(tmem + L::DV_COL, split_operand(tmem + KV_S + 64 * bf, kk), dost + ((kk * 16 * 32) >> 4), IDESC_DV,
                   1u);
       }
       __syncwarp();
@@ -855,14 +915,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     warp_wait(drain, 0, lim, nullptr);
   } else if (warp < NROWW) {
     // ---------------------------------------------------------- row warps
-    const int q4 = warp & 3, hf = warp >> 2, cb = 32 * hf;  // lane quarter, first column
+    const int q4 = warp & 3, cq = warp >> 2, cb = COLS * cq;  // lane quarter, first column
     const int r = q4 * 32 + lane;
     const int64_t j = static_cast<int64_t>(kb) * TBQ + r;  // this thread's key
     const bool row_ok = j < N;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
     const uint64_t c2x2 = pack_f2(a.scale_log2, a.scale_log2);
-    tmem_zero(lane_addr + KV_DK + hf * (D / 2), D / 64);
-    tmem_zero(lane_addr + L::DV_COL + hf * (D / 2), D / 64);
+    constexpr int DPW = D / CSPLIT;  // accumulator columns of this warp in the epilogue
+    tmem_zero16(lane_addr + KV_DK + cq * DPW, DPW / 16);
+    tmem_zero16(lane_addr + L::DV_COL + cq * DPW, DPW / 16);
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
@@ -885,14 +946,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const int64_t cm = j - q0 + W;
-          const int cmax = cm < -1 ? -1 : (cm > 31 ? 31 : static_cast<int>(cm));
-          uint32_t su[32];
-          tmem_ld32(s_addr, su);
-          tmem_wait_ld(su);
+          const int cmax = cm < -1 ? -1 : (cm > COLS - 1 ? COLS - 1 : static_cast<int>(cm));
+          uint32_t su[COLS];
+          ld_cols(s_addr, su);
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
+          for (int c = 0; c < COLS; ++c)
             if (c > cmax) su[c] = 0u;
-          tmem_st32(s_addr, su);
+          st_cols(s_addr, su);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -907,24 +967,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
-      uint32_t su[32], dp[32];
+      uint32_t su[COLS], dp[COLS];
       if (pw_full(w) | pw_bnd(w)) {
-        tmem_ld32x2(s_addr, su, dp_addr, dp);
+        ld_cols2(s_addr, su, dp_addr, dp);
       } else {
-        tmem_ld32(dp_addr, dp);
-        tmem_wait_ld(dp);
+        ld_cols(dp_addr, dp);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) su[c] = 0u;
+        for (int c = 0; c < COLS; ++c) su[c] = 0u;
       }
       // P^T = exp2(S^T c2 - LSE_i log2 e) on the causal pairs i >= j of valid
       // queries, dS^T = P^T (dP^T - D_i)
-      const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512) + hf * 8;
+      const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512) + cq * (COLS / 4);
       const int64_t cm0 = j - q0, cv = N - 1 - q0;  // my first causal and last valid column
-      const int lo = !row_ok ? 32 : (cm0 < 0 ? 0 : (cm0 > 32 ? 32 : static_cast<int>(cm0)));
-      const int hi = cv > 31 ? 31 : static_cast<int>(cv);
-      float pf[32], ds[32];
+      const int lo = !row_ok ? COLS : (cm0 < 0 ? 0 : (cm0 > COLS ? COLS : static_cast<int>(cm0)));
+      const int hi = cv > COLS - 1 ? COLS - 1 : static_cast<int>(cv);
+      float pf[COLS], ds[COLS];
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
+      for (int c4 = 0; c4 < COLS / 4; ++c4) {
         const float4 l4 = ld4[c4], d4 = ld4[16 + c4];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -945,8 +1004,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ds[c + 1] = d1;
         }
       }
-      store_bf16_32(s_addr, pf, lo, hi);
-      store_bf16_32(dp_addr, ds, lo, hi);
+      store_bf16_cols(s_addr, pf, lo, hi);
+      store_bf16_cols(dp_addr, ds, lo, hi);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -959,8 +1018,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int64_t cm = j - q0 + W;
-        const int cmax = cm < -1 ? -1 : (cm > 31 ? 31 : static_cast<int>(cm));
-        store_bf16_32(dp_addr, ds, lo, hi < cmax ? hi : cmax);
+        const int cmax = cm < -1 ? -1 : (cm > COLS - 1 ? COLS - 1 : static_cast<int>(cm));
+        store_bf16_cols(dp_addr, ds, lo, hi < cmax ? hi : cmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -969,19 +1028,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prev = W;
       }
     }
-    __nv_bfloat16 *dkrow = a.dk + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + hf * (D / 2);
-    __nv_bfloat16 *dvrow = a.dv + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + hf * (D / 2);
+    __nv_bfloat16 *dkrow = a.dk + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + cq * DPW;
+    __nv_bfloat16 *dvrow = a.dv + ((static_cast<int64_t>(b) * a.N + j) * a.Hkv + hk) * D + cq * DPW;
     if (ok && nsub > 0 && warp_wait(kv_final, 0, lim, abort_flag)) {
       tc_fence_after();
-      for (int c = 0; c < D / 64; ++c) {
-        store_row32(lane_addr + KV_DK + hf * (D / 2) + 32 * c, a.scale, dkrow + 32 * c, row_ok);
-        store_row32(lane_addr + L::DV_COL + hf * (D / 2) + 32 * c, 1.f, dvrow + 32 * c, row_ok);
+      for (int c = 0; c < DPW / 16; ++c) {
+        store_row16(lane_addr + KV_DK + cq * DPW + 16 * c, a.scale, dkrow + 16 * c, row_ok);
+        store_row16(lane_addr + L::DV_COL + cq * DPW + 16 * c, 1.f, dvrow + 16 * c, row_ok);
       }
     } else {
       *abort_flag = 1;
       if (row_ok) {
-        store_nan(dkrow, D / 2);
-        store_nan(dvrow, D / 2);
+        store_nan(dkrow, DPW);
+        store_nan(dvrow, DPW);
       }
     }
   }
