@@ -651,6 +651,10 @@ def run_ours(args, rank, world, local):
                  "useful_tflops": round(ex_flops / (ex_ms * 1e-3) / 1e12, 2), "useful_flops": ex_flops,
                  "peak": peaks["bf16_tflops"],
                  "frac": round(ex_flops / (ex_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                 "traffic": (profiled_traffic("prefill_exact_kernel_32k_dram.txt",
+                                              "rope_period_truncated_b200/csrc/wp_prefill_exact.cu")
+                             if args.prefill_n in (0, 32768) and args.grouping == "half-split" else None),
+                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                  "note": "useful FLOPs pair exact: 4 per kept channel per pair (its two dims) + 2*d for PV"}
         path.prefill()  # the grouped forward's outputs again
 
