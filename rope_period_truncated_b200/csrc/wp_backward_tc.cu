@@ -28,10 +28,12 @@
 //   warps 0-7 two threads per query row: warp w reads TMEM lanes 32 (w % 4)..
 //            and the sub-tile's columns 32 (w / 4) .. +31, and forms P and
 //            dS = P (dP - D) there in packed f32x2 arithmetic (no row
-//            reduction is needed: P comes from the forward's LSE). Each writes
-//            its dS as bf16 over the first 16 of its own S columns, and the
-//            MMAs address the two halves separately. The epilogue scales dQ
-//            and writes it as bf16.
+//            reduction is needed: P comes from the forward's LSE). S and dP
+//            have one TMEM buffer: the row warps release it as soon as they
+//            have loaded it, so S(u + 1) runs on the tensor cores while they
+//            compute u, and they write dS as bf16 into one of two operand
+//            buffers that the dQ products read. The epilogue scales dQ and
+//            writes it as bf16.
 // Boundary groups (cutoff inside the sub-tile's distance range), as in the
 // forward kernel: their S products go first, one cutoff class at a time in
 // ascending order, and the row warps mask S in place after each (nested
@@ -39,9 +41,11 @@
 // order: before each class's products the row warps overwrite dS in TMEM
 // with dS masked by that class's cutoff. Both are round trips between the
 // MMA warp and the row warps, so the MMA warp issues S(v) of a sub-tile with
-// boundary classes only after it has issued dQ(v - 1) (a sub-tile without
-// them is issued two ahead): the row warps finish sub-tile v - 1 before they
-// mask S(v), and the MMA warp never waits on them for a later sub-tile.
+// boundary classes only after it has issued dQ(v - 1): the row warps finish
+// sub-tile v - 1 before they mask S(v), and the MMA warp never waits on them
+// for a later sub-tile.
+// (Without boundary classes, S(v) goes out as soon as the row warps have
+// loaded S(v - 1).)
 //
 // dkdv_tc_kernel: one CTA per (128-row key block, KV head), the same roles
 // with keys as rows: K and V of the block once; per 64-query sub-tile (the
@@ -112,6 +116,17 @@ __device__ __forceinline__ bool prev_boundary_class(const int32_t *cut, uint32_t
   *W = static_cast<int32_t>(best);
   *mask = mk;
   return true;
+}
+
+// 4-byte asynchronous copy global -> shared; src_bytes 0 writes zero.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// The barrier's current phase also waits for this thread's earlier cp.async
+// copies (its pending count rises now and falls when they land).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
@@ -191,13 +206,6 @@ __device__ __forceinline__ void store_bf16_cols(uint32_t taddr, const float (&x)
     tmem_st8(taddr, pk);
 }
 
-// TMEM address of K16 step kk of a bf16 operand written by the column
-// splits: keys (or queries) 16 kk .. belong to split 16 kk / COLS, which
-// keeps its COLS / 2 packed columns at the start of its own COLS.
-__device__ __forceinline__ uint32_t split_operand(uint32_t base, int kk) {
-  return base + COLS * (16 * kk / COLS) + (16 * kk % COLS) / 2;
-}
-
 // Zero n16 x 16 TMEM columns of this warp's lanes.
 __device__ __forceinline__ void tmem_zero16(uint32_t taddr, int n16) {
   uint32_t z[16];
@@ -228,28 +236,12 @@ __device__ __forceinline__ void store_nan(__nv_bfloat16 *dst, int n) {
   for (int k = 0; k < n / 8; ++k) reinterpret_cast<uint4 *>(dst)[k] = nan4;
 }
 
-// The MMA warp's issue order, shared by both kernels: S(v) of sub-tile v goes
-// out two ahead of the gradient products, or one ahead when v has boundary
-// classes (its handshakes must follow the row warps' finish of v - 1).
-// `plan(v)` waits for v's stage and returns its plan word; `sdp(v)` issues
-// S(v) and dP(v).
-template <class PlanFn, class SdpFn>
-__device__ __forceinline__ bool advance_sdp(int &next, int done, int nsub, PlanFn plan, SdpFn sdp) {
-  while (next < nsub && next <= done + 2) {
-    uint32_t w;
-    if (!plan(next, w)) return false;
-    if (pw_bnd(w) != 0u && next > done + 1) break;
-    if (!sdp(next, w)) return false;
-    ++next;
-  }
-  return true;
-}
-
 // ============================================================ dQ kernel
 
 // TMEM columns of the dQ kernel
-constexpr uint32_t DQ_S = 0;     // S / dS of buffer b at 64 b
-constexpr uint32_t DQ_DP = 128;  // dP of buffer b at 128 + 64 b
+constexpr uint32_t DQ_S = 0;     // S (fp32, 64 columns)
+constexpr uint32_t DQ_DP = 64;   // dP
+constexpr uint32_t DQ_OB = 128;  // dS as bf16, operand buffer b at 128 + 32 b
 constexpr uint32_t DQ_ACC = 256;
 
 template <int D>
@@ -261,9 +253,9 @@ struct DqTL {
   static constexpr uint32_t STAGE = G * TILE64;
   static constexpr uint32_t V_OFF = K_OFF + TNST * STAGE;
   static constexpr uint32_t BAR_OFF = V_OFF + TNST * STAGE;
-  // qd_full, kv_full[TNST], kv_empty[TNST], s_ready[2], ds_ready[2],
-  // bnd_ready, bnd_done, dsm_req, dsm_done, dq_final, drain
-  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
+  // qd_full, kv_full[TNST], kv_empty[TNST], s_ready, s_free, ds_ready[2],
+  // ob_free[2], bnd_ready, bnd_done, dsm_req, dsm_done, dq_final, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 12;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr uint32_t CUT_OFF = MISC_OFF + 16;  // the head's group cutoffs, 8 int32
   static constexpr uint32_t PLAN_OFF = CUT_OFF + 32;  // plan word per stage
@@ -286,9 +278,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t *qd_full = bars;
   uint64_t *kv_full = bars + 1;
   uint64_t *kv_empty = kv_full + TNST;
-  uint64_t *s_ready = kv_empty + TNST;  // [2 buffers]
-  uint64_t *ds_ready = s_ready + 2;     // [2 buffers]
-  uint64_t *bnd_ready = ds_ready + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
+  uint64_t *s_ready = kv_empty + TNST, *s_free = s_ready + 1;
+  uint64_t *ds_ready = s_free + 1;   // [2 operand buffers]
+  uint64_t *ob_free = ds_ready + 2;  // [2 operand buffers]
+  uint64_t *bnd_ready = ob_free + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
   uint64_t *dq_final = dsm_done + 1, *drain = dq_final + 1;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
@@ -310,9 +303,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
+    mbar_init(s_ready, 1);
+    mbar_init(s_free, NROWW);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_ready[s], 1);
       mbar_init(&ds_ready[s], NROWW);
+      mbar_init(&ob_free[s], 1);
     }
     mbar_init(bnd_ready, 1);
     mbar_init(bnd_done, NROWW);
@@ -397,11 +392,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       w = plans[u % TNST];
       return true;
     };
-    // S(u) and dP(u) into buffer u & 1 (its stage loaded)
+    // S(u) and dP(u) into the S buffer (its stage loaded, S(u - 1) loaded by the row warps)
     auto issue_sdp = [&](int u, uint32_t w) -> bool {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       tc_fence_after();
-      const uint32_t s_col = tmem + DQ_S + 64 * bf;
+      const uint32_t s_col = tmem + DQ_S;
       const uint64_t kst = k_desc + ((st * L::STAGE) >> 4);
       uint32_t acc = 0;
       if (pw_bnd(w)) {
@@ -437,17 +432,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (pw_any(w)) {
 #pragma unroll
           for (int g = 0; g < G; ++g)
-            umma_ss(tmem + DQ_DP + 64 * bf, do_desc + g * GD128, vst + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
+            umma_ss(tmem + DQ_DP, do_desc + g * GD128, vst + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
         }
-        umma_commit(&s_ready[bf]);
+        umma_commit(s_ready);
       }
       __syncwarp();
       return true;
     };
     // dQ[groups] += dS(u) K[groups], one product set per run of consecutive groups
     auto issue_dq_groups = [&](int u, uint32_t groups) {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       const uint64_t kst = kmn_desc + ((st * L::STAGE) >> 4);
+      const uint32_t ob = tmem + DQ_OB + 32 * (u & 1);
       while (groups) {
         const int g0 = __ffs(groups) - 1;
         int g1 = g0;
@@ -457,8 +453,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + DQ_ACC + 16 * g0, split_operand(tmem + DQ_S + 64 * bf, kk),
-                    kst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
+            umma_ts(tmem + DQ_ACC + 16 * g0, ob + 8 * kk, kst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
       }
@@ -480,21 +475,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         issue_dq_groups(u, cls);
         prev = W;
       }
-      if (leader) umma_commit(&kv_empty[u % TNST]);
+      if (leader) {
+        umma_commit(&kv_empty[u % TNST]);
+        umma_commit(&ob_free[u & 1]);
+      }
       __syncwarp();
       return true;
     };
+    // S(v + 1) once the row warps have loaded S(v)
+    auto next_sdp = [&](int v) -> bool {
+      uint32_t w;
+      if (!warp_wait(s_free, v & 1, lim, abort_flag) || !plan(v + 1, w)) return false;
+      return issue_sdp(v + 1, w);
+    };
 
-    int next = 0;
-    if (ok) ok = advance_sdp(next, -1, nsub, plan, issue_sdp);
+    if (ok && nsub > 0) {
+      uint32_t w;
+      ok = plan(0, w) && issue_sdp(0, w);
+    }
     for (int u = 0; ok && u < nsub; ++u) {
+      // S(u + 1) overlaps the row warps' work on u, unless it has boundary
+      // classes: then its handshakes follow dQ(u) and the row warps' masking for u
+      bool early = false;
+      if (u + 1 < nsub) {
+        uint32_t w1;
+        if (!plan(u + 1, w1)) {
+          ok = false;
+          break;
+        }
+        if (pw_bnd(w1) == 0u) {
+          early = true;
+          if (!(ok = next_sdp(u))) break;
+        }
+      }
       if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       ok = issue_dq(u);
-      if (ok) ok = advance_sdp(next, u, nsub, plan, issue_sdp);
+      if (ok && u + 1 < nsub && !early) ok = next_sdp(u);
     }
     if (leader) {
       umma_commit(dq_final);
@@ -509,6 +529,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int64_t i = static_cast<int64_t>(qb) * TBQ + r;
     const bool row_ok = i < N;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t s_addr = lane_addr + DQ_S + cb, dp_addr = lane_addr + DQ_DP + cb;
     const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N + (row_ok ? i : 0);
     const float lse2 = row_ok ? a.lse[lrow] * TLOG2E : 0.f;
     const float di = row_ok ? a.delta[lrow] : 0.f;
@@ -518,9 +539,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       const int64_t k0 = static_cast<int64_t>(2 * qb + 1 - u) * TBS + cb;  // first key of my columns
-      const uint32_t s_addr = lane_addr + DQ_S + 64 * bf + cb;
+      const uint32_t ob_addr = lane_addr + DQ_OB + 32 * (u & 1) + (COLS / 2) * cq;
       if (!warp_wait(&kv_full[st], (u / TNST) & 1, lim, abort_flag)) {
         ok = false;
         break;
@@ -552,19 +573,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
       }
-      if (!warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
+      if (!warp_wait(s_ready, u & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t su[COLS], dp[COLS];
       if (pw_full(w) | pw_bnd(w)) {
-        ld_cols2(s_addr, su, lane_addr + DQ_DP + 64 * bf + cb, dp);
+        ld_cols2(s_addr, su, dp_addr, dp);
       } else {
-        ld_cols(lane_addr + DQ_DP + 64 * bf + cb, dp);
+        ld_cols(dp_addr, dp);
 #pragma unroll
         for (int c = 0; c < COLS; ++c) su[c] = 0u;
       }
+      // S and dP are in registers: the buffer is free for S(u + 1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       // P = exp2(S c2 - LSE log2 e) and dS = P (dP - D) on the causal pairs of a valid row
       const int64_t jm = i - k0;  // my last causal column
       const int jmax = !row_ok ? -1 : (jm > COLS - 1 ? COLS - 1 : (jm < -1 ? -1 : static_cast<int>(jm)));
@@ -580,11 +605,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ds[2 * k] = d0;
         ds[2 * k + 1] = d1;
       }
-      store_bf16_cols(s_addr, ds, 0, jmax);
+      // operand buffer u & 1 is free once dQ(u - 2) has read it
+      if (u >= 2 && !warp_wait(&ob_free[u & 1], ((u >> 1) - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      store_bf16_cols(ob_addr, ds, 0, jmax);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_ready[bf]);
+      if (lane == 0) mbar_arrive(&ds_ready[u & 1]);
       // boundary classes of dQ, descending cutoffs: dS masked for each
       int64_t prev = INT64_MAX;
       int32_t W;
@@ -594,7 +625,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int64_t cm = i - k0 - W;
-        store_bf16_cols(s_addr, ds, cm < 0 ? 0 : (cm > COLS ? COLS : static_cast<int>(cm)), jmax);
+        store_bf16_cols(ob_addr, ds, cm < 0 ? 0 : (cm > COLS ? COLS : static_cast<int>(cm)), jmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -626,8 +657,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // ========================================================= dK/dV kernel
 
 // TMEM columns of the dK/dV kernel
-constexpr uint32_t KV_S = 0;     // S^T / P^T of buffer b at 64 b
-constexpr uint32_t KV_DP = 128;  // dP^T / dS^T of buffer b at 128 + 64 b
+constexpr uint32_t KV_S = 0;     // S^T (fp32, 64 columns)
+constexpr uint32_t KV_DP = 64;   // dP^T
+constexpr uint32_t KV_OB = 128;  // operand buffer b at 128 + 64 b: P^T (bf16, 32 columns), then dS^T
 constexpr uint32_t KV_DK = 256;
 
 template <int D>
@@ -639,13 +671,13 @@ struct KvTL {
   static constexpr uint32_t Q_OFF = V_OFF + G * TILE128;
   static constexpr uint32_t STAGE = G * TILE64;
   static constexpr uint32_t DO_OFF = Q_OFF + TNST * STAGE;
-  static constexpr uint32_t LD_OFF = DO_OFF + TNST * STAGE;  // per stage: LSE (log2 units) and D, 64 each
+  static constexpr uint32_t LD_OFF = DO_OFF + TNST * STAGE;  // per stage: LSE and D of the 64 queries
   static constexpr uint32_t BAR_OFF = LD_OFF + TNST * 512;
-  // kv_full, qd_full[TNST], qd_empty[TNST], s_ready[2], ds_ready[2],
-  // bnd_ready, bnd_done, dsm_req, dsm_done, kv_final, drain
-  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 4 + 6;
+  // kv_full, qd_full[TNST], qd_empty[TNST], s_ready, s_free, ds_ready[2],
+  // ob_free[2], bnd_ready, bnd_done, dsm_req, dsm_done, kv_final, drain
+  static constexpr uint32_t NUM_BARS = 1 + 2 * TNST + 12;
   static constexpr uint32_t MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr uint32_t PLAN_OFF = MISC_OFF + 16;  // plan word and head of each stage
+  static constexpr uint32_t PLAN_OFF = MISC_OFF + 16;       // plan word and head of each stage
   static constexpr uint32_t CUT_OFF = PLAN_OFF + 8 * TNST;  // cutoff rows of the KV head's query heads, [rep][8]
   static constexpr uint32_t BYTES = CUT_OFF + 64 * 8 * 4 + 1024;
 };
@@ -666,9 +698,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t *kv_full = bars;
   uint64_t *qd_full = bars + 1;
   uint64_t *qd_empty = qd_full + TNST;
-  uint64_t *s_ready = qd_empty + TNST;  // [2 buffers]
-  uint64_t *ds_ready = s_ready + 2;     // [2 buffers]
-  uint64_t *bnd_ready = ds_ready + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
+  uint64_t *s_ready = qd_empty + TNST, *s_free = s_ready + 1;
+  uint64_t *ds_ready = s_free + 1;   // [2 operand buffers]
+  uint64_t *ob_free = ds_ready + 2;  // [2 operand buffers]
+  uint64_t *bnd_ready = ob_free + 2, *bnd_done = bnd_ready + 1, *dsm_req = bnd_done + 1, *dsm_done = dsm_req + 1;
   uint64_t *kv_final = dsm_done + 1, *drain = kv_final + 1;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC_OFF);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC_OFF + 4);
@@ -691,9 +724,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
     }
+    mbar_init(s_ready, 1);
+    mbar_init(s_free, NROWW);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_ready[s], 1);
       mbar_init(&ds_ready[s], NROWW);
+      mbar_init(&ob_free[s], 1);
     }
     mbar_init(bnd_ready, 1);
     mbar_init(bnd_done, NROWW);
@@ -744,10 +779,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int64_t dmin = 0, dmax = -1;
       const bool any = tile_distance_range(N, TBS, TBQ, 2 * kb + u % per_head, kb, &dmin, &dmax);
       const uint32_t w = plan_word(cuts + 8 * hr, G, any, dmin, dmax);
-      // The bulk copies go out first; the plan and the sub-tile's LSE (log2
-      // units) and D, which the row warps read, are written while they fly,
-      // and the arrival that carries the expected bytes comes last (the
-      // copies' completions may precede it: the phase waits for both).
+      // The bulk copies go out first, then the sub-tile's LSE and D as
+      // asynchronous 4-byte copies (zero past N) tracked by the same barrier,
+      // and the plan; the arrival that carries the expected bytes comes last
+      // (the copies' completions may precede it: the phase waits for all).
       const uint32_t need = pw_full(w) | pw_bnd(w);
       if (leader) {
         for (uint32_t m = need; m; m &= m - 1) {
@@ -763,9 +798,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int64_t lrow = (static_cast<int64_t>(b) * a.Hq + h) * a.N;
       for (int c = lane; c < TBS; c += 32) {
         const bool in = q0 + c < N;
-        ld[c] = in ? a.lse[lrow + q0 + c] * TLOG2E : 0.f;
-        ld[TBS + c] = in ? a.delta[lrow + q0 + c] : 0.f;
+        const int64_t e = lrow + (in ? q0 + c : 0);
+        cp_async4(ld + c, a.lse + e, in ? 4u : 0u);
+        cp_async4(ld + TBS + c, a.delta + e, in ? 4u : 0u);
       }
+      cp_async_arrive(&qd_full[st]);
       if (lane == 0) {
         plans[2 * st] = w;
         plans[2 * st + 1] = static_cast<uint32_t>(hr);
@@ -799,11 +836,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       w = plans[2 * (u % TNST)];
       return true;
     };
+    // S^T(u) and dP^T(u) into the S buffer
     auto issue_sdp = [&](int u, uint32_t w) -> bool {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       tc_fence_after();
       const int32_t *cut = cuts + 8 * static_cast<int>(plans[2 * st + 1]);
-      const uint32_t s_col = tmem + KV_S + 64 * bf;
+      const uint32_t s_col = tmem + KV_S;
       const uint64_t qst = q_desc + ((st * L::STAGE) >> 4);
       uint32_t acc = 0;
       if (pw_bnd(w)) {
@@ -838,16 +876,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t dost = do_desc + ((st * L::STAGE) >> 4);
 #pragma unroll
         for (int g = 0; g < G; ++g)
-          umma_ss(tmem + KV_DP + 64 * bf, v_desc + g * GD128, dost + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
-        umma_commit(&s_ready[bf]);
+          umma_ss(tmem + KV_DP, v_desc + g * GD128, dost + g * GD64, IDESC_S, g > 0 ? 1u : 0u);
+        umma_commit(s_ready);
       }
       __syncwarp();
       return true;
     };
     // dK[groups] += dS^T Q[groups], one product set per run of consecutive groups
     auto issue_dk_groups = [&](int u, uint32_t groups) {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       const uint64_t qst = qmn_desc + ((st * L::STAGE) >> 4);
+      const uint32_t ob = tmem + KV_OB + 64 * (u & 1) + 32;  // dS^T
       while (groups) {
         const int g0 = __ffs(groups) - 1;
         int g1 = g0;
@@ -857,8 +896,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < TBS / 16; ++kk)
-            umma_ts(tmem + KV_DK + 16 * g0, split_operand(tmem + KV_DP + 64 * bf, kk),
-                    qst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
+            umma_ts(tmem + KV_DK + 16 * g0, ob + 8 * kk, qst + g0 * GD64 + ((kk * 16 * 32) >> 4), idesc, 1u);
         }
         __syncwarp();
       }
@@ -866,16 +904,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // dV(u), then dK(u): full groups on dS^T as it is, then the boundary
     // classes in descending cutoff order, each after the row warps masked dS^T
     auto issue_dkdv = [&](int u) -> bool {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       const uint32_t w = plans[2 * st];
       const int32_t *cut = cuts + 8 * static_cast<int>(plans[2 * st + 1]);
       if (leader) {
         constexpr uint32_t IDESC_DV = idesc_bf16_f32(128, D, false, true);
         const uint64_t dost = domn_desc + ((st * L::STAGE) >> 4);
+        const uint32_t ob = tmem + KV_OB + 64 * (u & 1);  // P^T
 #pragma unroll
         for (int kk = 0; kk < TBS / 16; ++kk)
-          umma_ts(tmem + L::DV_COL, split_operand(tmem + KV_S + 64 * bf, kk), dost + ((kk * 16 * 32) >> 4), IDESC_DV,
-                  1u);
+          umma_ts(tmem + L::DV_COL, ob + 8 * kk, dost + ((kk * 16 * 32) >> 4), IDESC_DV, 1u);
       }
       __syncwarp();
       issue_dk_groups(u, pw_full(w));
@@ -891,21 +929,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         issue_dk_groups(u, cls);
         prev = W;
       }
-      if (leader) umma_commit(&qd_empty[st]);
+      if (leader) {
+        umma_commit(&qd_empty[st]);
+        umma_commit(&ob_free[u & 1]);
+      }
       __syncwarp();
       return true;
     };
+    // S^T(v + 1) once the row warps have loaded S^T(v)
+    auto next_sdp = [&](int v) -> bool {
+      uint32_t w;
+      if (!warp_wait(s_free, v & 1, lim, abort_flag) || !plan(v + 1, w)) return false;
+      return issue_sdp(v + 1, w);
+    };
 
-    int next = 0;
-    if (ok) ok = advance_sdp(next, -1, nsub, plan, issue_sdp);
+    if (ok && nsub > 0) {
+      uint32_t w;
+      ok = plan(0, w) && issue_sdp(0, w);
+    }
     for (int u = 0; ok && u < nsub; ++u) {
+      // S(u + 1) overlaps the row warps' work on u, unless it has boundary
+      // classes: then its handshakes follow dK(u) and the row warps' masking for u
+      bool early = false;
+      if (u + 1 < nsub) {
+        uint32_t w1;
+        if (!plan(u + 1, w1)) {
+          ok = false;
+          break;
+        }
+        if (pw_bnd(w1) == 0u) {
+          early = true;
+          if (!(ok = next_sdp(u))) break;
+        }
+      }
       if (!warp_wait(&ds_ready[u & 1], (u >> 1) & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
       tc_fence_after();
       ok = issue_dkdv(u);
-      if (ok) ok = advance_sdp(next, u, nsub, plan, issue_sdp);
+      if (ok && u + 1 < nsub && !early) ok = next_sdp(u);
     }
     if (leader) {
       umma_commit(kv_final);
@@ -920,6 +983,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int64_t j = static_cast<int64_t>(kb) * TBQ + r;  // this thread's key
     const bool row_ok = j < N;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
+    const uint32_t s_addr = lane_addr + KV_S + cb, dp_addr = lane_addr + KV_DP + cb;
     const uint64_t c2x2 = pack_f2(a.scale_log2, a.scale_log2);
     constexpr int DPW = D / CSPLIT;  // accumulator columns of this warp in the epilogue
     tmem_zero16(lane_addr + KV_DK + cq * DPW, DPW / 16);
@@ -927,9 +991,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int bnd_cnt = 0, dsm_cnt = 0;
     bool ok = true;
     for (int u = 0; ok && u < nsub; ++u) {
-      const int st = u % TNST, bf = u & 1;
+      const int st = u % TNST;
       const int64_t q0 = q0_of(u) + cb;  // query of my first column
-      const uint32_t s_addr = lane_addr + KV_S + 64 * bf + cb, dp_addr = lane_addr + KV_DP + 64 * bf + cb;
+      const uint32_t pt_addr = lane_addr + KV_OB + 64 * (u & 1) + (COLS / 2) * cq, dst_addr = pt_addr + 32;
       if (!warp_wait(&qd_full[st], (u / TNST) & 1, lim, abort_flag)) {
         ok = false;
         break;
@@ -962,7 +1026,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
       }
-      if (!warp_wait(&s_ready[bf], (u >> 1) & 1, lim, abort_flag)) {
+      if (!warp_wait(s_ready, u & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
@@ -975,6 +1039,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < COLS; ++c) su[c] = 0u;
       }
+      // S^T and dP^T are in registers: the buffer is free for S^T(u + 1)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
       // P^T = exp2(S^T c2 - LSE_i log2 e) on the causal pairs i >= j of valid
       // queries, dS^T = P^T (dP^T - D_i)
       const float4 *ld4 = reinterpret_cast<const float4 *>(smem + L::LD_OFF + st * 512) + cq * (COLS / 4);
@@ -988,7 +1056,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int c = 4 * c4 + 2 * e;
-          const float la = e == 0 ? l4.x : l4.z, lb = e == 0 ? l4.y : l4.w;
+          const float la = (e == 0 ? l4.x : l4.z) * TLOG2E, lb = (e == 0 ? l4.y : l4.w) * TLOG2E;
           const float da = e == 0 ? d4.x : d4.z, db = e == 0 ? d4.y : d4.w;
           const uint64_t x2 = ffma2(pack_f2(__uint_as_float(su[c]), __uint_as_float(su[c + 1])), c2x2,
                                     pack_f2(-la, -lb));
@@ -1004,12 +1072,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ds[c + 1] = d1;
         }
       }
-      store_bf16_cols(s_addr, pf, lo, hi);
-      store_bf16_cols(dp_addr, ds, lo, hi);
+      // operand buffer u & 1 is free once the products of u - 2 have read it
+      if (u >= 2 && !warp_wait(&ob_free[u & 1], ((u >> 1) - 1) & 1, lim, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      store_bf16_cols(pt_addr, pf, lo, hi);
+      store_bf16_cols(dst_addr, ds, lo, hi);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_ready[bf]);
+      if (lane == 0) mbar_arrive(&ds_ready[u & 1]);
       int64_t prev = INT64_MAX;
       int32_t W;
       uint32_t cls;
@@ -1019,7 +1093,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_fence_after();
         const int64_t cm = j - q0 + W;
         const int cmax = cm < -1 ? -1 : (cm > COLS - 1 ? COLS - 1 : static_cast<int>(cm));
-        store_bf16_cols(dp_addr, ds, lo, hi < cmax ? hi : cmax);
+        store_bf16_cols(dst_addr, ds, lo, hi < cmax ? hi : cmax);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
