@@ -573,7 +573,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
       }
-      if (!warp_wait(s_ready, u & 1, lim, abort_flag)) {
+      // a sleeping poll: a spinning row warp would take issue slots from the
+      // MMA warp that shares its scheduler, which is what S(u) waits for
+      if (!warp_wait_idle<32>(s_ready, u & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
@@ -1026,7 +1028,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
       }
-      if (!warp_wait(s_ready, u & 1, lim, abort_flag)) {
+      // a sleeping poll: a spinning row warp would take issue slots from the
+      // MMA warp that shares its scheduler, which is what S(u) waits for
+      if (!warp_wait_idle<32>(s_ready, u & 1, lim, abort_flag)) {
         ok = false;
         break;
       }
