@@ -607,6 +607,25 @@ def run_ours(args, rank, world, local):
                        "frac": round(rows_gbs / peaks["hbm_gbs"], 4), "kernel_ms": round(rows_ms, 5),
                        "required_bytes": dec_bytes}
 
+    # wp_decode on a windowed K cache: every group keeps only the keys its
+    # cutoff can still reach (the rest evicted)
+    decode_windowed = None
+    if args.only == "all" and not args.page_size:
+        kwin = wp.wp_kcache_windowed(path.kc_rows, path.lens, path.dwg)
+        win_ms = statistics.median(
+            time_kernel(lambda: wp.wp_decode(path.dqr.reshape(dw.B, dw.Hq, dw.d), kwin, path.vc, path.lens,
+                                             path.dwg, out=path.do, lse=path.dlse, workspace=path.ws), 10, 3)
+            for _ in range(3))
+        win_ms = max_over_ranks([win_ms], dev)[0]
+        win_gbs = dec_bytes / (win_ms * 1e-3) / 1e9
+        decode_windowed = {"kernel": "wp_decode, windowed K cache (per-group rings of round_up_16(W_g + 1) keys)",
+                           "bound": "hbm", "value": round(win_gbs, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                           "frac": round(win_gbs / peaks["hbm_gbs"], 4), "kernel_ms": round(win_ms, 5),
+                           "required_bytes": dec_bytes, "k_cache_bytes": kwin.numel() * 2,
+                           "k_cache_bytes_full": path.kc_rows.numel() * 2,
+                           "k_cache_kept": round(kwin.numel() / path.kc_rows.numel(), 4)}
+        del kwin
+
     # backward of the 32K prefill (wp_prefill_backward), wave and dense
     backward = None
     if args.only in ("all", "backward") and not args.no_backward:
@@ -714,6 +733,7 @@ def run_ours(args, rank, world, local):
             "required_bytes": dec_bytes,
         },
         "decode_rows": decode_rows,
+        "decode_windowed": decode_windowed,
         "rope": ({"kernel": "wp_rope_apply of Q and K (2 launches)", "bound": "hbm",
                   "value": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
                   "frac": round(rope_bytes / (rope_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),

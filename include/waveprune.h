@@ -275,7 +275,51 @@ int wp_decode(const void *q, const void *kcache, const void *vcache, const int32
  *                           The pages fix no layout; this one is a choice of
  *                           this library.
  */
-enum wp_kcache_layout { WP_KCACHE_ROWS = 0, WP_KCACHE_GROUP_MAJOR = 1 };
+enum wp_kcache_layout { WP_KCACHE_ROWS = 0, WP_KCACHE_GROUP_MAJOR = 1, WP_KCACHE_WINDOWED = 2 };
+
+/*
+ * WP_KCACHE_WINDOWED — the K cache with every group's out-of-window keys
+ * evicted (SURVEY's per-channel KV eviction, at the granularity the kernels
+ * read: a 16-dim group). [RN §2.3, last paragraph] leaves freeing cache
+ * capacity as future work; a decode at position len - 1 reads group g only
+ * for keys j >= len - 1 - W_g, and len only grows, so a key older than W_g
+ * positions is never read for that group again. Layout, per (b, hk): the
+ * groups' rings back to back; group g keeps cap_g = min(round_up_16(W_g + 1),
+ * round_up_16(Lmax)) records of 16 bf16, key j in slot j mod cap_g. Its size
+ * per (b, hk) is wp_kcache_windowed_elems(Lmax, d_h, group_cut) elements;
+ * the 32K decode workload's half-split table keeps 54 % of the K cache.
+ * Decode it with wp_decode_kl(k_layout = WP_KCACHE_WINDOWED) and the SAME
+ * group_cut it was built with (the table fixes the geometry; a different
+ * table reads the wrong slots). Grouped mode, shared table, contiguous
+ * cache only.
+ */
+
+/* Elements (bf16) of one (b, hk) of a windowed K cache; 0 on bad arguments. */
+size_t wp_kcache_windowed_elems(int Lmax, int d_h, const int32_t *group_cut);
+
+/*
+ * wp_kcache_windowed_from_rows — build a windowed K cache from rows.
+ *   k_rows    device bf16 [B, H_kv, Lmax, d_h] (read only), 16-byte aligned.
+ *   lens      device int32 [B]: keys 0 .. lens[b]-1 are the sequence's.
+ *   k_win     device bf16 out, B * H_kv * wp_kcache_windowed_elems(...)
+ *             elements, 16-byte aligned, not overlapping k_rows; slot s of
+ *             group g receives the latest key j < lens[b] with j mod cap_g = s
+ *             (zeros where there is none).
+ *   group_cut the group cutoffs [d_h/16] (required).
+ * Asynchronous on `stream`. Errors: WP_ERR_ARG, WP_ERR_UNSUPPORTED (d_h),
+ * WP_ERR_CUDA.
+ */
+int wp_kcache_windowed_from_rows(const void *k_rows, const int32_t *lens, void *k_win, int B, int H_kv, int Lmax,
+                                 int d_h, const int32_t *group_cut, void *stream);
+
+/*
+ * wp_kcache_windowed_append — write one new key per sequence into a windowed
+ * K cache: k_new device bf16 [B, H_kv, d_h] (the token at position pos[b],
+ * device int32 [B]) into slot pos[b] mod cap_g of every group. A position
+ * outside [0, Lmax) writes nothing. Errors as wp_kcache_windowed_from_rows.
+ */
+int wp_kcache_windowed_append(const void *k_new, const int32_t *pos, void *k_win, int B, int H_kv, int Lmax, int d_h,
+                              const int32_t *group_cut, void *stream);
 
 /*
  * wp_kcache_group_major — copy a K cache from WP_KCACHE_ROWS to
@@ -293,7 +337,9 @@ int wp_kcache_group_major(const void *k_rows, void *k_gm, int B, int H_kv, int L
  * wp_decode_kl — wp_decode with the K cache in layout `k_layout`
  * (wp_kcache_layout); V stays [B, H_kv, Lmax, d_h]. All other arguments,
  * results and errors are those of wp_decode; a k_layout outside the enum is
- * WP_ERR_ARG. Both layouts give bit-identical results.
+ * WP_ERR_ARG. All layouts give bit-identical results. WP_KCACHE_WINDOWED
+ * needs group_cut (WP_ERR_ARG without) and is WP_ERR_UNSUPPORTED in
+ * wp_decode_ex's masked modes and in wp_decode_paged.
  */
 int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
                  int B, int H_q, int H_kv, int d_h, const int32_t *group_cut, float softmax_scale, void *o, float *lse,

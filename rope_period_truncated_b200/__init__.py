@@ -26,6 +26,7 @@ __all__ = [
     "wp_cutoffs", "wp_schedule", "wp_rope_apply", "wp_prefill", "wp_prefill_backward", "wp_decode",
     "wp_decode_workspace_bytes",
     "wp_decode_static", "DECODE_STATIC_SCRATCH_BYTES", "wp_kcache_group_major", "KCACHE_ROWS", "KCACHE_GROUP_MAJOR",
+    "KCACHE_WINDOWED", "wp_kcache_windowed_elems", "wp_kcache_windowed", "wp_kcache_windowed_append",
     "wp_decode_paged",
     "wp_device_status", "wp_set_wait_limit", "wp_wait_probe", "wp_status_str",
 ]
@@ -39,7 +40,7 @@ CUTOFF_INF = 2 ** 31 - 1
 DECODE_STATIC_SCRATCH_BYTES = 16 << 20
 
 WP_OK, WP_ERR_ARG, WP_ERR_UNSUPPORTED, WP_ERR_CUDA, WP_ERR_TIMEOUT = range(5)
-KCACHE_ROWS, KCACHE_GROUP_MAJOR = 0, 1  # wp_kcache_layout
+KCACHE_ROWS, KCACHE_GROUP_MAJOR, KCACHE_WINDOWED = 0, 1, 2  # wp_kcache_layout
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libwaveprune.so")
@@ -94,6 +95,12 @@ def load_library():
     lib.wp_decode_paged.argtypes = [P, P, I, P, I, I, P, I, P, I, I, I, I, P, F, P, P, P, ctypes.c_size_t, P]
     lib.wp_kcache_group_major.restype = I
     lib.wp_kcache_group_major.argtypes = [P, P, I, I, I, I, P]
+    lib.wp_kcache_windowed_elems.restype = ctypes.c_size_t
+    lib.wp_kcache_windowed_elems.argtypes = [I, I, P]
+    lib.wp_kcache_windowed_from_rows.restype = I
+    lib.wp_kcache_windowed_from_rows.argtypes = [P, P, P, I, I, I, I, P, P]
+    lib.wp_kcache_windowed_append.restype = I
+    lib.wp_kcache_windowed_append.argtypes = [P, P, P, I, I, I, I, P, P]
     lib.wp_device_status.restype = I
     lib.wp_device_status.argtypes = [P]
     lib.wp_set_wait_limit.restype = ctypes.c_longlong
@@ -319,13 +326,59 @@ def wp_kcache_group_major(kcache: torch.Tensor, out: torch.Tensor | None = None,
     return out
 
 
+def wp_kcache_windowed_elems(Lmax: int, d: int, group_cut) -> int:
+    """bf16 elements of one (b, hk) of a windowed K cache under ``group_cut`` [d/16]."""
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    n = load_library().wp_kcache_windowed_elems(int(Lmax), int(d), cut_p)
+    if n == 0:
+        raise WavePruneError(WP_ERR_ARG, "wp_kcache_windowed_elems")
+    return int(n)
+
+
+def wp_kcache_windowed(kcache: torch.Tensor, lens: torch.Tensor, group_cut, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """K cache [B,Hkv,Lmax,d] bf16 (rows) -> windowed [B,Hkv,elems]: every
+    group keeps only the keys its cutoff can still reach (rings of
+    round_up_16(W_g + 1) keys). ``lens`` int32 [B] (device)."""
+    _need(kcache, "kcache", torch.bfloat16, 4)
+    _need(lens, "lens", torch.int32, 1)
+    B, Hkv, Lmax, d = kcache.shape
+    n = wp_kcache_windowed_elems(Lmax, d, group_cut)
+    if out is None:
+        out = torch.empty((B, Hkv, n), dtype=torch.bfloat16, device=kcache.device)
+    _need(out, "out", torch.bfloat16, 3)
+    if tuple(out.shape) != (B, Hkv, n):
+        raise ValueError("out shape mismatch")
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    _check("wp_kcache_windowed", load_library().wp_kcache_windowed_from_rows(
+        _ptr(kcache), _ptr(lens), _ptr(out), B, Hkv, Lmax, d, cut_p, _stream(stream)))
+    return out
+
+
+def wp_kcache_windowed_append(k_new: torch.Tensor, pos: torch.Tensor, kwin: torch.Tensor, Lmax: int, group_cut,
+                              stream=None) -> torch.Tensor:
+    """Write the keys k_new [B,Hkv,d] (token positions ``pos`` int32 [B],
+    device) into a windowed K cache [B,Hkv,elems] in place; returns it."""
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(pos, "pos", torch.int32, 1)
+    _need(kwin, "kwin", torch.bfloat16, 3)
+    B, Hkv, d = k_new.shape
+    if tuple(kwin.shape) != (B, Hkv, wp_kcache_windowed_elems(Lmax, d, group_cut)):
+        raise ValueError("windowed K cache shape mismatch")
+    cut_a, cut_p = _host_i32(group_cut, d // 16)
+    _check("wp_kcache_windowed_append", load_library().wp_kcache_windowed_append(
+        _ptr(k_new), _ptr(pos), _ptr(kwin), B, Hkv, int(Lmax), d, cut_p, _stream(stream)))
+    return kwin
+
+
 def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens: torch.Tensor, group_cut=None,
               softmax_scale: float = 0.0, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
               workspace: torch.Tensor | None = None, want_lse: bool = True, stream=None, mode: int = MODE_GROUPED,
               layout: int = ROPE_INTERLEAVED):
     """Split-KV decode. q [B,Hq,d] (rotated), V cache [B,Hkv,Lmax,d] bf16, K
-    cache the same (rows) or [B,Hkv,d/16,Lmax,16] (group-major, from
-    wp_kcache_group_major), lens int32 [B] (device). ``group_cut``: group
+    cache the same (rows), [B,Hkv,d/16,Lmax,16] (group-major, from
+    wp_kcache_group_major) or [B,Hkv,elems] (windowed, from
+    wp_kcache_windowed with the same ``group_cut``), lens int32 [B] (device). ``group_cut``: group
     cutoffs [d/16], per-head [Hq, d/16], or (mode=MODE_CHANNEL) channel
     cutoffs [d/2] with ``layout``; None = dense. Returns (o [B,Hq,d] bf16,
     lse [B,Hq] fp32)."""
@@ -341,6 +394,13 @@ def wp_decode(q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor, lens:
         if tuple(kcache.shape) != (B, Hkv, d // 16, Lmax, 16):
             raise ValueError("group-major K cache shape mismatch")
         k_layout = KCACHE_GROUP_MAJOR
+    elif kcache.dim() == 3:
+        _need(kcache, "kcache", torch.bfloat16, 3)
+        if group_cut is None or np.asarray(group_cut).ndim != 1 or mode != MODE_GROUPED:
+            raise ValueError("a windowed K cache takes its own group cutoff table")
+        if tuple(kcache.shape) != (B, Hkv, wp_kcache_windowed_elems(Lmax, d, group_cut)):
+            raise ValueError("windowed K cache shape mismatch")
+        k_layout = KCACHE_WINDOWED
     else:
         _need(kcache, "kcache", torch.bfloat16, 4)
         if tuple(kcache.shape) != tuple(vcache.shape):

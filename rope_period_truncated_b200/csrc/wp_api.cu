@@ -356,7 +356,12 @@ static int decode_launch(const void *q, const void *kcache, int k_layout, const 
   if (q == nullptr || kcache == nullptr || vcache == nullptr || lens == nullptr || o == nullptr ||
       workspace == nullptr)
     return WP_ERR_ARG;
-  if (k_layout != WP_KCACHE_ROWS && k_layout != WP_KCACHE_GROUP_MAJOR) return WP_ERR_ARG;
+  if (k_layout != WP_KCACHE_ROWS && k_layout != WP_KCACHE_GROUP_MAJOR && k_layout != WP_KCACHE_WINDOWED)
+    return WP_ERR_ARG;
+  // the windowed rings follow the group cutoffs of a plain grouped decode
+  if (k_layout == WP_KCACHE_WINDOWED &&
+      (group_cut == nullptr || block_table != nullptr || mask != DECODE_MASK_GROUP_SHARED))
+    return group_cut == nullptr ? WP_ERR_ARG : WP_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || (reinterpret_cast<uintptr_t>(lens) & 3u) != 0 ||
       (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0))
@@ -386,7 +391,8 @@ static int decode_launch(const void *q, const void *kcache, int k_layout, const 
   a.Lmax = Lmax;
   a.nsplit = nsplit;
   a.chunk = DECODE_CHUNK;
-  a.k_group_major = k_layout == WP_KCACHE_GROUP_MAJOR ? 1 : 0;
+  a.k_group_major = k_layout != WP_KCACHE_ROWS ? 1 : 0;
+  a.k_windowed = k_layout == WP_KCACHE_WINDOWED ? 1 : 0;
   a.block_table = block_table;
   a.max_pages = max_pages;
   a.page_size = page_size;
@@ -395,6 +401,12 @@ static int decode_launch(const void *q, const void *kcache, int k_layout, const 
     a.cut[g] = (group_cut == nullptr || g >= d_h / 16) ? WP_CUTOFF_INF : group_cut[g];
     if (a.cut[g] < 0) return WP_ERR_ARG;
   }
+  a.wstride = a.k_windowed ? kcache_window_layout(a.cut, d_h / 16, Lmax, a.wcap, a.wbase) : 0;
+  if (!a.k_windowed)
+    for (int g = 0; g < 8; ++g) {
+      a.wcap[g] = 0;
+      a.wbase[g] = 0;
+    }
   a.scale_log2 = static_cast<float>(static_cast<double>(scale) * kLog2e);
   a.mask = mask;
   a.layout = layout;
@@ -469,6 +481,52 @@ int wp_decode(const void *q, const void *kcache, const void *vcache, const int32
               void *workspace, size_t ws_bytes, void *stream) {
   return wp_decode_kl(q, kcache, WP_KCACHE_ROWS, vcache, lens, Lmax, B, H_q, H_kv, d_h, group_cut, softmax_scale, o,
                       lse, workspace, ws_bytes, stream);
+}
+
+// Checks shared by the windowed-cache calls; fills the ring geometry.
+static int window_args(int B, int H_kv, int Lmax, int d_h, const int32_t *group_cut, int32_t *wcap, int64_t *wbase,
+                       int64_t *wstride) {
+  if (B <= 0 || H_kv <= 0 || Lmax <= 0 || group_cut == nullptr) return WP_ERR_ARG;
+  if (!head_dim_supported(d_h)) return d_h > 0 && d_h % 16 == 0 ? WP_ERR_UNSUPPORTED : WP_ERR_ARG;
+  int32_t cut[8];
+  for (int g = 0; g < 8; ++g) {
+    cut[g] = g < d_h / 16 ? group_cut[g] : 0;
+    if (cut[g] < 0) return WP_ERR_ARG;
+  }
+  *wstride = kcache_window_layout(cut, d_h / 16, Lmax, wcap, wbase);
+  return WP_OK;
+}
+size_t wp_kcache_windowed_elems(int Lmax, int d_h, const int32_t *group_cut) {
+  int32_t wcap[8];
+  int64_t wbase[8], wstride = 0;
+  if (window_args(1, 1, Lmax, d_h, group_cut, wcap, wbase, &wstride) != WP_OK) return 0;
+  return static_cast<size_t>(wstride);
+}
+int wp_kcache_windowed_from_rows(const void *k_rows, const int32_t *lens, void *k_win, int B, int H_kv, int Lmax,
+                                 int d_h, const int32_t *group_cut, void *stream) {
+  if (k_rows == nullptr || lens == nullptr || k_win == nullptr || !aligned16(k_rows) || !aligned16(k_win) ||
+      (reinterpret_cast<uintptr_t>(lens) & 3u) != 0 || k_rows == k_win)
+    return WP_ERR_ARG;
+  int32_t wcap[8];
+  int64_t wbase[8], wstride = 0;
+  const int rc = window_args(B, H_kv, Lmax, d_h, group_cut, wcap, wbase, &wstride);
+  if (rc != WP_OK) return rc;
+  return from_cuda(launch_kcache_window_from_rows(static_cast<const __nv_bfloat16 *>(k_rows), lens,
+                                                  static_cast<__nv_bfloat16 *>(k_win), B, H_kv, Lmax, d_h, wcap,
+                                                  wbase, wstride, static_cast<cudaStream_t>(stream)));
+}
+int wp_kcache_windowed_append(const void *k_new, const int32_t *pos, void *k_win, int B, int H_kv, int Lmax, int d_h,
+                              const int32_t *group_cut, void *stream) {
+  if (k_new == nullptr || pos == nullptr || k_win == nullptr || !aligned16(k_new) || !aligned16(k_win) ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u) != 0)
+    return WP_ERR_ARG;
+  int32_t wcap[8];
+  int64_t wbase[8], wstride = 0;
+  const int rc = window_args(B, H_kv, Lmax, d_h, group_cut, wcap, wbase, &wstride);
+  if (rc != WP_OK) return rc;
+  return from_cuda(launch_kcache_window_append(static_cast<const __nv_bfloat16 *>(k_new), pos,
+                                               static_cast<__nv_bfloat16 *>(k_win), B, H_kv, Lmax, d_h, wcap, wbase,
+                                               wstride, static_cast<cudaStream_t>(stream)));
 }
 
 int wp_kcache_group_major(const void *k_rows, void *k_gm, int B, int H_kv, int Lmax, int d_h, void *stream) {

@@ -184,6 +184,10 @@ __global__ void __launch_bounds__(DEC_THREADS)
       kblk = a.kc + pbase + (KGM ? static_cast<int64_t>(off) * 16 : static_cast<int64_t>(off) * D);
       vblk = a.vc + pbase + static_cast<int64_t>(off) * D;
       kgs = static_cast<int64_t>(a.page_size) * 16;
+    } else if (KGM && a.k_windowed) {
+      kblk = a.kc + (static_cast<int64_t>(b) * a.Hkv + hk) * a.wstride;  // the (b, hk) rings; per group below
+      vblk = vbase + static_cast<int64_t>(kb0) * D;
+      kgs = 0;
     } else {
       kblk = kbase + (KGM ? static_cast<int64_t>(kb0) * 16 : static_cast<int64_t>(kb0) * D);
       vblk = vbase + static_cast<int64_t>(kb0) * D;
@@ -191,8 +195,20 @@ __global__ void __launch_bounds__(DEC_THREADS)
     }
   };
   const uint32_t ring = smem_u32(dsmem) + warp * L::WARP_BYTES;
+  // This warp's blocks: start + 16*(warp + 4n).
+  const int first = start + KEYS * warp;
+  const int stride = KEYS * DEC_WARPS;
+  // Windowed rings: the slot of the next block to load in each group's ring,
+  // advanced by stride mod capacity per block (the blocks load in order).
+  int wslot[8], wstep[8];
+#pragma unroll
+  for (int gi = 0; gi < 8; ++gi) {
+    const int cap = (KGM && !PAGED && a.k_windowed && gi < D / 16) ? a.wcap[gi] : 16;
+    wslot[gi] = first % cap;
+    wstep[gi] = stride % cap;
+  }
 
-  // Issue the loads of one 16-key block into stage `st`.
+  // Issue the loads of one 16-key block into stage `st` (blocks in order).
   auto load_block = [&](int kb0, int st) {
     const uint32_t kdst = ring + st * L::STAGE, vdst = kdst + L::TILE;
     const __nv_bfloat16 *kblk, *vblk;
@@ -224,7 +240,19 @@ __global__ void __launch_bounds__(DEC_THREADS)
         const bool valid = key < end;
         const int64_t rr = valid ? r : 0;
         const bool kin = valid && qpos - key <= static_cast<int64_t>(a.cut[gi]);
-        cp_async16(kdst + piece_off<D>(r, 2 * gi + half), kblk + gi * kgs + rr * 16 + 8 * half, kin ? 16u : 0u);
+        // windowed rings: kb0 is a multiple of 16 and so is every capacity,
+        // so the block's 16 slots are contiguous in the ring
+        const __nv_bfloat16 *src = (!PAGED && a.k_windowed)
+                                       ? kblk + a.wbase[gi] + (static_cast<int64_t>(wslot[gi]) + rr) * 16
+                                       : kblk + gi * kgs + rr * 16;
+        cp_async16(kdst + piece_off<D>(r, 2 * gi + half), src + 8 * half, kin ? 16u : 0u);
+      }
+      if (!PAGED && a.k_windowed) {
+#pragma unroll
+        for (int gi = 0; gi < D / 16; ++gi) {
+          wslot[gi] += wstep[gi];
+          if (wslot[gi] >= a.wcap[gi]) wslot[gi] -= a.wcap[gi];
+        }
       }
     }
   };
@@ -234,9 +262,6 @@ __global__ void __launch_bounds__(DEC_THREADS)
 #pragma unroll
   for (int j = 0; j < NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
 
-  // This warp's blocks: start + 16*(warp + 4n).
-  const int first = start + KEYS * warp;
-  const int stride = KEYS * DEC_WARPS;
   const int nblk = first < end ? (end - first + stride - 1) / stride : 0;
 #pragma unroll
   for (int s = 0; s < STAGES - 1; ++s) {
@@ -447,6 +472,56 @@ cudaError_t launch_split_r(const DecodeArgs &a, const DecodeTables *tables, int 
 
 }  // namespace
 
+// The windowed cache's ring geometry, by value into the kernels below.
+struct WindowGeom {
+  int32_t wcap[8];
+  int64_t wbase[8];
+  int64_t wstride;
+};
+
+// One thread per (b, hk, group, slot) 16-byte half: the latest key j < len
+// with j % cap == slot, or zeros.
+__global__ void kcache_window_from_rows_kernel(const uint4 *__restrict__ src, const int32_t *__restrict__ lens,
+                                               uint4 *__restrict__ dst, int B, int Hkv, int Lmax, int D,
+                                               const __grid_constant__ WindowGeom geo) {
+  const int G = D / 16;
+  const int64_t per_bh = geo.wstride / 8;  // uint4 per (b, hk)
+  const int64_t total = static_cast<int64_t>(B) * Hkv * per_bh;
+  for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < total;
+       x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t bh = x / per_bh, e = (x % per_bh) * 8;  // element offset within (b, hk)
+    int g = G - 1;
+    while (g > 0 && e < geo.wbase[g]) --g;
+    const int64_t cap = geo.wcap[g];
+    const int64_t within = e - geo.wbase[g];
+    const int64_t slot = within / 16, half = (within % 16) / 8;
+    const int len = lens[bh / Hkv];
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (len >= 1 && len <= Lmax && slot <= len - 1) {
+      const int64_t j = slot + cap * ((len - 1 - slot) / cap);
+      v = src[((bh * Lmax + j) * D + 16 * g) / 8 + half];
+    }
+    dst[x] = v;
+  }
+}
+
+// One thread per (b, hk, group, half): the new key of sequence b into slot pos % cap.
+__global__ void kcache_window_append_kernel(const uint4 *__restrict__ k_new, const int32_t *__restrict__ pos,
+                                            uint4 *__restrict__ dst, int B, int Hkv, int Lmax, int D,
+                                            const __grid_constant__ WindowGeom geo) {
+  const int G = D / 16;
+  const int64_t total = static_cast<int64_t>(B) * Hkv * G * 2;
+  for (int64_t x = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; x < total;
+       x += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t bh = x / (G * 2);
+    const int g = static_cast<int>((x / 2) % G), half = static_cast<int>(x % 2);
+    const int p = pos[bh / Hkv];
+    if (p < 0 || p >= Lmax) continue;  // outside the cache: nothing written
+    const int64_t slot = p % geo.wcap[g];
+    dst[(bh * geo.wstride + geo.wbase[g] + slot * 16) / 8 + half] = k_new[(bh * D + 16 * g) / 8 + half];
+  }
+}
+
 cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int64_t BH, int Lmax, int D,
                                       cudaStream_t stream) {
   int dev = 0, nsm = 148;
@@ -457,6 +532,38 @@ cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *d
     kcache_group_major_kernel<128><<<nsm * 8, 256, 0, stream>>>(s, d, BH, Lmax);
   else
     kcache_group_major_kernel<64><<<nsm * 8, 256, 0, stream>>>(s, d, BH, Lmax);
+  return cudaGetLastError();
+}
+
+static WindowGeom window_geom(const int32_t *wcap, const int64_t *wbase, int64_t wstride) {
+  WindowGeom g;
+  for (int k = 0; k < 8; ++k) {
+    g.wcap[k] = wcap[k];
+    g.wbase[k] = wbase[k];
+  }
+  g.wstride = wstride;
+  return g;
+}
+
+cudaError_t launch_kcache_window_from_rows(const __nv_bfloat16 *src, const int32_t *lens, __nv_bfloat16 *dst, int B,
+                                           int Hkv, int Lmax, int D, const int32_t *wcap, const int64_t *wbase,
+                                           int64_t wstride, cudaStream_t stream) {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  kcache_window_from_rows_kernel<<<nsm * 8, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(src), lens,
+                                                              reinterpret_cast<uint4 *>(dst), B, Hkv, Lmax, D,
+                                                              window_geom(wcap, wbase, wstride));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kcache_window_append(const __nv_bfloat16 *k_new, const int32_t *pos, __nv_bfloat16 *dst, int B,
+                                        int Hkv, int Lmax, int D, const int32_t *wcap, const int64_t *wbase,
+                                        int64_t wstride, cudaStream_t stream) {
+  const int64_t total = static_cast<int64_t>(B) * Hkv * (D / 16) * 2;
+  const int grid = static_cast<int>((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
+  kcache_window_append_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4 *>(k_new), pos,
+                                                        reinterpret_cast<uint4 *>(dst), B, Hkv, Lmax, D,
+                                                        window_geom(wcap, wbase, wstride));
   return cudaGetLastError();
 }
 

@@ -20,7 +20,12 @@ struct DecodeArgs {
   float *o_part;                     // [B, Hq, nsplit, D]
   float *lse_part;                   // [B, Hq, nsplit], base-2
   int B, Hq, Hkv, Lmax, nsplit, chunk;
-  int k_group_major;                 // K cache layout: 0 rows, 1 group-major
+  int k_group_major;                 // K cache layout: 0 rows, 1 group-major (or windowed, below)
+  int k_windowed;                    // K cache as per-group rings: group g of (b, hk) at
+                                     // kc + (b * Hkv + hk) * wstride + wbase[g], key j in slot j % wcap[g]
+  int32_t wcap[8];                   // ring capacity of each group (multiple of 16)
+  int64_t wbase[8];                  // element offset of each group's ring
+  int64_t wstride;                   // elements per (b, hk)
   const int32_t *block_table;        // paged cache: [B, max_pages] page of each page_size-key block, or null
   int max_pages, page_size, n_pages;
   int32_t cut[8];                    // group cutoffs (of the K loads: the union over heads / channels)
@@ -53,6 +58,35 @@ inline size_t decode_workspace_bytes(int B, int Hq, int nsplit, int D) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, const DecodeTables *tables, int d_h, cudaStream_t stream);
+
+// Ring capacities of the windowed K cache: group g keeps the last
+// min(W_g + 1, Lmax) keys, rounded up to 16 (so a 16-key block aligned to 16
+// never wraps). Returns the elements per (b, hk).
+inline int64_t kcache_window_layout(const int32_t *cut, int G, int Lmax, int32_t *wcap, int64_t *wbase) {
+  const int64_t lm = (static_cast<int64_t>(Lmax) + 15) / 16 * 16;
+  int64_t off = 0;
+  for (int g = 0; g < 8; ++g) {
+    int64_t c = 0;
+    if (g < G) {
+      c = (static_cast<int64_t>(cut[g]) + 1 + 15) / 16 * 16;
+      if (c > lm) c = lm;
+    }
+    wcap[g] = static_cast<int32_t>(c);
+    wbase[g] = off;
+    off += c * 16;
+  }
+  return off;
+}
+
+// Windowed K cache from rows: slot s of group g holds the latest key j < len
+// with j % wcap[g] == s (zeros where there is none).
+cudaError_t launch_kcache_window_from_rows(const __nv_bfloat16 *src, const int32_t *lens, __nv_bfloat16 *dst, int B,
+                                           int Hkv, int Lmax, int D, const int32_t *wcap, const int64_t *wbase,
+                                           int64_t wstride, cudaStream_t stream);
+// Append one key per sequence (k_new [B, Hkv, D] at position pos[b]) into its rings.
+cudaError_t launch_kcache_window_append(const __nv_bfloat16 *k_new, const int32_t *pos, __nv_bfloat16 *dst, int B,
+                                        int Hkv, int Lmax, int D, const int32_t *wcap, const int64_t *wbase,
+                                        int64_t wstride, cudaStream_t stream);
 
 // K cache rows [BH, Lmax, D] -> group-major [BH, D/16, Lmax, 16] (BH = B * H_kv).
 cudaError_t launch_kcache_group_major(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int64_t BH, int Lmax, int D,

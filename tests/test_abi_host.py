@@ -234,3 +234,29 @@ def test_status_strings(lib):
     for code in range(5):
         assert wp.wp_status_str(code)
     assert "unknown" in wp.wp_status_str(99)
+
+
+def test_kcache_windowed_geometry_and_checks(lib):
+    """Ring capacities round_up_16(W_g + 1), capped at round_up_16(Lmax);
+    null or misaligned buffers and missing or negative tables are refused on
+    the host."""
+    def expect(Lmax, d, cut):
+        lm = (Lmax + 15) // 16 * 16
+        return 16 * sum(min((int(w) + 1 + 15) // 16 * 16, lm) for w in cut[: d // 16])
+    for Lmax, d, cut in [(3000, 128, [5, 40, 300, 1100, 2000, 10 ** 6, 7, 1024]), (32768, 128, [160, 5063, 160114,
+                         5063255] * 2), (1, 64, [0, 0, 0, 0]), (17, 64, [15, 16, 2 ** 31 - 1, 31])]:
+        assert wp.wp_kcache_windowed_elems(Lmax, d, cut) == expect(Lmax, d, cut)
+    P = ctypes.c_void_p
+    cut = (ctypes.c_int32 * 8)(*([100] * 8))
+    bad = (ctypes.c_int32 * 8)(*([100] * 7 + [-1]))
+    assert lib.wp_kcache_windowed_elems(0, 128, cut) == 0
+    assert lib.wp_kcache_windowed_elems(100, 128, None) == 0
+    assert lib.wp_kcache_windowed_elems(100, 128, bad) == 0
+    buf = ctypes.create_string_buffer(1 << 16)
+    base = (ctypes.addressof(buf) + 255) & ~255
+    assert lib.wp_kcache_windowed_from_rows(None, P(base), P(base + 4096), 1, 1, 16, 128, cut, None) == 1
+    assert lib.wp_kcache_windowed_from_rows(P(base), P(base), P(base + 1), 1, 1, 16, 128, cut, None) == 1
+    assert lib.wp_kcache_windowed_from_rows(P(base), P(base), P(base + 4096), 1, 1, 16, 128, None, None) == 1
+    assert lib.wp_kcache_windowed_append(P(base), P(base + 2), P(base + 4096), 1, 1, 16, 128, cut, None) == 1
+    assert lib.wp_kcache_windowed_append(P(base), P(base), P(base + 4096), 0, 1, 16, 128, cut, None) == 1
+    assert lib.wp_kcache_windowed_from_rows(P(base), P(base), P(base + 4096), 1, 1, 16, 96, cut, None) == 2

@@ -129,6 +129,38 @@ def test_decode_group_major_kcache(d):
     assert_attention_close(o_gm, lse_gm, ro, rl, f"decode group-major d={d}")
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_windowed_kcache(d):
+    """Evicting every group's out-of-window keys changes nothing: the windowed
+    K cache (per-group rings of round_up_16(W_g + 1) keys, wrapping many times
+    for the small cutoffs here) gives results bit-identical to the full cache
+    and matches the oracle; appending each sequence's last key to a cache
+    built for one key less gives the same cache, slot for slot."""
+    g = torch.Generator().manual_seed(41 + d)
+    B, Hq, Hkv, Lmax = 4, 8, 2, 3000
+    lens = torch.tensor([1, 2999, 1500, 1025], dtype=torch.int32)
+    q = torch.randn(B, Hq, d, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    wg = np.array([5, 40, 300, 1100, 2000, 10 ** 6, 7, 1024][: d // 16], dtype=np.int32)
+    o_rows, lse_rows = _gpu_decode(q, kc, vc, lens, wg)
+    kw = wp.wp_kcache_windowed(kc.cuda(), lens.cuda(), wg)
+    caps = [min((int(w) + 1 + 15) // 16 * 16, (Lmax + 15) // 16 * 16) for w in wg]
+    assert kw.shape == (B, Hkv, 16 * sum(caps)) and kw.shape[2] < Lmax * d
+    o_w, lse_w = wp.wp_decode(q.cuda(), kw, vc.cuda(), lens.cuda(), wg)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    assert torch.equal(o_w, o_rows) and torch.equal(lse_w, lse_rows)
+    ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o_w, lse_w, ro, rl, f"decode windowed d={d}")
+    # one decode step: the cache for len - 1 keys plus the key at len - 1
+    kw_prev = wp.wp_kcache_windowed(kc.cuda(), (lens - 1).cuda(), wg)
+    k_new = torch.stack([kc[b, :, int(lens[b]) - 1, :] for b in range(B)]).contiguous()
+    wp.wp_kcache_windowed_append(k_new.cuda(), (lens - 1).cuda(), kw_prev, Lmax, wg)
+    torch.cuda.synchronize()
+    assert torch.equal(kw_prev, kw)
+
+
 def test_decode_group_major_workload():
     """The 32K decode workload with a group-major K cache: every row checked
     against the oracle."""
