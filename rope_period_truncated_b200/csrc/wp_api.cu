@@ -222,12 +222,15 @@ int wp_prefill_ex(const void *q, const void *k, const void *v, void *o, float *l
     }
     a.scale_log2 = scale_log2;
     a.wait_limit = g_wait_limit;
-    // uniform batches run on the tensor cores, packed batches on the CUDA cores
-    if (cu_seqlens == nullptr && (N + 127) / 128 <= 65535 && static_cast<int64_t>(H_kv) * B <= 65535) {
+    // the tensor-core kernel (uniform and packed batches) within its grid limits,
+    // else the CUDA-core kernel
+    if ((N + 127) / 128 <= 65535 && static_cast<int64_t>(H_kv) * B <= 65535) {
+      const int mB = cu_seqlens != nullptr ? 1 : B;
+      const int mN = cu_seqlens != nullptr ? static_cast<int>(total_tokens) : N;
       CUtensorMap tq, tk, tv;
-      if (!make_map(&tq, q, B, N, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-          !make_map(&tk, k, B, N, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
-          !make_map(&tv, v, B, N, H_kv, d_h, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      if (!make_map(&tq, q, mB, mN, H_q, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+          !make_map(&tk, k, mB, mN, H_kv, d_h, 16, CU_TENSOR_MAP_SWIZZLE_32B) ||
+          !make_map(&tv, v, mB, mN, H_kv, d_h, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return WP_ERR_CUDA;
       return from_cuda(launch_prefill_exact(d_h, tq, tk, tv, a, s));
     }

@@ -51,7 +51,7 @@ cudaError_t launch_prefill_grouped(int d_h, const CUtensorMap &tq, const CUtenso
                                    const PrefillArgs &a, const HeadCuts *head_cuts, cudaStream_t stream);
 cudaError_t launch_prefill_channel(int d_h, const ChannelPrefillArgs &a, cudaStream_t stream);
 
-// Exact per-channel rule on the tensor cores (uniform batches).
+// Exact per-channel rule on the tensor cores (uniform and packed batches).
 constexpr uint32_t PREFILL_SMEM_CAP = 232448;  // dynamic shared memory of one CTA
 cudaError_t launch_prefill_exact(int d_h, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                                  const ChannelPrefillArgs &a, cudaStream_t stream);

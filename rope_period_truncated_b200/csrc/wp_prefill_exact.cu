@@ -221,7 +221,8 @@ struct XBarriers {
   uint64_t *q_full, *k_full, *k_empty, *k_plan, *v_full, *v_empty, *s_ready, *p_ready, *o_ready, *o_final, *drain;
 };
 
-template <int D>
+// PACKED: sequences located by cu_seqlens (else a uniform batch).
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(XTHREADS, 1)
     prefill_exact_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ ChannelPrefillArgs a) {
@@ -263,7 +264,23 @@ __global__ void __launch_bounds__(XTHREADS, 1)
   const int h0 = hk * rep + static_cast<int>(blockIdx.x) * nslot;  // head of slot s = h0 + s
   const int nqb = (a.N + XBM - 1) / XBM;
   const int qb = nqb - 1 - static_cast<int>(blockIdx.y);
-  const int64_t N = a.N;
+  // The sequence: batch entry b of a uniform batch (length a.N, coordinate b
+  // of the 4-D tensor view) or rows [row0, row0 + N) of a packed one.
+  int64_t N = a.N, row0 = 0;
+  if constexpr (PACKED) {
+    row0 = a.cu_seqlens[b];
+    const int64_t row1 = a.cu_seqlens[b + 1];
+    if (row0 < 0 || row1 < row0 || row1 > a.T || row1 - row0 > a.N) {
+      // Offsets out of range: nothing of this sequence can be located.
+      if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0 && hk == 0) record_status(WP_ERR_ARG);
+      return;
+    }
+    N = row1 - row0;
+    if (static_cast<int64_t>(qb) * XBM >= N) return;  // past this sequence's end (whole CTA)
+  }
+  // TMA row coordinate of query / key block x and the batch coordinate
+  const auto block_row = [&](int x) { return PACKED ? static_cast<int>(row0 + static_cast<int64_t>(x) * XBM) : x * XBM; };
+  const int bcoord = PACKED ? 0 : b;
   // one plan (cutoff row, masked copies) for both slots, or one per slot
   const int nplan = a.cut_rows == 1 ? 1 : nslot;
   const long long lim = a.wait_limit;
@@ -328,7 +345,7 @@ __global__ void __launch_bounds__(XTHREADS, 1)
       for (int s = 0; s < nslot; ++s)
         for (int g = 0; g < G; ++g)
           tma_load_4d(smem + L::Q_OFF + s * L::Q_SLOT + g * XGROUP_BYTES, &tm_q, B.q_full, 16 * g, h0 + s,
-                      qb * XBM, b);
+                      block_row(qb), bcoord);
     }
     __syncwarp();
     int k_issued = 0, v_issued = 0;
@@ -340,7 +357,7 @@ __global__ void __launch_bounds__(XTHREADS, 1)
         mbar_arrive_expect_tx(&B.v_full[st], (D / 64) * XV_CHUNK);
         for (int c = 0; c < D / 64; ++c)
           tma_load_4d(smem + L::V_OFF + st * L::V_STAGE + c * XV_CHUNK, &tm_v, &B.v_full[st], 64 * c, hk,
-                      (qb - t) * XBN, b);
+                      block_row(qb - t), bcoord);
       }
       __syncwarp();
       ++v_issued;
@@ -365,7 +382,7 @@ __global__ void __launch_bounds__(XTHREADS, 1)
         for (uint32_t m = need; m; m &= m - 1) {
           const int g = __ffs(m) - 1;
           tma_load_4d(smem + L::K_OFF + st * L::K_STAGE + g * XGROUP_BYTES, &tm_k, &B.k_full[st], 16 * g, hk,
-                      (qb - t) * XBN, b);
+                      block_row(qb - t), bcoord);
         }
       }
       __syncwarp();
@@ -653,7 +670,12 @@ __global__ void __launch_bounds__(XTHREADS, 1)
         m_run = m_new;
       }
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      exp_half<true>(su, c2x2, m_run, acc, s_addr);
+      // a packed batch's diagonal tile takes every exponential on MUFU, so its
+      // causally masked entries (possibly the next sequence's keys) give exactly 0
+      if (PACKED && t == 0)
+        exp_half<false>(su, c2x2, m_run, acc, s_addr);
+      else
+        exp_half<true>(su, c2x2, m_run, acc, s_addr);
       float s0, s1, s2, s3, s4, s5, s6, s7;
       unpack_f2(acc[0], s0, s1);
       unpack_f2(acc[1], s2, s3);
@@ -665,8 +687,10 @@ __global__ void __launch_bounds__(XTHREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&B.p_ready[2 * slot + hh]);
     }
-    __nv_bfloat16 *orow = a.o + ((static_cast<int64_t>(b) * a.N + i) * a.Hq + h) * D;
-    float *lse_at = a.lse == nullptr ? nullptr : a.lse + (static_cast<int64_t>(b) * a.Hq + h) * a.N + i;
+    __nv_bfloat16 *orow = a.o + (((PACKED ? row0 : static_cast<int64_t>(b) * a.N) + i) * a.Hq + h) * D;
+    float *lse_at = a.lse == nullptr ? nullptr
+                                     : a.lse + (PACKED ? static_cast<int64_t>(h) * a.T + row0 + i
+                                                       : (static_cast<int64_t>(b) * a.Hq + h) * a.N + i);
     if (ok && nsub > 0 && warp_wait(&B.o_final[slot], 0, lim, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.f / l_run;
@@ -714,11 +738,18 @@ cudaError_t launch_exact(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
   const int rep = a.Hq / a.Hkv;
   const int nslot = rep % 2 == 0 ? 2 : 1;
   const uint32_t smem = XLayout<D>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(prefill_exact_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
   const dim3 grid(rep / nslot, nqb, a.Hkv * a.B);
-  prefill_exact_kernel<D><<<grid, XTHREADS, smem, stream>>>(tq, tk, tv, a);
+  if (a.cu_seqlens != nullptr) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_exact_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    prefill_exact_kernel<D, true><<<grid, XTHREADS, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(prefill_exact_kernel<D, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    prefill_exact_kernel<D, false><<<grid, XTHREADS, smem, stream>>>(tq, tk, tv, a);
+  }
   return cudaGetLastError();
 }
 

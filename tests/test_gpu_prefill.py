@@ -272,7 +272,8 @@ def test_packed_batch_of_equal_lengths_is_the_uniform_batch():
     assert (l1.permute(1, 0, 2).reshape(Hq, B * N) - l2).abs().max().item() <= 1e-4
 
 
-def test_packed_batch_bad_offsets_are_reported():
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_packed_batch_bad_offsets_are_reported(mode):
     """Offsets that run backwards are not followed: the kernel records
     WP_ERR_ARG in the status word (read and cleared by wp_device_status),
     and a later correct call runs normally."""
@@ -280,9 +281,9 @@ def test_packed_batch_bad_offsets_are_reported():
     q = torch.randn(T, Hq, d, device="cuda").to(torch.bfloat16)
     k = torch.randn(T, Hkv, d, device="cuda").to(torch.bfloat16)
     cu_bad = torch.tensor([0, 300, 100, 400], dtype=torch.int32, device="cuda")
-    wp.wp_prefill(q, k, k, None, cu_seqlens=cu_bad, max_seqlen=300)
+    wp.wp_prefill(q, k, k, None, mode, cu_seqlens=cu_bad, max_seqlen=300)
     assert wp.wp_device_status() == wp.WP_ERR_ARG
     cu = torch.tensor([0, 100, 400], dtype=torch.int32, device="cuda")
-    o, lse = wp.wp_prefill(q, k, k, None, cu_seqlens=cu, max_seqlen=300)
+    o, lse = wp.wp_prefill(q, k, k, None, mode, cu_seqlens=cu, max_seqlen=300)
     assert wp.wp_device_status() == wp.WP_OK
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
