@@ -122,10 +122,38 @@ def bench_config(args, world, wg):
     }
 
 
+def source_digest(source: str) -> str:
+    """sha256 prefix (16 hex digits) of a kernel source followed by every
+    header it pulls in with #include "..." (looked up beside the including
+    file, then in include/), each once, in the order of first inclusion: a
+    kernel compiled from the same text hashes the same."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    seen = set()
+
+    def visit(path):
+        if path in seen:
+            return
+        seen.add(path)
+        with open(path, "rb") as f:
+            data = f.read()
+        h.update(data)
+        for name in re.findall(rb'^[ \t]*#[ \t]*include[ \t]+"([^"]+)"', data, re.M):
+            for d in (os.path.dirname(path), os.path.join(ROOT, "include")):
+                cand = os.path.join(d, name.decode())
+                if os.path.exists(cand):
+                    visit(cand)
+                    break
+
+    visit(os.path.join(ROOT, source))
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic(summary: str, source: str):
     """DRAM bytes per launch from a committed ncu summary under profiles/, or
-    None when the kernel source has changed since it was captured."""
-    import hashlib
+    None when the kernel source (with its headers) has changed since it was
+    captured."""
     try:
         kv = {}
         with open(os.path.join(ROOT, "profiles", summary)) as f:
@@ -133,9 +161,7 @@ def profiled_traffic(summary: str, source: str):
                 if ":" in line and not line.startswith("#"):
                     key, val = line.split(":", 1)
                     kv[key.strip()] = val.strip()
-        with open(os.path.join(ROOT, source), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()[:16]
-        if kv.get("source_sha256_16") != digest:
+        if kv.get("source_sha256_16") != source_digest(source):
             return None
         return int(kv["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):

@@ -155,14 +155,22 @@ __device__ __forceinline__ void poly_exp2x2(uint64_t x2, float &p0, float &p1) {
   p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// 64 columns of S (or zeros when no group of the tile was computed).
+// 64 columns of S, or zeros when no product of the sub-tile was computed.
+// Called after the S-ready barrier, when every MMA that used the half has
+// completed: a sub-tile without products first writes zeros into its half,
+// and every sub-tile then takes the same TMEM load. (Zeroing the registers
+// on that path instead gives the 64 registers two definitions, and the
+// merge costs register moves on every sub-tile.)
 __device__ __forceinline__ void load_half(uint32_t taddr, bool any_group, uint32_t (&su)[64]) {
-  if (any_group) {
-    tmem_ld64(taddr, su);
-  } else {
+  if (!any_group) {
+    uint32_t z[32];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) su[c] = 0u;
+    for (int c = 0; c < 32; ++c) z[c] = 0u;
+    tmem_st32(taddr, z);
+    tmem_st32(taddr + 32, z);
+    tmem_wait_st();
   }
+  tmem_ld64(taddr, su);
 }
 
 // Causal mask of the diagonal tile: key column c0 + c comes after row r.

@@ -110,3 +110,24 @@ def test_profiled_traffic_follows_the_source(tmp_path, monkeypatch):
     src.write_text("kernel v2\n")  # the kernel changed since the capture
     assert bench.profiled_traffic("k.txt", "kernel.cu") is None
     assert bench.profiled_traffic("missing.txt", "kernel.cu") is None
+
+
+def test_source_digest_covers_included_headers(tmp_path, monkeypatch):
+    """A change to a header the kernel includes (beside it or in include/)
+    changes the digest; an unrelated file does not."""
+    (tmp_path / "csrc").mkdir()
+    (tmp_path / "include").mkdir()
+    (tmp_path / "csrc" / "k.cu").write_text('#include "a.cuh"\n#include <cstdint>\nkernel\n')
+    (tmp_path / "csrc" / "a.cuh").write_text('#include "api.h"\n#include "a.cuh"\nhelpers v1\n')
+    (tmp_path / "include" / "api.h").write_text("api v1\n")
+    (tmp_path / "csrc" / "other.cuh").write_text("unrelated v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    d0 = bench.source_digest("csrc/k.cu")
+    assert len(d0) == 16
+    (tmp_path / "csrc" / "other.cuh").write_text("unrelated v2\n")
+    assert bench.source_digest("csrc/k.cu") == d0
+    (tmp_path / "csrc" / "a.cuh").write_text('#include "api.h"\n#include "a.cuh"\nhelpers v2\n')
+    d1 = bench.source_digest("csrc/k.cu")
+    assert d1 != d0
+    (tmp_path / "include" / "api.h").write_text("api v2\n")
+    assert bench.source_digest("csrc/k.cu") not in (d0, d1)
