@@ -580,14 +580,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
+      // No S product for this sub-tile: its S is 0. Store the zeros into this
+      // warp's S columns (no MMA reads them) so that every sub-tile takes the
+      // same loads; zeroing the registers on that path instead gives them two
+      // definitions, and the merge costs register moves on every sub-tile.
+      if (!(pw_full(w) | pw_bnd(w))) tmem_zero16(s_addr, COLS / 16);
       uint32_t su[COLS], dp[COLS];
-      if (pw_full(w) | pw_bnd(w)) {
-        ld_cols2(s_addr, su, dp_addr, dp);
-      } else {
-        ld_cols(dp_addr, dp);
-#pragma unroll
-        for (int c = 0; c < COLS; ++c) su[c] = 0u;
-      }
+      ld_cols2(s_addr, su, dp_addr, dp);
       // S and dP are in registers: the buffer is free for S(u + 1)
       tc_fence_before();
       __syncwarp();
@@ -1035,14 +1034,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         break;
       }
       tc_fence_after();
+      // No S product for this sub-tile: its S is 0. Store the zeros into this
+      // warp's S columns (no MMA reads them) so that every sub-tile takes the
+      // same loads; zeroing the registers on that path instead gives them two
+      // definitions, and the merge costs register moves on every sub-tile.
+      if (!(pw_full(w) | pw_bnd(w))) tmem_zero16(s_addr, COLS / 16);
       uint32_t su[COLS], dp[COLS];
-      if (pw_full(w) | pw_bnd(w)) {
-        ld_cols2(s_addr, su, dp_addr, dp);
-      } else {
-        ld_cols(dp_addr, dp);
-#pragma unroll
-        for (int c = 0; c < COLS; ++c) su[c] = 0u;
-      }
+      ld_cols2(s_addr, su, dp_addr, dp);
       // S^T and dP^T are in registers: the buffer is free for S^T(u + 1)
       tc_fence_before();
       __syncwarp();
