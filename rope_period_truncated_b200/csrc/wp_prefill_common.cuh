@@ -150,9 +150,10 @@ __device__ __forceinline__ void poly_exp2x2(uint64_t x2, float &p0, float &p1) {
   unpack_f2(t2, t0, t1);
   unpack_f2(q2, p0, p1);
   // 2^j * 2^f: add j to the exponent field. The bits of t are those of ROUND
-  // plus j, and ROUND's own bits vanish from a 23-bit left shift.
-  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  // plus j, and ROUND's own bits vanish from a 23-bit left shift (unsigned:
+  // the shift and the sum wrap modulo 2^32, which is the intent).
+  p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // 64 columns of S, or zeros when no product of the sub-tile was computed.
