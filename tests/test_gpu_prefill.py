@@ -104,6 +104,29 @@ def test_small_full_rows(N, d, Hq, Hkv, theta, layout, kind, mode):
     assert_attention_close(o, lse, ro, rl, f"N={N} d={d} {kind} mode={mode}")
 
 
+@pytest.mark.parametrize("mode", [wp.MODE_GROUPED, wp.MODE_CHANNEL])
+def test_large_logits(mode):
+    """Logits spanning hundreds of base-2 units (Q and K scaled by 8, keys
+    further from the diagonal scaled up to 3x more): most exponentials fall
+    below the polynomial exp2's clamp at 2^-120, and row maxima keep growing
+    past the 2^8 rescale threshold as the kernel walks the key tiles back from
+    the diagonal. 700 rows: several tiles and a ragged tail."""
+    N, d, Hq, Hkv, theta, layout = 700, 128, 4, 2, 1e4, wp.ROPE_HALF_SPLIT
+    g = torch.Generator().manual_seed(4242)
+    ramp = (1.0 + 2.0 * torch.arange(N - 1, -1, -1, dtype=torch.float32) / N).view(1, N, 1, 1)
+    q = (8.0 * torch.randn(1, N, Hq, d, generator=g)).to(torch.bfloat16)
+    k = (8.0 * ramp * torch.randn(1, N, Hkv, d, generator=g)).to(torch.bfloat16)
+    v = torch.randn(1, N, Hkv, d, generator=g).to(torch.bfloat16)
+    cut = _cut_table("wave", d, theta, layout, mode)
+    o, lse = _gpu_path(q, k, v, theta, layout, cut, mode, rope=False)
+    ro, rl = oracle.attention(widen(q), widen(k), widen(v), cut, mode, layout)
+    # the case is what it claims: the last row's unmasked logits span far more
+    # than 120 base-2 units
+    s2 = (widen(q)[0, N - 1, 0] @ widen(k)[0, :, 0].T) / np.sqrt(d) / np.log(2.0)
+    assert s2.max() - s2.min() > 240
+    assert_attention_close(o, lse, ro, rl, f"large logits mode={mode}")
+
+
 def _sampled_check(name, per_head, mode=wp.MODE_GROUPED):
     w = syn.workload(name)
     q, k, v = syn.prefill_inputs(w)
