@@ -123,14 +123,21 @@ def bench_config(args, world, wg):
 
 
 def source_digest(source: str) -> str:
-    """sha256 prefix (16 hex digits) of a kernel source followed by every
-    header it pulls in with #include "..." (looked up beside the including
-    file, then in include/), each once, in the order of first inclusion: a
-    kernel compiled from the same text hashes the same."""
+    """sha256 prefix (16 hex digits) of a kernel source's code followed by the
+    code of every header it pulls in with #include "..." (looked up beside
+    the including file, then in include/), each once, in the order of first
+    inclusion. Comments are removed and runs of whitespace collapsed first,
+    so a change to the compiled text changes the digest and a change to a
+    comment does not."""
     import hashlib
     import re
     h = hashlib.sha256()
     seen = set()
+
+    def code_of(data: bytes) -> bytes:
+        data = re.sub(rb"/\*.*?\*/", b" ", data, flags=re.S)
+        data = re.sub(rb"//[^\n]*", b" ", data)
+        return re.sub(rb"\s+", b" ", data).strip()
 
     def visit(path):
         if path in seen:
@@ -138,7 +145,7 @@ def source_digest(source: str) -> str:
         seen.add(path)
         with open(path, "rb") as f:
             data = f.read()
-        h.update(data)
+        h.update(code_of(data) + b"\n")
         for name in re.findall(rb'^[ \t]*#[ \t]*include[ \t]+"([^"]+)"', data, re.M):
             for d in (os.path.dirname(path), os.path.join(ROOT, "include")):
                 cand = os.path.join(d, name.decode())

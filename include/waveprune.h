@@ -279,8 +279,8 @@ enum wp_kcache_layout { WP_KCACHE_ROWS = 0, WP_KCACHE_GROUP_MAJOR = 1, WP_KCACHE
 
 /*
  * WP_KCACHE_WINDOWED — the K cache with every group's out-of-window keys
- * evicted (SURVEY's per-channel KV eviction, at the granularity the kernels
- * read: a 16-dim group). [RN §2.3, last paragraph] leaves freeing cache
+ * evicted (KV eviction at the granularity the kernels read: a 16-dim group,
+ * not a single channel). [RN §2.3, last paragraph] leaves freeing cache
  * capacity as future work; a decode at position len - 1 reads group g only
  * for keys j >= len - 1 - W_g, and len only grows, so a key older than W_g
  * positions is never read for that group again. Layout, per (b, hk): the

@@ -98,14 +98,13 @@ def test_decode_required_bytes_match_enumeration():
 
 
 def test_profiled_traffic_follows_the_source(tmp_path, monkeypatch):
-    import hashlib
     src = tmp_path / "kernel.cu"
     src.write_text("kernel v1\n")
-    h = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_digest("kernel.cu")
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "k.txt").write_text(
         f"# comment: with a colon\nsource_sha256_16: {h}\ndram_bytes_per_launch: 12345\n")
-    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic("k.txt", "kernel.cu") == 12345
     src.write_text("kernel v2\n")  # the kernel changed since the capture
     assert bench.profiled_traffic("k.txt", "kernel.cu") is None
@@ -130,4 +129,8 @@ def test_source_digest_covers_included_headers(tmp_path, monkeypatch):
     d1 = bench.source_digest("csrc/k.cu")
     assert d1 != d0
     (tmp_path / "include" / "api.h").write_text("api v2\n")
-    assert bench.source_digest("csrc/k.cu") not in (d0, d1)
+    d2 = bench.source_digest("csrc/k.cu")
+    assert d2 not in (d0, d1)
+    # comments and whitespace are not compiled: editing them keeps the digest
+    (tmp_path / "include" / "api.h").write_text("// a note\napi   v2 /* more\n notes */\n")
+    assert bench.source_digest("csrc/k.cu") == d2
