@@ -49,6 +49,27 @@ def test_decode_dense_and_zero_cutoffs():
         assert_attention_close(o, lse, ro, rl, f"decode cut={'dense' if cut is None else 'zero'}")
 
 
+def test_decode_large_logits():
+    """Logits spanning hundreds of base-2 units (q and K scaled by 8, older
+    keys scaled up to 3x more): within a split most exponentials underflow,
+    and the splits' maxima differ by far more than fp32's range, so the
+    combine's LSE merge carries the result. Lengths across several 1024-key
+    splits with ragged ends."""
+    g = torch.Generator().manual_seed(77)
+    B, Hq, Hkv, d, Lmax = 3, 8, 2, 128, 3500
+    lens = torch.tensor([3500, 2049, 700], dtype=torch.int32)
+    ramp = (1.0 + 2.0 * torch.arange(Lmax - 1, -1, -1, dtype=torch.float32) / Lmax).view(1, 1, Lmax, 1)
+    q = (8.0 * torch.randn(B, Hq, d, generator=g)).to(torch.bfloat16)
+    kc = (8.0 * ramp * torch.randn(B, Hkv, Lmax, d, generator=g)).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, Lmax, d, generator=g).to(torch.bfloat16)
+    _, wg = oracle.cutoffs(d, 1e4, oracle.HALF_SPLIT)
+    s2 = (widen(q)[0, 0] @ widen(kc)[0, 0].T) / np.sqrt(d) / np.log(2.0)
+    assert s2.max() - s2.min() > 240  # the case is what it claims
+    o, lse = _gpu_decode(q, kc, vc, lens, wg)
+    ro, rl = oracle.decode(widen(q), widen(kc), widen(vc), lens.numpy(), wg)
+    assert_attention_close(o, lse, ro, rl, "decode large logits")
+
+
 def test_decode_workload_full():
     """16 sequences, H32/8, d128, lengths U[16384, 32768], theta 1e6 half-split:
     the query is rotated on the GPU at position len-1, every row checked."""
