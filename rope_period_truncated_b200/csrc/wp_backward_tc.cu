@@ -20,11 +20,12 @@
 //            the sub-tile's group classes (a plan word beside the stage),
 //            four stages.
 //   warp 9   MMA issuer: S(u) = sum_g Q_g K_g^T (M128 N64 K16 per non-skipped
-//            group) and dP(u) = dO V^T into double-buffered TMEM, then, once
-//            the row warps have written dS(u) (bf16, over S's first 32
-//            columns), dQ[g0:g1] += dS K[g0:g1] for each run of consecutive
-//            full groups as M128 N16*(g1-g0) K16 products with dS read from
-//            TMEM and K read MN-major from the same swizzled group tiles.
+//            group) and dP(u) = dO V^T into the S/dP buffer of TMEM, then,
+//            once the row warps have written dS(u) (bf16) into one of the two
+//            operand buffers, dQ[g0:g1] += dS K[g0:g1] for each run of
+//            consecutive full groups as M128 N16*(g1-g0) K16 products with dS
+//            read from TMEM and K read MN-major from the same swizzled group
+//            tiles.
 //   warps 0-7 two threads per query row: warp w reads TMEM lanes 32 (w % 4)..
 //            and the sub-tile's columns 32 (w / 4) .. +31, and forms P and
 //            dS = P (dP - D) there in packed f32x2 arithmetic (no row
