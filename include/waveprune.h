@@ -360,10 +360,17 @@ int wp_decode_kl(const void *q, const void *kcache, int k_layout, const void *vc
  *       has one position, so the dims of a channel out of window are zeroed
  *       per key before the product; a group's K bytes are skipped beyond its
  *       largest channel cutoff.
+ *     WP_MODE_CHANNEL, cut_rows = H_q: cut is [H_q][d_h/2], row h the
+ *       channel cutoffs of query head h, the exact rule per head. The query
+ *       heads of a KV head share its K loads (a group's K bytes are skipped
+ *       beyond the largest cutoff of its channels over all heads) and each
+ *       head's product takes the K dims masked by its own row: one product
+ *       per query head instead of one per KV head.
  * Everything else as in wp_decode_kl. Errors: those of wp_decode_kl, and
  * WP_ERR_ARG (mode, layout or cut_rows out of range, NULL cut with
- * cut_rows = H_q), WP_ERR_UNSUPPORTED (channel mode with cut_rows = H_q;
- * H_q x d_h/16 above 1024).
+ * cut_rows = H_q, a negative cutoff), WP_ERR_UNSUPPORTED (grouped mode with
+ * H_q x d_h/16 above 1024; channel mode with cut_rows = H_q and H_q x d_h/2
+ * above 2048).
  */
 int wp_decode_ex(const void *q, const void *kcache, int k_layout, const void *vcache, const int32_t *lens, int Lmax,
                  int B, int H_q, int H_kv, int d_h, int mode, const int32_t *cut, int cut_rows, int layout,

@@ -435,9 +435,30 @@ int wp_decode_ex(const void *q, const void *kcache, int k_layout, const void *vc
   if (mode == WP_MODE_GROUPED && cut_rows == 1)
     return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, cut, softmax_scale, o, lse,
                          workspace, ws_bytes, nullptr, 0, 0, 0, stream);
-  if (mode == WP_MODE_CHANNEL && cut_rows != 1) return WP_ERR_UNSUPPORTED;  // per-head exact tables: not built
+  if (mode == WP_MODE_CHANNEL && cut_rows != 1 && static_cast<int64_t>(H_q) * C > DECODE_HEAD_CHAN_CAP)
+    return WP_ERR_UNSUPPORTED;
   DecodeTables tables;
   int32_t load_cut[8];
+  if (mode == WP_MODE_CHANNEL && cut_rows != 1) {
+    // exact rule, one channel row per query head: a group's K loads follow the
+    // largest cutoff of its channels over all heads
+    for (int e = 0; e < H_q * C; ++e) {
+      if (cut[e] < 0) return WP_ERR_ARG;
+      tables.head_chan_cut[e] = cut[e];
+    }
+    for (int g = 0; g < G; ++g) {
+      int32_t m = 0;
+      for (int h = 0; h < H_q; ++h)
+        for (int k = 16 * g; k < 16 * g + 16; ++k) {
+          const int c = layout == WP_ROPE_INTERLEAVED ? k / 2 : k % C;
+          m = tables.head_chan_cut[h * C + c] > m ? tables.head_chan_cut[h * C + c] : m;
+        }
+      load_cut[g] = m;
+    }
+    return decode_launch(q, kcache, k_layout, vcache, lens, Lmax, B, H_q, H_kv, d_h, load_cut, softmax_scale, o,
+                         lse, workspace, ws_bytes, nullptr, 0, 0, 0, stream, DECODE_MASK_CHANNEL_PER_HEAD, layout,
+                         &tables);
+  }
   if (mode == WP_MODE_GROUPED) {
     if (static_cast<int64_t>(H_q) * G > 1024) return WP_ERR_UNSUPPORTED;
     // the K loads cover the union of the heads' windows

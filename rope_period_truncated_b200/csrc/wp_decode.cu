@@ -151,6 +151,10 @@ __global__ void __launch_bounds__(DEC_THREADS)
       mcut[e] = (e % 8) < D / 16 ? tabs.head_cut[(hq0 + e / 8) * (D / 16) + e % 8] : WP_CUTOFF_INF;
   } else if constexpr (MASK == DECODE_MASK_CHANNEL) {
     for (int e = threadIdx.x; e < D / 2; e += DEC_THREADS) mcut[e] = tabs.chan_cut[e];
+  } else if constexpr (MASK == DECODE_MASK_CHANNEL_PER_HEAD) {
+    // the channel rows of the KV head's R query heads, row r at mcut + r * D / 2
+    for (int e = threadIdx.x; e < R * (D / 2); e += DEC_THREADS)
+      mcut[e] = tabs.head_chan_cut[(hq0 + e / (D / 2)) * (D / 2) + e % (D / 2)];
   }
   if constexpr (MASK != DECODE_MASK_GROUP_SHARED) __syncthreads();
 
@@ -292,7 +296,28 @@ __global__ void __launch_bounds__(DEC_THREADS)
         b10 = mask_channels<D>(b10, 16 * c + 2 * t, d1, mcut, a.layout);
         b11 = mask_channels<D>(b11, 16 * c + 8 + 2 * t, d1, mcut, a.layout);
       }
-      if constexpr (MASK == DECODE_MASK_GROUP_PER_HEAD) {
+      if constexpr (MASK == DECODE_MASK_CHANNEL_PER_HEAD) {
+        // one product per query head r, with the shared K fragments masked by
+        // head r's channel row; lanes of row g keep head g's product
+        const int64_t d0 = qpos - (kb0 + g), d1 = d0 - 8;
+#pragma unroll 1
+        for (int r = 0; r < R; ++r) {
+          const int32_t *hc = mcut + r * (D / 2);
+          const uint32_t m00 = mask_channels<D>(b00, 16 * c + 2 * t, d0, hc, a.layout);
+          const uint32_t m01 = mask_channels<D>(b01, 16 * c + 8 + 2 * t, d0, hc, a.layout);
+          const uint32_t m10 = mask_channels<D>(b10, 16 * c + 2 * t, d1, hc, a.layout);
+          const uint32_t m11 = mask_channels<D>(b11, 16 * c + 8 + 2 * t, d1, hc, a.layout);
+          float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_16816(t0, qa[c][0], 0u, qa[c][1], 0u, m00, m01);
+          mma_16816(t1, qa[c][0], 0u, qa[c][1], 0u, m10, m11);
+          if (g == r) {
+            s0[0] += t0[0];
+            s0[1] += t0[1];
+            s1[0] += t1[0];
+            s1[1] += t1[1];
+          }
+        }
+      } else if constexpr (MASK == DECODE_MASK_GROUP_PER_HEAD) {
         // this group's products apart, then kept per head (row g) and key
         float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
         mma_16816(t0, qa[c][0], 0u, qa[c][1], 0u, b00, b01);
@@ -413,7 +438,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeArgs a) {
 
 template <int D, int R, bool KGM, bool PAGED, int MASK>
 cudaError_t launch_split_l(const DecodeArgs &a, const DecodeTables *tables, cudaStream_t stream) {
-  const uint32_t smem = DecLayout<D>::BYTES + (MASK == DECODE_MASK_GROUP_SHARED ? 0u : 256u);
+  const uint32_t smem = DecLayout<D>::BYTES + (MASK == DECODE_MASK_GROUP_SHARED         ? 0u
+                                               : MASK == DECODE_MASK_CHANNEL_PER_HEAD ? R * (D / 2) * 4u
+                                                                                      : 256u);
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, R, KGM, PAGED, MASK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -435,6 +462,9 @@ cudaError_t launch_split(const DecodeArgs &a, const DecodeTables *tables, cudaSt
   if (a.mask == DECODE_MASK_CHANNEL)
     return a.k_group_major ? launch_split_l<D, R, true, false, DECODE_MASK_CHANNEL>(a, tables, stream)
                            : launch_split_l<D, R, false, false, DECODE_MASK_CHANNEL>(a, tables, stream);
+  if (a.mask == DECODE_MASK_CHANNEL_PER_HEAD)
+    return a.k_group_major ? launch_split_l<D, R, true, false, DECODE_MASK_CHANNEL_PER_HEAD>(a, tables, stream)
+                           : launch_split_l<D, R, false, false, DECODE_MASK_CHANNEL_PER_HEAD>(a, tables, stream);
   if (a.block_table != nullptr)
     return a.k_group_major ? launch_split_l<D, R, true, true, 0>(a, tables, stream)
                            : launch_split_l<D, R, false, true, 0>(a, tables, stream);

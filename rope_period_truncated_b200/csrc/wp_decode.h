@@ -39,13 +39,24 @@ struct DecodeArgs {
 // query head h takes row h of a per-head table (the loads cover the union of
 // the heads' windows and each head's scores are masked group by group).
 // CHANNEL: the exact per-channel rule (one query position per sequence, so a
-// channel's K dims are zeroed per key before the product).
-enum : int { DECODE_MASK_GROUP_SHARED = 0, DECODE_MASK_GROUP_PER_HEAD = 1, DECODE_MASK_CHANNEL = 2 };
+// channel's K dims are zeroed per key before the product). CHANNEL_PER_HEAD:
+// the exact rule with one channel table per query head; the heads of a KV
+// head share the K fragments, so each head's product takes the fragments
+// masked by its own table (R products instead of one).
+enum : int {
+  DECODE_MASK_GROUP_SHARED = 0,
+  DECODE_MASK_GROUP_PER_HEAD = 1,
+  DECODE_MASK_CHANNEL = 2,
+  DECODE_MASK_CHANNEL_PER_HEAD = 3
+};
+
+constexpr int DECODE_HEAD_CHAN_CAP = 2048;  // entries of the per-head channel table (H_q x D/2)
 
 // Cutoff tables of the masked decode modes, a kernel parameter of their own.
 struct DecodeTables {
-  int32_t head_cut[1024];  // [Hq][D/16] (GROUP_PER_HEAD)
-  int32_t chan_cut[64];    // [D/2] (CHANNEL)
+  int32_t head_cut[1024];                         // [Hq][D/16] (GROUP_PER_HEAD)
+  int32_t chan_cut[64];                           // [D/2] (CHANNEL)
+  int32_t head_chan_cut[DECODE_HEAD_CHAN_CAP];  // [Hq][D/2] (CHANNEL_PER_HEAD)
 };
 
 // Scratch layout: o_part first, then lse_part at a 256-byte boundary.

@@ -175,6 +175,26 @@ def test_decode_kl_and_kcache_conversion_reject_bad_arguments(lib):
     assert g(FAKE, FAKE + 4096, 1, 2, 100, 80, None) == wp.WP_ERR_UNSUPPORTED
 
 
+def test_decode_ex_per_head_channel_tables_checked(lib):
+    """Exact rule with one channel row per query head: a NULL table, a
+    negative cutoff and a table beyond the kernel parameter's 2048 entries
+    are refused on the host, before any launch."""
+    f = lib.wp_decode_ex
+    ws = lib.wp_decode_workspace_bytes(2, 8, 128, 4096)
+
+    def call(Hq, Hkv, cut):
+        cp = None if cut is None else cut.ctypes.data_as(ctypes.c_void_p)
+        return f(FAKE, FAKE, wp.KCACHE_ROWS, FAKE, FAKE, 4096, 2, Hq, Hkv, 128, wp.MODE_CHANNEL, cp, Hq,
+                 wp.ROPE_HALF_SPLIT, ctypes.c_float(0.0), FAKE, None, FAKE, ws, None)
+
+    assert call(8, 2, None) == wp.WP_ERR_ARG
+    bad = np.full((8, 64), 100, dtype=np.int32)
+    bad[5, 17] = -1
+    assert call(8, 2, bad) == wp.WP_ERR_ARG
+    big = np.full((64, 64), 100, dtype=np.int32)  # 64 heads x 64 channels = 4096 entries
+    assert call(64, 8, big) == wp.WP_ERR_UNSUPPORTED
+
+
 def test_decode_paged_rejects_bad_arguments(lib):
     f = lib.wp_decode_paged
     ws = lib.wp_decode_workspace_bytes(2, 8, 128, 64 * 64)

@@ -327,3 +327,32 @@ def test_decode_exact_channel_mode(layout, group_major, table):
     ro, rl = oracle.attention_rows(widen(q).reshape(B * Hq, d), (rb, rh, ri), widen(kc).transpose(0, 2, 1, 3),
                                    widen(vc).transpose(0, 2, 1, 3), Hq, wc, oracle.MODE_CHANNEL, layout)
     assert_attention_close(o, lse, ro.reshape(B, Hq, d), rl.reshape(B, Hq), f"exact decode layout={layout}")
+
+
+@pytest.mark.parametrize("layout", [wp.ROPE_INTERLEAVED, wp.ROPE_HALF_SPLIT])
+@pytest.mark.parametrize("group_major", [False, True])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (8, 1), (4, 4)])
+def test_decode_exact_per_head_tables(layout, group_major, Hq, Hkv):
+    """Exact per-channel rule with one channel row per query head
+    (wp_decode_ex, channel mode, cut_rows = H_q): the heads of a KV head
+    share its K loads, each head's product takes K masked by its own row.
+    Oracle: channel-mode row len-1 one head at a time."""
+    B, d, Lmax = 3, 128, 2600
+    lens = torch.tensor([2600, 700, 1], dtype=torch.int32)
+    q, kc, vc = _decode_inputs(91 + layout + Hq + Hkv, B, Hq, Hkv, d, Lmax)
+    rng = np.random.default_rng(Hq * 3 + Hkv + layout)
+    cut = rng.integers(0, 2000, size=(Hq, d // 2)).astype(np.int32)
+    cut[1] = 2 ** 31 - 1  # a dense head next to pruned ones
+    kcd = wp.wp_kcache_group_major(kc.cuda()) if group_major else kc.cuda()
+    o, lse = wp.wp_decode(q.cuda(), kcd, vc.cuda(), lens.cuda(), cut, mode=wp.MODE_CHANNEL, layout=layout)
+    torch.cuda.synchronize()
+    assert wp.wp_device_status() == 0
+    kr, vr = widen(kc).transpose(0, 2, 1, 3), widen(vc).transpose(0, 2, 1, 3)
+    ri = lens.numpy().astype(np.int64) - 1
+    ro = np.zeros((B, Hq, d))
+    rl = np.zeros((B, Hq))
+    for h in range(Hq):
+        a, b_ = oracle.attention_rows(widen(q)[:, h], (np.arange(B), np.full(B, h), ri), kr, vr, Hq, cut[h],
+                                      oracle.MODE_CHANNEL, layout)
+        ro[:, h], rl[:, h] = a.reshape(B, d), b_.reshape(B)
+    assert_attention_close(o, lse, ro, rl, f"exact per-head decode Hq={Hq} Hkv={Hkv} gm={group_major}")
