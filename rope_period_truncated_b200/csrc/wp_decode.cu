@@ -24,6 +24,12 @@
 // (scores Q.K^T and P.V, fp32 accumulation); the online softmax keeps the row
 // max and row sum with warp shuffles. The 4 warps merge their states in
 // shared memory and write one partial (O normalised, LSE base 2) per split.
+// Masked modes (the MASK template parameter): one group table per query head
+// (the loads cover the union of the heads' windows; each head keeps a group's
+// product per key only inside its own window), the exact per-channel rule of
+// Eq. (6) (a channel's K dims zeroed per key before the product, the query
+// having one position), and the exact rule with one channel table per query
+// head (one product per query head on the K fragments masked by its row).
 // Combine kernel: per (sequence, query head) merge the splits by LSE.
 #include <cuda_bf16.h>
 #include <cstdint>
