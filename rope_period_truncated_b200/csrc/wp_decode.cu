@@ -163,6 +163,19 @@ __global__ void __launch_bounds__(DEC_THREADS)
       mcut[e] = tabs.head_chan_cut[(hq0 + e / (D / 2)) * (D / 2) + e % (D / 2)];
   }
   if constexpr (MASK != DECODE_MASK_GROUP_SHARED) __syncthreads();
+  // exact rule: the cutoffs of the channels that own this lane's B-fragment
+  // dims (16c + 2t, +1, 16c + 8 + 2t, +1 of every k-step c), held in registers
+  int32_t lcut[MASK == DECODE_MASK_CHANNEL ? KSTEPS : 1][4];
+  if constexpr (MASK == DECODE_MASK_CHANNEL) {
+#pragma unroll
+    for (int c = 0; c < KSTEPS; ++c) {
+      const int k0 = 16 * c + 2 * t, k1 = k0 + 8;
+      lcut[c][0] = mcut[a.layout == WP_ROPE_INTERLEAVED ? k0 >> 1 : k0 % (D / 2)];
+      lcut[c][1] = mcut[a.layout == WP_ROPE_INTERLEAVED ? k0 >> 1 : (k0 + 1) % (D / 2)];
+      lcut[c][2] = mcut[a.layout == WP_ROPE_INTERLEAVED ? k1 >> 1 : k1 % (D / 2)];
+      lcut[c][3] = mcut[a.layout == WP_ROPE_INTERLEAVED ? k1 >> 1 : (k1 + 1) % (D / 2)];
+    }
+  }
 
   // Q as the A operand (rows = query heads; rows >= R and 8..15 are zero).
   uint32_t qa[KSTEPS][2];
@@ -295,12 +308,13 @@ __global__ void __launch_bounds__(DEC_THREADS)
       uint32_t b00, b01, b10, b11;
       ldsm_x4(ks + piece_off<D>(rr, pp), b00, b01, b10, b11);
       if constexpr (MASK == DECODE_MASK_CHANNEL) {
-        // b00/b01: key g, dims 16c + 2t (+1) and 16c + 8 + 2t (+1); b10/b11: key 8 + g
-        const int64_t d0 = qpos - (kb0 + g), d1 = d0 - 8;
-        b00 = mask_channels<D>(b00, 16 * c + 2 * t, d0, mcut, a.layout);
-        b01 = mask_channels<D>(b01, 16 * c + 8 + 2 * t, d0, mcut, a.layout);
-        b10 = mask_channels<D>(b10, 16 * c + 2 * t, d1, mcut, a.layout);
-        b11 = mask_channels<D>(b11, 16 * c + 8 + 2 * t, d1, mcut, a.layout);
+        // b00/b01: key g, dims 16c + 2t (+1) and 16c + 8 + 2t (+1); b10/b11: key 8 + g.
+        // Distances fit 32 bits (Lmax < 2^31).
+        const int d0 = static_cast<int>(qpos - (kb0 + g)), d1 = d0 - 8;
+        b00 &= (d0 <= lcut[c][0] ? 0x0000ffffu : 0u) | (d0 <= lcut[c][1] ? 0xffff0000u : 0u);
+        b01 &= (d0 <= lcut[c][2] ? 0x0000ffffu : 0u) | (d0 <= lcut[c][3] ? 0xffff0000u : 0u);
+        b10 &= (d1 <= lcut[c][0] ? 0x0000ffffu : 0u) | (d1 <= lcut[c][1] ? 0xffff0000u : 0u);
+        b11 &= (d1 <= lcut[c][2] ? 0x0000ffffu : 0u) | (d1 <= lcut[c][3] ? 0xffff0000u : 0u);
       }
       if constexpr (MASK == DECODE_MASK_CHANNEL_PER_HEAD) {
         // one product per query head r, with the shared K fragments masked by
